@@ -1,0 +1,188 @@
+"""Seeded synthetic inputs: audio clips and random-init encoder weights.
+
+This module is the only code that both the CUDA path and the fp64 oracle consume. It
+holds input recipes only (random draws, a one-pole lowpass, tone bursts, bf16 rounding
+of the weights) and none of the encoder's own arithmetic.
+
+Audio recipes (the pages publish no audio; these stand in for the clip lengths they
+discuss: 30 s chunks, 10-minute and one-hour recordings):
+
+* ``tones``: 0.5 sin(2 pi 440 t) + 0.2 sin(2 pi 1000 t) + N(0, 0.01^2).
+* ``bursts``: white N(0, 0.1^2) through y[n] = 0.95 y[n-1] + 0.05 w[n], plus 20 tone
+  bursts (frequency U(100, 4000) Hz, amplitude U(0.05, 0.3), length U(0.1, 1.0) s,
+  start U(0, D - length), Hann-tapered), optionally multiplied by the 4 Hz envelope
+  0.55 + 0.45 sin(2 pi 4 t).
+
+Weights: every matrix and bias N(0, 0.02); LayerNorm and QK-norm gains 1 + N(0, 0.02);
+LayerNorm betas N(0, 0.02). Drawn in float64 with one PCG64 stream per tensor, rounded
+once to bf16 (round to nearest even), and returned both as bf16 bit patterns (uint16)
+and as the float32 values those bits encode.
+"""
+from __future__ import annotations
+
+from dataclasses import dataclass
+
+import numpy as np
+from scipy.signal import lfilter
+
+SAMPLE_RATE = 16000
+
+
+# ----------------------------------------------------------------------------- audio
+
+def tones_clip(n_samples: int = 16000, seed: int = 0) -> np.ndarray:
+    rng = np.random.default_rng(seed)
+    t = np.arange(n_samples, dtype=np.float64) / SAMPLE_RATE
+    x = 0.5 * np.sin(2 * np.pi * 440.0 * t) + 0.2 * np.sin(2 * np.pi * 1000.0 * t)
+    x += rng.normal(0.0, 0.01, n_samples)
+    return x.astype(np.float32)
+
+
+def bursts_clip(n_samples: int, seed: int, envelope: bool = False,
+                n_bursts: int = 20) -> np.ndarray:
+    rng = np.random.default_rng(seed)
+    w = rng.normal(0.0, 0.1, n_samples)
+    x = lfilter([0.05], [1.0, -0.95], w)
+    dur = n_samples / SAMPLE_RATE
+    for _ in range(n_bursts):
+        f = rng.uniform(100.0, 4000.0)
+        amp = rng.uniform(0.05, 0.3)
+        length = min(rng.uniform(0.1, 1.0), dur)
+        start = rng.uniform(0.0, dur - length)
+        i0 = int(start * SAMPLE_RATE)
+        n = min(int(length * SAMPLE_RATE), n_samples - i0)
+        if n <= 1:
+            continue
+        k = np.arange(n, dtype=np.float64)
+        taper = 0.5 - 0.5 * np.cos(2 * np.pi * k / (n - 1))
+        x[i0:i0 + n] += amp * taper * np.sin(2 * np.pi * f * k / SAMPLE_RATE)
+    if envelope:
+        t = np.arange(n_samples, dtype=np.float64) / SAMPLE_RATE
+        x *= 0.55 + 0.45 * np.sin(2 * np.pi * 4.0 * t)
+    return x.astype(np.float32)
+
+
+@dataclass(frozen=True)
+class Workload:
+    name: str
+    batch: int
+    n_samples: int
+    n_layers: int
+    kind: str          # "tones" | "bursts" | "bursts_env"
+    seed: int
+
+    @property
+    def audio_seconds(self) -> float:
+        return self.batch * self.n_samples / SAMPLE_RATE
+
+    def audio(self) -> np.ndarray:
+        """[batch, n_samples] float32, one seed per clip (seed + clip index)."""
+        out = np.empty((self.batch, self.n_samples), dtype=np.float32)
+        for b in range(self.batch):
+            if self.kind == "tones":
+                out[b] = tones_clip(self.n_samples, self.seed + b)
+            else:
+                out[b] = bursts_clip(self.n_samples, self.seed + b,
+                                     envelope=(self.kind == "bursts_env"))
+        return out
+
+
+# The five workloads: a 1 s tone clip (2 layers), a 30 s clip, 16 x 60 s clips, a
+# 10-minute recording and a one-hour recording (32 layers each).
+WORKLOADS = {
+    "tones_1s": Workload("tones_1s", 1, 16_000, 2, "tones", 0),
+    "clip_30s": Workload("clip_30s", 1, 480_000, 32, "bursts", 1),
+    "batch16_60s": Workload("batch16_60s", 16, 960_000, 32, "bursts", 100),
+    "rec_10min": Workload("rec_10min", 1, 9_600_000, 32, "bursts_env", 2),
+    "rec_1h": Workload("rec_1h", 1, 57_600_000, 32, "bursts_env", 3),
+}
+WORKLOAD_ORDER = ["tones_1s", "clip_30s", "batch16_60s", "rec_10min", "rec_1h"]
+
+
+# ----------------------------------------------------------------------------- weights
+
+def bf16_bits(x: np.ndarray) -> np.ndarray:
+    """Round float64/float32 values to bf16 (nearest even); return the uint16 bit patterns."""
+    f = np.asarray(x, dtype=np.float32)
+    u = f.view(np.uint32).astype(np.uint64)
+    rounded = (u + 0x7FFF + ((u >> 16) & 1)) >> 16
+    return rounded.astype(np.uint16)
+
+
+def bf16_to_f32(bits: np.ndarray) -> np.ndarray:
+    return (np.asarray(bits, dtype=np.uint16).astype(np.uint32) << 16).view(np.float32)
+
+
+LAYER_TENSORS = [
+    # name, shape (as a function of width W, ffn Fd, head dim hd), init kind
+    ("ln1_g", lambda W, Fd, hd: (W,), "gain"),
+    ("ln1_b", lambda W, Fd, hd: (W,), "normal"),
+    ("w_qkv", lambda W, Fd, hd: (3 * W, W), "normal"),
+    ("b_qkv", lambda W, Fd, hd: (3 * W,), "normal"),
+    ("qn_g", lambda W, Fd, hd: (hd,), "gain"),
+    ("kn_g", lambda W, Fd, hd: (hd,), "gain"),
+    ("w_o", lambda W, Fd, hd: (W, W), "normal"),
+    ("b_o", lambda W, Fd, hd: (W,), "normal"),
+    ("ln2_g", lambda W, Fd, hd: (W,), "gain"),
+    ("ln2_b", lambda W, Fd, hd: (W,), "normal"),
+    ("w1", lambda W, Fd, hd: (Fd, W), "normal"),
+    ("b1", lambda W, Fd, hd: (Fd,), "normal"),
+    ("w2", lambda W, Fd, hd: (W, Fd), "normal"),
+    ("b2", lambda W, Fd, hd: (W,), "normal"),
+]
+GLOBAL_TENSORS = [
+    ("w_proj", lambda W, S: (W, S), "normal"),
+    ("b_proj", lambda W, S: (W,), "normal"),
+    ("lnf_g", lambda W, S: (W,), "gain"),
+    ("lnf_b", lambda W, S: (W,), "normal"),
+]
+
+
+def _draw(shape, kind: str, seed: int, std: float, gain_std: float) -> np.ndarray:
+    rng = np.random.default_rng(seed)
+    z = rng.standard_normal(shape)
+    if kind == "gain":
+        return 1.0 + gain_std * z
+    return std * z
+
+
+def make_weights(n_layers: int, seed: int = 1000, width: int = 1280, ffn: int = 5120,
+                 head_dim: int = 128, stack_in: int = 1024, std: float = 0.02,
+                 gain_std: float = 0.02, qk_gain_scale: float = 1.0) -> dict:
+    """Random-init weights, bf16-rounded. Returns a nested dict of
+
+    ``{"w_proj": (bits, f32), ..., "layers": [{"ln1_g": (bits, f32), ...}, ...]}``.
+    Tensor i of the flat order (globals first, then layer by layer) uses seed + i.
+    ``qk_gain_scale`` multiplies the q/k norm gains (a sharp-attention test case).
+    """
+    out: dict = {"layers": []}
+    idx = 0
+    for name, shp, kind in GLOBAL_TENSORS:
+        v = _draw(shp(width, stack_in), kind, seed + idx, std, gain_std)
+        b = bf16_bits(v)
+        out[name] = (b, bf16_to_f32(b))
+        idx += 1
+    for _ in range(n_layers):
+        lw = {}
+        for name, shp, kind in LAYER_TENSORS:
+            v = _draw(shp(width, ffn, head_dim), kind, seed + idx, std, gain_std)
+            if name in ("qn_g", "kn_g"):
+                v = v * qk_gain_scale
+            b = bf16_bits(v)
+            lw[name] = (b, bf16_to_f32(b))
+            idx += 1
+        out["layers"].append(lw)
+    return out
+
+
+def weights_f32(w: dict) -> dict:
+    """The float32 values of :func:`make_weights` output, in the same nesting."""
+    out = {k: v[1] for k, v in w.items() if k != "layers"}
+    out["layers"] = [{k: v[1] for k, v in lw.items()} for lw in w["layers"]]
+    return out
+
+
+def random_bf16(shape, seed: int, std: float = 1.0):
+    """N(0, std^2) values rounded to bf16: (bits, float32 values)."""
+    b = bf16_bits(np.random.default_rng(seed).normal(0.0, std, shape))
+    return b, bf16_to_f32(b)
