@@ -1,0 +1,184 @@
+/*
+ * sal.h - C-ABI of libsal: the speech front end and ASR encoder of Nemotron 3.5
+ * Transcribe on one NVIDIA B200 (sm_100a).
+ *
+ * What the library computes is fixed by the page "Nemotron 3.5 Transcribe: From
+ * Recorded Speech to Dataset Audits" (flozi.net), section "How audio and speakers
+ * reach the language model", paragraph on the exported frontend: 16 kHz mono audio,
+ * 128 log-mel features from a 25 ms Hann window, a 512-point FFT and a 10 ms hop;
+ * eight successive frames stacked and projected to width 1,280; 32 Transformer layers
+ * with ten heads, QK normalisation, feed-forward expansion four and rotary position
+ * embeddings; 12.5 embeddings per second of audio. Where that paragraph is silent the
+ * library takes these readings:
+ *   frames F = N < 400 ? 0 : 1 + (N - 400) / 160, positions T = F / 8 (integer division,
+ *   no padding, remainder frames dropped); periodic Hann; power spectrum |X_k|^2;
+ *   Slaney mel filters over 0..8 kHz with Slaney area normalisation; natural log with a
+ *   clamp at 1e-10; frame-major stacking S[t][128 j + m] = M[8 t + j][m]; pre-norm
+ *   LayerNorm (eps 1e-5) with a final LayerNorm; RMS QK-norm over head_dim 128
+ *   (eps 1e-6, one gain vector for q and one for k, shared by heads) before RoPE;
+ *   rotate-half RoPE, base 10000, positions 0..T-1 per clip; full bidirectional
+ *   softmax attention scaled by 1/sqrt(128); exact-erf GELU; two-matrix FFN 1280 ->
+ *   5120 -> 1280; every linear layer has a bias.
+ *
+ * Conventions for every call:
+ *   - Pointers are DEVICE pointers unless a call says otherwise. The caller owns every
+ *     buffer and keeps it alive until the stream has passed the call.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = the legacy default stream).
+ *     Calls are asynchronous: they validate arguments on the host, enqueue kernels and
+ *     return.
+ *   - Errors come back as a sal_status code; nothing is thrown across the ABI. A
+ *     bounded device-side wait that gave up is reported by sal_last_device_status().
+ *   - Every pointer must be 16-byte aligned (SAL_EINVAL otherwise); a clip batch is
+ *     `batch` clips of equal length stored back to back.
+ *   - bf16 tensors are IEEE bfloat16 bit patterns (uint16_t); parameters are bf16.
+ *   - T > 45000 (more than one hour of audio per clip) is SAL_ESHAPE; N < 400 samples
+ *     or T = 0 is a valid empty problem that launches nothing and returns SAL_OK.
+ *   - The library allocates no device memory. Scratch space is the caller's
+ *     `workspace`; sal_encoder_workspace_bytes() gives its size.
+ *   - Thread safety: calls on different streams may run concurrently.
+ */
+#ifndef SAL_H_
+#define SAL_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    SAL_OK = 0,
+    SAL_EINVAL = 1,     /* null or misaligned pointer, bad enum value, bad count */
+    SAL_ESHAPE = 2,     /* a size outside what the library supports */
+    SAL_EWORKSPACE = 3, /* workspace smaller than sal_encoder_workspace_bytes() */
+    SAL_ECUDA = 4,      /* a CUDA runtime call or kernel launch failed */
+    SAL_ETIMEOUT = 5,   /* a bounded device wait gave up (see sal_last_device_status) */
+    SAL_EDEVICE = 6     /* the current device is not a B200-class sm_100 GPU */
+} sal_status;
+
+#define SAL_N_MELS 128
+#define SAL_STACK 8
+#define SAL_STACK_DIM 1024
+#define SAL_WIDTH 1280
+#define SAL_HEADS 10
+#define SAL_HEAD_DIM 128
+#define SAL_FFN 5120
+#define SAL_MAX_POSITIONS 45000
+
+/* Frames of a clip of n_samples samples: n < 400 ? 0 : 1 + (n - 400) / 160.
+ * (Exported-frontend paragraph: 25 ms window, 10 ms hop at 16 kHz.) */
+int64_t sal_frame_count(int64_t n_samples);
+
+/* Encoder positions: sal_frame_count(n) / 8 (eight stacked frames per position,
+ * 12.5 per second). */
+int64_t sal_position_count(int64_t n_samples);
+
+/* Static English text for a status code. Never NULL. */
+const char* sal_status_string(int status);
+
+/* Per-layer parameters, all DEVICE pointers to bf16 arrays (row-major, [out, in]):
+ *   ln1_g, ln1_b [1280]      pre-attention LayerNorm gain and bias
+ *   w_qkv [3840, 1280]       rows 0..1279 = q, 1280..2559 = k, 2560..3839 = v; head h of
+ *   b_qkv [3840]             each uses rows 128 h .. 128 h + 127 of its block
+ *   qn_g, kn_g [128]         RMS QK-norm gains (shared by the ten heads)
+ *   w_o [1280, 1280], b_o [1280]     attention output projection
+ *   ln2_g, ln2_b [1280]      pre-FFN LayerNorm
+ *   w1 [5120, 1280], b1 [5120]       FFN up (GELU)
+ *   w2 [1280, 5120], b2 [1280]       FFN down
+ * Weight matrices must be 16-byte aligned (they are read by TMA). */
+typedef struct {
+    const void *ln1_g, *ln1_b, *w_qkv, *b_qkv, *qn_g, *kn_g, *w_o, *b_o;
+    const void *ln2_g, *ln2_b, *w1, *b1, *w2, *b2;
+} sal_layer;
+
+/* Whole-encoder parameters. w_proj [1280, 1024] and b_proj [1280] are the stack
+ * projection; lnf_g, lnf_b [1280] the final LayerNorm; `layers` is a HOST array of
+ * n_layers sal_layer records (read during the call only). */
+typedef struct {
+    const void *w_proj, *b_proj;
+    const sal_layer* layers;
+    int n_layers;
+    const void *lnf_g, *lnf_b;
+} sal_weights;
+
+/* Front end: wave [batch, n_samples] float32 at 16 kHz ->
+ *   logmel  [batch, F, 128] float32, natural-log mel energies (required), and
+ *   stacked [batch, T, 1024] bf16, the frame-major stack of the first 8 T frames
+ *           (the projection's input; may be NULL).
+ * One kernel: framing, Hann window, 512-point real FFT, power, 128 Slaney mel filters,
+ * log and the bf16 stacked copy. */
+sal_status sal_frontend(const float* wave, int64_t n_samples, int batch, float* logmel,
+                        void* stacked, void* stream);
+
+/* Stack projection x0 = S P^T + p: stacked [batch * T, 1024] bf16 ->
+ * x [batch * T, 1280] float32 (the encoder's residual stream). */
+sal_status sal_stack_project(const void* stacked, int batch, int64_t T, const sal_weights* w,
+                             float* x, void* stream);
+
+/* Bytes of scratch that sal_encoder_forward needs for `batch` clips of T positions. */
+size_t sal_encoder_workspace_bytes(int batch, int64_t T);
+
+/* Encoder: x [batch * T, 1280] float32 holds x0 on entry and the residual stream after
+ * n_layers layers on return (clobbered); emb [batch * T, 1280] bf16 receives the final
+ * LayerNorm of it. n_layers may be 0..w->n_layers. Positions restart at 0 in each clip
+ * and attention never crosses clips. `workspace` is device scratch of ws_bytes >=
+ * sal_encoder_workspace_bytes(batch, T), 256-byte aligned. */
+sal_status sal_encoder_forward(float* x, int batch, int64_t T, const sal_weights* w, int n_layers,
+                               void* emb, void* workspace, size_t ws_bytes, void* stream);
+
+/* Whole path: wave -> log-mel -> stack -> projection -> n_layers layers -> final LN.
+ * `wave` [batch, n_samples] float32 and `emb` [batch, T, 1280] bf16 may each be HOST or
+ * DEVICE memory (host buffers are copied through the workspace on `stream`; pinned host
+ * memory makes the copies asynchronous). `workspace` must hold
+ * sal_encode_workspace_bytes(batch, n_samples) bytes of device memory. */
+size_t sal_encode_workspace_bytes(int batch, int64_t n_samples);
+sal_status sal_encode(const float* wave, int64_t n_samples, int batch, const sal_weights* w,
+                      int n_layers, void* emb, void* workspace, size_t ws_bytes, void* stream);
+
+/* Synchronises `stream` and reports (then clears) the device status word that bounded
+ * waits set when they give up: SAL_OK or SAL_ETIMEOUT. */
+sal_status sal_last_device_status(void* stream);
+
+/* Upper bound in nanoseconds of every mbarrier wait inside the kernels (default 4e9).
+ * A wait that exceeds it sets the device status word and the kernel returns early. */
+void sal_set_wait_limit_ns(uint64_t ns);
+
+/* ---------------------------------------------------------------------------------
+ * Single-step entry points (the stages sal_encoder_forward chains; for tests and
+ * per-kernel timing). Layouts as above; M = batch * T rows.
+ * --------------------------------------------------------------------------------- */
+
+/* y = LayerNorm(x) * g + b over rows of 1280 (eps 1e-5): x float32 -> y bf16. */
+sal_status sal_layernorm(const float* x, int64_t rows, const void* g, const void* b, void* y,
+                         void* stream);
+
+typedef enum {
+    SAL_EPI_STORE_F32 = 0,  /* out f32 [M, N] = A W^T + bias                 */
+    SAL_EPI_STORE_BF16 = 1, /* out bf16 [M, N] = A W^T + bias                */
+    SAL_EPI_GELU_BF16 = 2,  /* out bf16 [M, N] = GELU_erf(A W^T + bias)      */
+    SAL_EPI_RESID_F32 = 3   /* out f32 [M, N] += A W^T + bias (residual add) */
+} sal_epilogue;
+
+/* Linear layer on the tensor cores: A [M, K] bf16 (row-major), W [N, K] bf16, bias [N]
+ * bf16. K must be a multiple of 64 and N of 64 (N of 128 when M > 512). */
+sal_status sal_linear(int epilogue, const void* A, int64_t M, int K, const void* W, int N,
+                      const void* bias, void* out, void* stream);
+
+/* QKV projection with the QK-norm and RoPE epilogue: h [batch * T, 1280] bf16 ->
+ * q, k, v [batch, 10, T, 128] bf16 (q and k RMS-normalised with qn_g / kn_g, then
+ * rotated by RoPE at position t of their clip). rope_cs is device scratch of
+ * 2 * T * 64 float32 that the call fills with the rotation table. */
+sal_status sal_qkv_rope(const void* h, int batch, int64_t T, const sal_layer* layer, void* q,
+                        void* k, void* v, float* rope_cs, void* stream);
+
+/* Bidirectional attention per (clip, head): q, k, v [batch, 10, T, 128] bf16 ->
+ * o [batch * T, 1280] bf16, o[b*T + t][128 h + d] = softmax(q k^T / sqrt(128)) v. */
+sal_status sal_attention(const void* q, const void* k, const void* v, int batch, int64_t T,
+                         void* o, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SAL_H_ */

@@ -1,0 +1,279 @@
+"""Thin Python binding of libsal (include/sal.h): argument marshalling over ctypes.
+
+Every computation runs in the CUDA library; this module only allocates output buffers
+with PyTorch (device memory and streams are PyTorch's), passes raw pointers, and turns
+status codes into exceptions. There is no CPU fallback: if libsal.so is missing or the
+device is not an sm_100 GPU, the calls raise.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import numpy as np
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libsal.so")
+
+N_MELS, STACK, STACK_DIM, WIDTH, HEADS, HEAD_DIM, FFN = 128, 8, 1024, 1280, 10, 128, 5120
+MAX_POSITIONS = 45000
+
+SAL_EPI_STORE_F32, SAL_EPI_STORE_BF16, SAL_EPI_GELU_BF16, SAL_EPI_RESID_F32 = 0, 1, 2, 3
+
+LAYER_FIELDS = ["ln1_g", "ln1_b", "w_qkv", "b_qkv", "qn_g", "kn_g", "w_o", "b_o",
+                "ln2_g", "ln2_b", "w1", "b1", "w2", "b2"]
+
+
+class SalError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        self.status = status
+        super().__init__(f"{fn}: {status_string(status)} (status {status})")
+
+
+class sal_layer(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in LAYER_FIELDS]
+
+
+class sal_weights(ctypes.Structure):
+    _fields_ = [("w_proj", ctypes.c_void_p), ("b_proj", ctypes.c_void_p),
+                ("layers", ctypes.POINTER(sal_layer)), ("n_layers", ctypes.c_int),
+                ("lnf_g", ctypes.c_void_p), ("lnf_b", ctypes.c_void_p)]
+
+
+EXPORTS = {
+    # name: (restype, argtypes)
+    "sal_frame_count": (ctypes.c_int64, [ctypes.c_int64]),
+    "sal_position_count": (ctypes.c_int64, [ctypes.c_int64]),
+    "sal_status_string": (ctypes.c_char_p, [ctypes.c_int]),
+    "sal_frontend": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_void_p,
+                                     ctypes.c_void_p, ctypes.c_void_p]),
+    "sal_stack_project": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int, ctypes.c_int64,
+                                          ctypes.POINTER(sal_weights), ctypes.c_void_p, ctypes.c_void_p]),
+    "sal_encoder_workspace_bytes": (ctypes.c_size_t, [ctypes.c_int, ctypes.c_int64]),
+    "sal_encoder_forward": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int, ctypes.c_int64,
+                                            ctypes.POINTER(sal_weights), ctypes.c_int, ctypes.c_void_p,
+                                            ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]),
+    "sal_encode_workspace_bytes": (ctypes.c_size_t, [ctypes.c_int, ctypes.c_int64]),
+    "sal_encode": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.POINTER(sal_weights),
+                                   ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_size_t,
+                                   ctypes.c_void_p]),
+    "sal_last_device_status": (ctypes.c_int, [ctypes.c_void_p]),
+    "sal_set_wait_limit_ns": (None, [ctypes.c_uint64]),
+    "sal_layernorm": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int64, ctypes.c_void_p, ctypes.c_void_p,
+                                      ctypes.c_void_p, ctypes.c_void_p]),
+    "sal_linear": (ctypes.c_int, [ctypes.c_int, ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_void_p,
+                                   ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p]),
+    "sal_qkv_rope": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.POINTER(sal_layer),
+                                     ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+                                     ctypes.c_void_p]),
+    "sal_attention": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int,
+                                      ctypes.c_int64, ctypes.c_void_p, ctypes.c_void_p]),
+}
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded libsal.so. Raises if it has not been built."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: run `python -m speech_audio_encoder_b200.build`")
+        l = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in EXPORTS.items():
+            f = getattr(l, name)
+            f.restype = res
+            f.argtypes = args
+        _lib = l
+    return _lib
+
+
+def status_string(status: int) -> str:
+    return lib().sal_status_string(int(status)).decode()
+
+
+def _check(fn: str, status: int) -> None:
+    if status != 0:
+        raise SalError(fn, status)
+
+
+def _ptr(t) -> int:
+    if t is None:
+        return 0
+    if isinstance(t, torch.Tensor):
+        if not t.is_contiguous():
+            raise ValueError("tensors passed to libsal must be contiguous")
+        return t.data_ptr()
+    return int(t)
+
+
+def _stream(stream) -> int:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+# ----------------------------------------------------------------------------- counts
+
+def frame_count(n_samples: int) -> int:
+    return lib().sal_frame_count(int(n_samples))
+
+
+def position_count(n_samples: int) -> int:
+    return lib().sal_position_count(int(n_samples))
+
+
+# ----------------------------------------------------------------------------- weights
+
+class DeviceWeights:
+    """Encoder parameters in one device buffer, plus the sal_weights record that points into it.
+
+    ``w`` is the nested dict of (bf16 bits, float32) pairs from ``synth.make_weights``.
+    """
+
+    def __init__(self, w: dict, device="cuda"):
+        names, arrays = [], []
+        for k in ("w_proj", "b_proj", "lnf_g", "lnf_b"):
+            names.append((None, k))
+            arrays.append(w[k][0])
+        for i, lw in enumerate(w["layers"]):
+            for k in LAYER_FIELDS:
+                names.append((i, k))
+                arrays.append(lw[k][0])
+        offsets, off = [], 0
+        for a in arrays:
+            offsets.append(off)
+            off += (a.size + 127) // 128 * 128  # 256-byte aligned bf16 offsets
+        host = np.zeros(off, dtype=np.uint16)
+        for a, o in zip(arrays, offsets):
+            host[o:o + a.size] = a.reshape(-1)
+        self.buffer = torch.from_numpy(host.view(np.int16)).to(device).view(torch.bfloat16)
+        base = self.buffer.data_ptr()
+        self.n_layers = len(w["layers"])
+        self._layers = (sal_layer * max(self.n_layers, 1))()
+        self.ptr = {}
+        for (i, k), o in zip(names, offsets):
+            p = base + 2 * o
+            self.ptr[(i, k)] = p
+            if i is not None:
+                setattr(self._layers[i], k, p)
+        self.record = sal_weights(self.ptr[(None, "w_proj")], self.ptr[(None, "b_proj")],
+                                  self._layers, self.n_layers, self.ptr[(None, "lnf_g")],
+                                  self.ptr[(None, "lnf_b")])
+
+    def layer(self, i: int) -> sal_layer:
+        return self._layers[i]
+
+    def sub(self, first: int, count: int) -> sal_weights:
+        """A sal_weights record over layers [first, first + count) (shares this buffer)."""
+        arr = ctypes.cast(ctypes.byref(self._layers, first * ctypes.sizeof(sal_layer)),
+                          ctypes.POINTER(sal_layer))
+        rec = sal_weights(self.record.w_proj, self.record.b_proj, arr, count,
+                          self.record.lnf_g, self.record.lnf_b)
+        rec._keep = self  # keep the layer array alive
+        return rec
+
+
+# ----------------------------------------------------------------------------- calls
+
+def sal_frontend(wave: torch.Tensor, stacked: bool = True, stream=None):
+    """wave [batch, n] float32 (device) -> (logmel [batch, F, 128] f32, stacked [batch, T, 1024] bf16)."""
+    batch, n = wave.shape
+    F, T = frame_count(n), position_count(n)
+    logmel = torch.empty((batch, F, N_MELS), dtype=torch.float32, device=wave.device)
+    st = torch.empty((batch, T, STACK_DIM), dtype=torch.bfloat16, device=wave.device) if stacked else None
+    _check("sal_frontend", lib().sal_frontend(_ptr(wave), n, batch, _ptr(logmel), _ptr(st), _stream(stream)))
+    return logmel, st
+
+
+def sal_stack_project(stacked: torch.Tensor, weights: DeviceWeights, stream=None) -> torch.Tensor:
+    """stacked [batch, T, 1024] bf16 -> x [batch * T, 1280] float32."""
+    batch, T, _ = stacked.shape
+    x = torch.empty((batch * T, WIDTH), dtype=torch.float32, device=stacked.device)
+    _check("sal_stack_project", lib().sal_stack_project(_ptr(stacked), batch, T, ctypes.byref(weights.record),
+                                                        _ptr(x), _stream(stream)))
+    return x
+
+
+def encoder_workspace(batch: int, T: int, device="cuda") -> torch.Tensor:
+    n = lib().sal_encoder_workspace_bytes(batch, T)
+    return torch.empty(max(n, 256), dtype=torch.uint8, device=device)
+
+
+def sal_encoder_forward(x: torch.Tensor, batch: int, T: int, weights, n_layers: int,
+                        workspace: torch.Tensor | None = None, emb: torch.Tensor | None = None,
+                        stream=None) -> torch.Tensor:
+    """x [batch * T, 1280] f32 (clobbered: the residual stream after n_layers) -> emb bf16."""
+    rec = weights.record if isinstance(weights, DeviceWeights) else weights
+    if workspace is None:
+        workspace = encoder_workspace(batch, T, x.device)
+    if emb is None:
+        emb = torch.empty((batch * T, WIDTH), dtype=torch.bfloat16, device=x.device)
+    _check("sal_encoder_forward", lib().sal_encoder_forward(
+        _ptr(x), batch, T, ctypes.byref(rec), n_layers, _ptr(emb), _ptr(workspace),
+        workspace.numel(), _stream(stream)))
+    return emb
+
+
+def encode_workspace(batch: int, n_samples: int, device="cuda") -> torch.Tensor:
+    n = lib().sal_encode_workspace_bytes(batch, n_samples)
+    return torch.empty(max(n, 256), dtype=torch.uint8, device=device)
+
+
+def sal_encode(wave: torch.Tensor, weights: DeviceWeights, n_layers: int, emb: torch.Tensor | None = None,
+               workspace: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """Whole path; ``wave`` and ``emb`` may live on the host (pinned or not) or the device."""
+    batch, n = wave.shape
+    T = position_count(n)
+    if workspace is None:
+        workspace = encode_workspace(batch, n)
+    if emb is None:
+        emb = torch.empty((batch, T, WIDTH), dtype=torch.bfloat16, device=wave.device)
+    _check("sal_encode", lib().sal_encode(_ptr(wave), n, batch, ctypes.byref(weights.record), n_layers,
+                                          _ptr(emb), _ptr(workspace), workspace.numel(), _stream(stream)))
+    return emb
+
+
+def sal_layernorm(x: torch.Tensor, g: int, b: int, stream=None) -> torch.Tensor:
+    y = torch.empty(x.shape, dtype=torch.bfloat16, device=x.device)
+    _check("sal_layernorm", lib().sal_layernorm(_ptr(x), x.shape[0], g, b, _ptr(y), _stream(stream)))
+    return y
+
+
+def sal_linear(epilogue: int, A: torch.Tensor, W: torch.Tensor, bias: torch.Tensor,
+               out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    M, K = A.shape
+    N = W.shape[0]
+    if out is None:
+        dt = torch.float32 if epilogue in (SAL_EPI_STORE_F32, SAL_EPI_RESID_F32) else torch.bfloat16
+        out = torch.empty((M, N), dtype=dt, device=A.device)
+    _check("sal_linear", lib().sal_linear(epilogue, _ptr(A), M, K, _ptr(W), N, _ptr(bias), _ptr(out),
+                                          _stream(stream)))
+    return out
+
+
+def sal_qkv_rope(h: torch.Tensor, batch: int, T: int, layer: sal_layer, stream=None):
+    shape = (batch, HEADS, T, HEAD_DIM)
+    q = torch.empty(shape, dtype=torch.bfloat16, device=h.device)
+    k = torch.empty_like(q)
+    v = torch.empty_like(q)
+    cs = torch.empty((2, T, 64), dtype=torch.float32, device=h.device)
+    _check("sal_qkv_rope", lib().sal_qkv_rope(_ptr(h), batch, T, ctypes.byref(layer), _ptr(q), _ptr(k), _ptr(v),
+                                              _ptr(cs), _stream(stream)))
+    return q, k, v
+
+
+def sal_attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, stream=None) -> torch.Tensor:
+    batch, H, T, hd = q.shape
+    o = torch.empty((batch * T, H * hd), dtype=torch.bfloat16, device=q.device)
+    _check("sal_attention", lib().sal_attention(_ptr(q), _ptr(k), _ptr(v), batch, T, _ptr(o), _stream(stream)))
+    return o
+
+
+def sal_last_device_status(stream=None) -> int:
+    return lib().sal_last_device_status(_stream(stream))
+
+
+def sal_set_wait_limit_ns(ns: int) -> None:
+    lib().sal_set_wait_limit_ns(int(ns))

@@ -1,0 +1,322 @@
+// Bidirectional multi-head attention of the encoder on the tensor cores:
+//   O[b, t, 128 h + :] = softmax(q_h k_h^T / sqrt(128)) v_h   over all T positions of clip b
+// (page "Nemotron 3.5 Transcribe: From Recorded Speech to Dataset Audits", section "How
+// audio and speakers reach the language model": ten heads over width 1,280; full-clip
+// bidirectional attention, no mask).
+//
+// Flash-style streaming: the T x T score matrix is never stored. One CTA owns a tile of
+// 128 query rows of one (clip, head) and walks the keys 128 at a time:
+//   * warp 0 loads Q once and K / V tiles through a two-stage TMA ring (128-byte swizzle);
+//   * warp 1 (one thread) issues S_j = Q K_j^T (tcgen05.mma, both operands in shared
+//     memory) into one of two TMEM score buffers, then O += P_j V_j with P_j read from TMEM
+//     (A operand) and V_j from shared memory (MN-major B operand);
+//   * warps 2-5 own one query row per thread: read S_j from TMEM, online softmax in the
+//     log2 domain (exp2 on the SFU), write P_j back to TMEM as bf16 pairs, and rescale the
+//     TMEM accumulator O only when the running maximum grew by more than 2^8 (otherwise
+//     the stale maximum keeps every p <= 256, exact in fp32 and bf16 range);
+//   * S_{j+1} is computed while the softmax of S_j runs.
+// TMEM columns: S0 [0,128), S1 [128,256), O [256,384), P0 [384,448), P1 [448,512).
+#include <cuda_bf16.h>
+#include <math.h>
+
+#include <mutex>
+
+#include "sal_internal.h"
+#include "sal_ptx.cuh"
+
+namespace sal {
+namespace {
+
+constexpr int kTile = 128;
+constexpr int kBox = kTile * 64 * 2;       // one 64-column half of a 128 x 128 bf16 tile
+constexpr int kTileBytes = 2 * kBox;       // 32 KB
+constexpr uint32_t kColO = 256;
+__device__ __forceinline__ uint32_t col_s(int s) { return s ? 128u : 0u; }    // score buffers
+__device__ __forceinline__ uint32_t col_p(int s) { return s ? 448u : 384u; }  // bf16 P buffers
+constexpr size_t kSmem = 1024 + 5 * kTileBytes + 256;
+constexpr float kRescaleThreshold = 8.0f;  // log2 units
+
+struct AttnArgs {
+  int64_t T;
+  int heads;
+  __nv_bfloat16* o;
+  float scale_log2;
+  uint64_t limit_ns;
+  unsigned int* status;
+};
+
+__global__ void __launch_bounds__(192, 1)
+    attention_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                     const __grid_constant__ CUtensorMap tmV, const AttnArgs args) {
+  extern __shared__ unsigned char smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sQ = smem;
+  uint8_t* sK[2] = {smem + kTileBytes, smem + 2 * kTileBytes};
+  uint8_t* sV[2] = {smem + 3 * kTileBytes, smem + 4 * kTileBytes};
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + 5 * kTileBytes);
+  uint64_t* q_full = bars + 0;
+  uint64_t* k_full = bars + 1;    // [2]
+  uint64_t* v_full = bars + 3;    // [2]
+  uint64_t* kv_empty = bars + 5;  // [2]
+  uint64_t* s_full = bars + 7;    // [2]
+  uint64_t* p_full = bars + 9;
+  uint64_t* o_done = bars + 10;
+  uint64_t* drain = bars + 11;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 12);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int64_t T = args.T;
+  const int bh = blockIdx.y;
+  const int qt = blockIdx.x;
+  const int n_kv = static_cast<int>((T + kTile - 1) / kTile);
+
+  if (threadIdx.x == 0) {
+    mbar_init(q_full, 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&k_full[s], 1);
+      mbar_init(&v_full[s], 1);
+      mbar_init(&kv_empty[s], 1);
+      mbar_init(&s_full[s], 1);
+    }
+    mbar_init(p_full, 128);
+    mbar_init(o_done, 1);
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+    tma_prefetch_desc(&tmQ);
+    tma_prefetch_desc(&tmK);
+    tma_prefetch_desc(&tmV);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const WaitGuard guard{abort_flag, args.limit_ns, args.status};
+
+  if (warp == 0) {
+    if (lane == 0) {
+      uint32_t issued_q = 0, issued = 0, par_k = 0;
+      mbar_arrive_expect_tx(q_full, kTileBytes);
+      tma_load_3d(sQ, &tmQ, q_full, 0, qt * kTile, bh);
+      tma_load_3d(sQ + kBox, &tmQ, q_full, 64, qt * kTile, bh);
+      issued_q = 1;
+      for (int j = 0; j < n_kv; ++j) {
+        const int s = j & 1;
+        const uint32_t use_par = (j >> 1) & 1;
+        if (!mbar_wait(&kv_empty[s], use_par ^ 1, guard)) break;
+        mbar_arrive_expect_tx(&k_full[s], kTileBytes);
+        tma_load_3d(sK[s], &tmK, &k_full[s], 0, j * kTile, bh);
+        tma_load_3d(sK[s] + kBox, &tmK, &k_full[s], 64, j * kTile, bh);
+        mbar_arrive_expect_tx(&v_full[s], kTileBytes);
+        tma_load_3d(sV[s], &tmV, &v_full[s], 0, j * kTile, bh);
+        tma_load_3d(sV[s] + kBox, &tmV, &v_full[s], 64, j * kTile, bh);
+        issued |= 1u << s;
+        par_k = (par_k & ~(1u << s)) | (use_par << s);
+      }
+      if (*abort_flag) {
+        if (issued_q) drain_wait(q_full, 0, args.limit_ns);
+        for (int s = 0; s < 2; ++s)
+          if (issued & (1u << s)) {
+            drain_wait(&k_full[s], (par_k >> s) & 1, args.limit_ns);
+            drain_wait(&v_full[s], (par_k >> s) & 1, args.limit_ns);
+          }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      constexpr uint32_t IDESC_S = idesc_bf16(128, 128, false, false);
+      constexpr uint32_t IDESC_O = idesc_bf16(128, 128, false, true);
+      bool ok = mbar_wait(q_full, 0, guard);
+      bool any_mma = false;
+      const uint32_t q0 = smem_u32(sQ);
+      auto issue_s = [&](int j) -> bool {
+        const int s = j & 1;
+        if (!mbar_wait(&k_full[s], (j >> 1) & 1, guard)) return false;
+        tc_fence_after();
+        const uint32_t k0 = smem_u32(sK[s]);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint32_t off = (kk >> 2) * kBox + (kk & 3) * 32;
+          umma_ss(tmem + col_s(s), sdesc_kmajor_sw128(q0 + off), sdesc_kmajor_sw128(k0 + off), IDESC_S,
+                  kk > 0);
+        }
+        umma_commit(&s_full[s]);
+        any_mma = true;
+        return true;
+      };
+      if (ok) ok = issue_s(0);
+      for (int j = 0; ok && j < n_kv; ++j) {
+        const int s = j & 1;
+        if (j + 1 < n_kv && !issue_s(j + 1)) break;
+        if (!mbar_wait(p_full, j & 1, guard)) break;
+        if (!mbar_wait(&v_full[s], (j >> 1) & 1, guard)) break;
+        tc_fence_after();
+        const uint32_t v0 = smem_u32(sV[s]);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          umma_ts(tmem + kColO, tmem + col_p(s) + kk * 8, sdesc_mnmajor_sw128(v0 + kk * 2048, kBox), IDESC_O,
+                  (j > 0 || kk > 0));
+        umma_commit(&kv_empty[s]);
+        umma_commit(o_done);
+      }
+      if (*abort_flag && any_mma) {
+        // every MMA issued so far is covered by one more commit
+        umma_commit(drain);
+        drain_wait(drain, 0, args.limit_ns);
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ softmax warps 2..5
+    const int quarter = warp & 3;
+    const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
+    const int row = quarter * 32 + lane;
+    const float sl2 = args.scale_log2;
+    float m_ref = -INFINITY, l = 0.f;
+    bool ok = true;
+    for (int j = 0; j < n_kv; ++j) {
+      const int s = j & 1;
+      if (!mbar_wait_warp(&s_full[s], (j >> 1) & 1, guard)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      uint32_t r[4][32];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) tmem_ld32(tmem + lane_base + col_s(s) + 32 * c, r[c]);
+      tmem_wait_ld();
+      const int64_t rem = T - static_cast<int64_t>(j) * kTile;
+      const int valid = static_cast<int>(rem < kTile ? rem : kTile);
+      float mx = -INFINITY;
+#pragma unroll
+      for (int c = 0; c < 4; ++c)
+#pragma unroll
+        for (int i = 0; i < 32; ++i)
+          if (32 * c + i < valid) mx = fmaxf(mx, __uint_as_float(r[c][i]));
+      mx *= sl2;
+      float alpha = 1.f;
+      bool rescale = false;
+      if (j == 0) {
+        m_ref = mx;
+      } else if (mx > m_ref + kRescaleThreshold) {
+        alpha = fast_exp2(m_ref - mx);
+        m_ref = mx;
+        rescale = true;
+      }
+      float sum = 0.f;
+      uint32_t p[2][32];
+#pragma unroll
+      for (int c = 0; c < 4; ++c)
+#pragma unroll
+        for (int i = 0; i < 32; i += 2) {
+          const int col = 32 * c + i;
+          const float e0 = col < valid ? fast_exp2(fmaf(__uint_as_float(r[c][i]), sl2, -m_ref)) : 0.f;
+          const float e1 = col + 1 < valid ? fast_exp2(fmaf(__uint_as_float(r[c][i + 1]), sl2, -m_ref)) : 0.f;
+          sum += e0 + e1;
+          p[c >> 1][(c & 1) * 16 + (i >> 1)] = pack_bf16x2(e0, e1);
+        }
+      if (j > 0) {
+        // PV_{j-1} must be complete before O is rescaled or P buffer s is overwritten
+        if (!mbar_wait_warp(o_done, (j - 1) & 1, guard)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        if (__any_sync(0xffffffffu, rescale)) {
+#pragma unroll 1
+          for (int c = 0; c < 4; ++c) {
+            uint32_t o[32];
+            tmem_ld32(tmem + lane_base + kColO + 32 * c, o);
+            tmem_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+            tmem_st32(tmem + lane_base + kColO + 32 * c, o);
+          }
+        }
+      }
+      l = l * alpha + sum;
+      tmem_st32(tmem + lane_base + col_p(s), p[0]);
+      tmem_st32(tmem + lane_base + col_p(s) + 32, p[1]);
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(p_full);
+    }
+    if (ok && mbar_wait_warp(o_done, (n_kv - 1) & 1, guard)) {
+      tc_fence_after();
+      const int64_t t = static_cast<int64_t>(qt) * kTile + row;
+      const int b = bh / args.heads, h = bh % args.heads;
+      const float inv_l = 1.0f / l;
+      __nv_bfloat16* dst = args.o + (static_cast<int64_t>(b) * T + t) * (args.heads * kHeadDim) + h * kHeadDim;
+#pragma unroll 1
+      for (int c = 0; c < 4; ++c) {
+        uint32_t o[32];
+        tmem_ld32(tmem + lane_base + kColO + 32 * c, o);
+        tmem_wait_ld();
+        if (t < T) {
+          uint4* d4 = reinterpret_cast<uint4*>(dst + 32 * c);
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            uint4 u;
+            u.x = pack_bf16x2(__uint_as_float(o[8 * i + 0]) * inv_l, __uint_as_float(o[8 * i + 1]) * inv_l);
+            u.y = pack_bf16x2(__uint_as_float(o[8 * i + 2]) * inv_l, __uint_as_float(o[8 * i + 3]) * inv_l);
+            u.z = pack_bf16x2(__uint_as_float(o[8 * i + 4]) * inv_l, __uint_as_float(o[8 * i + 5]) * inv_l);
+            u.w = pack_bf16x2(__uint_as_float(o[8 * i + 6]) * inv_l, __uint_as_float(o[8 * i + 7]) * inv_l);
+            d4[i] = u;
+          }
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+std::mutex g_mu;
+bool g_attr[64] = {};
+
+}  // namespace
+
+sal_status attention_launch(const void* q, const void* k, const void* v, int batch, int64_t T,
+                            void* o, cudaStream_t s) {
+  if (T == 0 || batch == 0) return SAL_OK;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  {
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (dev >= 0 && dev < 64 && !g_attr[dev]) {
+      if (cudaFuncSetAttribute(attention_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               static_cast<int>(kSmem)) != cudaSuccess)
+        return SAL_ECUDA;
+      g_attr[dev] = true;
+    }
+  }
+  const uint64_t bh = static_cast<uint64_t>(batch) * kHeads;
+  CUtensorMap tq, tk, tv;
+  if (!make_tmap_3d_bf16(&tq, q, kHeadDim, T, bh, 64, kTile, 1)) return SAL_ECUDA;
+  if (!make_tmap_3d_bf16(&tk, k, kHeadDim, T, bh, 64, kTile, 1)) return SAL_ECUDA;
+  if (!make_tmap_3d_bf16(&tv, v, kHeadDim, T, bh, 64, kTile, 1)) return SAL_ECUDA;
+  AttnArgs a;
+  a.T = T;
+  a.heads = kHeads;
+  a.o = static_cast<__nv_bfloat16*>(o);
+  a.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(128.0));
+  a.limit_ns = wait_limit_ns();
+  a.status = device_status_ptr();
+  if (!a.status) return SAL_ECUDA;
+  const dim3 grid(static_cast<unsigned>((T + kTile - 1) / kTile), static_cast<unsigned>(bh));
+  attention_kernel<<<grid, 192, kSmem, s>>>(tq, tk, tv, a);
+  return cudaGetLastError() == cudaSuccess ? SAL_OK : SAL_ECUDA;
+}
+
+}  // namespace sal

@@ -1,0 +1,100 @@
+// Row kernels of the encoder: the pre-norm / final LayerNorm, and the RoPE table.
+//
+// LayerNorm (eps 1e-5, affine) normalises each 1280-wide fp32 row of the residual
+// stream and writes it as bf16, the operand of the next tensor-core GEMM. One warp per
+// row: 40 values per lane held in registers, two-pass mean and variance.
+//
+// RoPE table: cos and sin of t * 10000^(-2 i / 128), i < 64, t < T. The angle reaches
+// 4.5e4 rad at one hour, where fp32 would lose ~3 digits, so it is formed and reduced in
+// fp64 before the fp32 table entry is written.
+#include <cuda_bf16.h>
+#include <math.h>
+
+#include "sal_internal.h"
+
+namespace sal {
+namespace {
+
+constexpr int kLnWarps = 8;
+constexpr int kVec = kWidth / 4 / 32;  // float4 per lane = 10
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+__global__ void __launch_bounds__(256) layernorm_kernel(const float* __restrict__ x, int64_t rows,
+                                                        const __nv_bfloat16* __restrict__ g,
+                                                        const __nv_bfloat16* __restrict__ b,
+                                                        __nv_bfloat16* __restrict__ y) {
+  const int lane = threadIdx.x & 31;
+  const int64_t row = static_cast<int64_t>(blockIdx.x) * kLnWarps + (threadIdx.x >> 5);
+  if (row >= rows) return;
+  const float4* xr = reinterpret_cast<const float4*>(x + row * kWidth);
+  float4 v[kVec];
+  float s = 0.f;
+#pragma unroll
+  for (int i = 0; i < kVec; ++i) {
+    v[i] = xr[lane + 32 * i];
+    s += (v[i].x + v[i].y) + (v[i].z + v[i].w);
+  }
+  const float mean = warp_sum(s) * (1.0f / kWidth);
+  float q = 0.f;
+#pragma unroll
+  for (int i = 0; i < kVec; ++i) {
+    const float a = v[i].x - mean, bb = v[i].y - mean, c = v[i].z - mean, d = v[i].w - mean;
+    q += (a * a + bb * bb) + (c * c + d * d);
+  }
+  const float rstd = 1.0f / sqrtf(warp_sum(q) * (1.0f / kWidth) + 1e-5f);
+  const uint2* g2 = reinterpret_cast<const uint2*>(g);
+  const uint2* b2 = reinterpret_cast<const uint2*>(b);
+  uint2* yr = reinterpret_cast<uint2*>(y + row * kWidth);
+#pragma unroll
+  for (int i = 0; i < kVec; ++i) {
+    const int c4 = lane + 32 * i;
+    const uint2 gg = __ldg(g2 + c4), bb = __ldg(b2 + c4);
+    const float o0 = (v[i].x - mean) * rstd * __uint_as_float(gg.x << 16) + __uint_as_float(bb.x << 16);
+    const float o1 = (v[i].y - mean) * rstd * __uint_as_float(gg.x & 0xFFFF0000u) + __uint_as_float(bb.x & 0xFFFF0000u);
+    const float o2 = (v[i].z - mean) * rstd * __uint_as_float(gg.y << 16) + __uint_as_float(bb.y << 16);
+    const float o3 = (v[i].w - mean) * rstd * __uint_as_float(gg.y & 0xFFFF0000u) + __uint_as_float(bb.y & 0xFFFF0000u);
+    __nv_bfloat162 p0 = __floats2bfloat162_rn(o0, o1), p1 = __floats2bfloat162_rn(o2, o3);
+    uint2 out;
+    out.x = *reinterpret_cast<uint32_t*>(&p0);
+    out.y = *reinterpret_cast<uint32_t*>(&p1);
+    yr[c4] = out;
+  }
+}
+
+__global__ void rope_table_kernel(float* __restrict__ cs, int64_t T) {
+  const int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (idx >= T * 64) return;
+  const int64_t t = idx >> 6;
+  const int i = static_cast<int>(idx & 63);
+  const double inv = pow(10000.0, -static_cast<double>(2 * i) / 128.0);
+  double s, c;
+  sincos(static_cast<double>(t) * inv, &s, &c);
+  cs[idx] = static_cast<float>(c);
+  cs[T * 64 + idx] = static_cast<float>(s);
+}
+
+}  // namespace
+
+sal_status layernorm_launch(const float* x, int64_t rows, const void* g, const void* b, void* y,
+                            cudaStream_t s) {
+  if (rows == 0) return SAL_OK;
+  const unsigned grid = static_cast<unsigned>((rows + kLnWarps - 1) / kLnWarps);
+  layernorm_kernel<<<grid, 32 * kLnWarps, 0, s>>>(x, rows, static_cast<const __nv_bfloat16*>(g),
+                                                  static_cast<const __nv_bfloat16*>(b),
+                                                  static_cast<__nv_bfloat16*>(y));
+  return cudaGetLastError() == cudaSuccess ? SAL_OK : SAL_ECUDA;
+}
+
+sal_status rope_table_launch(float* cs, int64_t T, cudaStream_t s) {
+  if (T == 0) return SAL_OK;
+  const int64_t n = T * 64;
+  rope_table_kernel<<<static_cast<unsigned>((n + 255) / 256), 256, 0, s>>>(cs, T);
+  return cudaGetLastError() == cudaSuccess ? SAL_OK : SAL_ECUDA;
+}
+
+}  // namespace sal

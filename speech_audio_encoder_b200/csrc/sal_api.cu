@@ -1,0 +1,357 @@
+// The extern "C" entry points of libsal (declared in include/sal.h): argument checks,
+// tensor-map construction, workspace layout and the per-layer launch sequence.
+//
+// Per encoder layer, on the caller's stream (page "Nemotron 3.5 Transcribe: From Recorded
+// Speech to Dataset Audits", section "How audio and speakers reach the language model"):
+//   1. h = LayerNorm1(x)                                  (row kernel, fp32 -> bf16)
+//   2. q, k, v = RoPE(RMSNorm(h Wqkv^T + b))              (GEMM, QK-norm + RoPE epilogue)
+//   3. o = softmax(q k^T / sqrt(128)) v                   (attention kernel)
+//   4. x += o Wo^T + bo                                   (GEMM, residual epilogue)
+//   5. h = LayerNorm2(x)                                  (row kernel)
+//   6. u = GELU(h W1^T + b1)                              (GEMM, GELU epilogue)
+//   7. x += u W2^T + b2                                   (GEMM, residual epilogue)
+// and after the last layer emb = LayerNormF(x).
+#include <cudaTypedefs.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <atomic>
+#include <mutex>
+
+#include "sal_internal.h"
+#include "sal_ptx.cuh"
+
+namespace sal {
+
+__device__ unsigned int g_status = 0;
+
+namespace {
+
+std::atomic<uint64_t> g_wait_limit_ns{4000000000ull};
+
+PFN_cuTensorMapEncodeTiled_v12000 g_encode_tiled = nullptr;
+std::once_flag g_encode_once;
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  std::call_once(g_encode_once, [] {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      g_encode_tiled = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  });
+  return g_encode_tiled;
+}
+
+std::mutex g_dev_mu;
+int g_dev_ok[64] = {};  // 0 unknown, 1 sm_100, 2 other
+
+sal_status check_device() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return SAL_ECUDA;
+  if (dev < 0 || dev >= 64) return SAL_EDEVICE;
+  std::lock_guard<std::mutex> lk(g_dev_mu);
+  if (!g_dev_ok[dev]) {
+    int major = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess) return SAL_ECUDA;
+    g_dev_ok[dev] = major == 10 ? 1 : 2;
+  }
+  return g_dev_ok[dev] == 1 ? SAL_OK : SAL_EDEVICE;
+}
+
+constexpr size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+struct EncoderWs {
+  void* h;      // [M, 1280] bf16
+  void *q, *k, *v, *o;  // [M, 1280] bf16 each; u [M, 5120] bf16 overlays all four
+  void* u;
+  float* rope;  // [2, T, 64] f32
+  size_t bytes;
+};
+
+EncoderWs encoder_ws_layout(void* base, int batch, int64_t T) {
+  const size_t M = static_cast<size_t>(batch) * static_cast<size_t>(T);
+  const size_t act = align256(M * kWidth * 2);
+  EncoderWs w{};
+  char* p = static_cast<char*>(base);
+  size_t off = 0;
+  w.h = p + off;
+  off += act;
+  w.q = p + off;
+  w.k = p + off + act;
+  w.v = p + off + 2 * act;
+  w.o = p + off + 3 * act;
+  w.u = p + off;
+  off += std::max(4 * act, align256(M * kFfn * 2));
+  w.rope = reinterpret_cast<float*>(p + off);
+  off += align256(static_cast<size_t>(T) * 64 * 2 * sizeof(float));
+  w.bytes = off;
+  return w;
+}
+
+bool layer_ok(const sal_layer& L) {
+  const void* ps[] = {L.ln1_g, L.ln1_b, L.w_qkv, L.b_qkv, L.qn_g, L.kn_g, L.w_o,
+                      L.b_o,   L.ln2_g, L.ln2_b, L.w1,    L.b1,    L.w2,   L.b2};
+  for (const void* p : ps)
+    if (!p || !aligned16(p)) return false;
+  return true;
+}
+
+bool is_device_ptr(const void* p) {
+  cudaPointerAttributes a;
+  if (cudaPointerGetAttributes(&a, p) != cudaSuccess) {
+    cudaGetLastError();
+    return false;
+  }
+  return a.type == cudaMemoryTypeDevice || a.type == cudaMemoryTypeManaged;
+}
+
+}  // namespace
+
+uint64_t wait_limit_ns() { return g_wait_limit_ns.load(); }
+
+unsigned int* device_status_ptr() {
+  static std::mutex mu;
+  static unsigned int* ptrs[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  std::lock_guard<std::mutex> lk(mu);
+  if (!ptrs[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_status) != cudaSuccess) return nullptr;
+    ptrs[dev] = static_cast<unsigned int*>(p);
+  }
+  return ptrs[dev];
+}
+
+bool make_tmap_2d_bf16(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer,
+                       uint32_t box_inner, uint32_t box_outer) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {inner * 2};
+  cuuint32_t box[2] = {box_inner, box_outer};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool make_tmap_3d_bf16(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1, uint64_t d2,
+                       uint32_t b0, uint32_t b1, uint32_t b2) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {d0, d1, d2};
+  cuuint64_t strides[2] = {d0 * 2, d0 * d1 * 2};
+  cuuint32_t box[3] = {b0, b1, b2};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace sal
+
+using namespace sal;
+
+#define SAL_TRY(expr)                 \
+  do {                                \
+    const sal_status st_ = (expr);    \
+    if (st_ != SAL_OK) return st_;    \
+  } while (0)
+
+extern "C" {
+
+int64_t sal_frame_count(int64_t n) { return n < kWin ? 0 : 1 + (n - kWin) / kHop; }
+
+int64_t sal_position_count(int64_t n) { return sal_frame_count(n) / kStack; }
+
+const char* sal_status_string(int status) {
+  switch (status) {
+    case SAL_OK: return "ok";
+    case SAL_EINVAL: return "invalid argument (null or misaligned pointer, bad value)";
+    case SAL_ESHAPE: return "unsupported shape";
+    case SAL_EWORKSPACE: return "workspace too small";
+    case SAL_ECUDA: return "CUDA runtime error";
+    case SAL_ETIMEOUT: return "a bounded device wait gave up";
+    case SAL_EDEVICE: return "device is not an sm_100 GPU";
+    default: return "unknown status";
+  }
+}
+
+void sal_set_wait_limit_ns(uint64_t ns) { g_wait_limit_ns.store(ns ? ns : 1); }
+
+sal_status sal_last_device_status(void* stream) {
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return SAL_ECUDA;
+  unsigned int v = 0, zero = 0;
+  if (cudaMemcpyFromSymbol(&v, g_status, sizeof(v)) != cudaSuccess) return SAL_ECUDA;
+  if (v && cudaMemcpyToSymbol(g_status, &zero, sizeof(zero)) != cudaSuccess) return SAL_ECUDA;
+  return (v & kStatusTimeout) ? SAL_ETIMEOUT : SAL_OK;
+}
+
+sal_status sal_frontend(const float* wave, int64_t n_samples, int batch, float* logmel, void* stacked,
+                        void* stream) {
+  if (batch < 0 || n_samples < 0) return SAL_EINVAL;
+  const int64_t F = sal_frame_count(n_samples), T = F / kStack;
+  if (T > SAL_MAX_POSITIONS) return SAL_ESHAPE;
+  if (batch == 0 || F == 0) return SAL_OK;
+  if (batch > 65535) return SAL_ESHAPE;
+  if (!wave || !logmel || !aligned16(wave) || !aligned16(logmel)) return SAL_EINVAL;
+  if (stacked && !aligned16(stacked)) return SAL_EINVAL;
+  SAL_TRY(check_device());
+  return frontend_launch(wave, n_samples, batch, F, T, logmel, stacked, static_cast<cudaStream_t>(stream));
+}
+
+sal_status sal_stack_project(const void* stacked, int batch, int64_t T, const sal_weights* w, float* x,
+                             void* stream) {
+  if (batch < 0 || T < 0 || !w) return SAL_EINVAL;
+  if (T > SAL_MAX_POSITIONS) return SAL_ESHAPE;
+  if (batch == 0 || T == 0) return SAL_OK;
+  if (!stacked || !x || !w->w_proj || !w->b_proj || !aligned16(stacked) || !aligned16(x) ||
+      !aligned16(w->w_proj) || !aligned16(w->b_proj))
+    return SAL_EINVAL;
+  SAL_TRY(check_device());
+  return gemm_launch(SAL_EPI_STORE_F32, stacked, static_cast<int64_t>(batch) * T, SAL_STACK_DIM, w->w_proj,
+                     kWidth, w->b_proj, x, nullptr, static_cast<cudaStream_t>(stream));
+}
+
+size_t sal_encoder_workspace_bytes(int batch, int64_t T) {
+  if (batch <= 0 || T <= 0) return 0;
+  return encoder_ws_layout(nullptr, batch, T).bytes;
+}
+
+sal_status sal_encoder_forward(float* x, int batch, int64_t T, const sal_weights* w, int n_layers, void* emb,
+                               void* workspace, size_t ws_bytes, void* stream) {
+  if (batch < 0 || T < 0 || !w || n_layers < 0 || n_layers > w->n_layers) return SAL_EINVAL;
+  if (T > SAL_MAX_POSITIONS) return SAL_ESHAPE;
+  if (batch == 0 || T == 0) return SAL_OK;
+  if (batch > 6553) return SAL_ESHAPE;  // attention grid.y = 10 * batch
+  if (!x || !emb || !aligned16(x) || !aligned16(emb)) return SAL_EINVAL;
+  if (!w->lnf_g || !w->lnf_b || !aligned16(w->lnf_g) || !aligned16(w->lnf_b)) return SAL_EINVAL;
+  if (n_layers > 0 && !w->layers) return SAL_EINVAL;
+  for (int i = 0; i < n_layers; ++i)
+    if (!layer_ok(w->layers[i])) return SAL_EINVAL;
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u)) return SAL_EINVAL;
+  const EncoderWs ws = encoder_ws_layout(workspace, batch, T);
+  if (ws_bytes < ws.bytes) return SAL_EWORKSPACE;
+  SAL_TRY(check_device());
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int64_t M = static_cast<int64_t>(batch) * T;
+  if (n_layers > 0) SAL_TRY(rope_table_launch(ws.rope, T, s));
+  for (int i = 0; i < n_layers; ++i) {
+    const sal_layer& L = w->layers[i];
+    SAL_TRY(layernorm_launch(x, M, L.ln1_g, L.ln1_b, ws.h, s));
+    QkvOut qo{ws.q, ws.k, ws.v, L.qn_g, L.kn_g, ws.rope, T};
+    SAL_TRY(gemm_launch(kEpiQkv, ws.h, M, kWidth, L.w_qkv, 3 * kWidth, L.b_qkv, nullptr, &qo, s));
+    SAL_TRY(attention_launch(ws.q, ws.k, ws.v, batch, T, ws.o, s));
+    SAL_TRY(gemm_launch(SAL_EPI_RESID_F32, ws.o, M, kWidth, L.w_o, kWidth, L.b_o, x, nullptr, s));
+    SAL_TRY(layernorm_launch(x, M, L.ln2_g, L.ln2_b, ws.h, s));
+    SAL_TRY(gemm_launch(SAL_EPI_GELU_BF16, ws.h, M, kWidth, L.w1, kFfn, L.b1, ws.u, nullptr, s));
+    SAL_TRY(gemm_launch(SAL_EPI_RESID_F32, ws.u, M, kFfn, L.w2, kWidth, L.b2, x, nullptr, s));
+  }
+  return layernorm_launch(x, M, w->lnf_g, w->lnf_b, emb, s);
+}
+
+size_t sal_encode_workspace_bytes(int batch, int64_t n_samples) {
+  if (batch <= 0 || n_samples < 0) return 0;
+  const int64_t F = sal_frame_count(n_samples), T = F / kStack;
+  const size_t M = static_cast<size_t>(batch) * static_cast<size_t>(T);
+  size_t b = align256(static_cast<size_t>(batch) * n_samples * 4);          // staged wave
+  b += align256(static_cast<size_t>(batch) * F * kMels * 4);                // log-mel
+  b += align256(M * SAL_STACK_DIM * 2);                                     // stacked
+  b += align256(M * kWidth * 4);                                            // x
+  b += align256(M * kWidth * 2);                                            // staged emb
+  b += T > 0 ? encoder_ws_layout(nullptr, batch, T).bytes : 0;
+  return b;
+}
+
+sal_status sal_encode(const float* wave, int64_t n_samples, int batch, const sal_weights* w, int n_layers,
+                      void* emb, void* workspace, size_t ws_bytes, void* stream) {
+  if (batch < 0 || n_samples < 0 || !w) return SAL_EINVAL;
+  const int64_t F = sal_frame_count(n_samples), T = F / kStack;
+  if (T > SAL_MAX_POSITIONS) return SAL_ESHAPE;
+  if (batch == 0 || T == 0) return SAL_OK;
+  if (!wave || !emb || !workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u)) return SAL_EINVAL;
+  if (ws_bytes < sal_encode_workspace_bytes(batch, n_samples)) return SAL_EWORKSPACE;
+  SAL_TRY(check_device());
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const size_t M = static_cast<size_t>(batch) * static_cast<size_t>(T);
+  char* p = static_cast<char*>(workspace);
+  float* wave_d = reinterpret_cast<float*>(p);
+  p += align256(static_cast<size_t>(batch) * n_samples * 4);
+  float* logmel = reinterpret_cast<float*>(p);
+  p += align256(static_cast<size_t>(batch) * F * kMels * 4);
+  void* stacked = p;
+  p += align256(M * SAL_STACK_DIM * 2);
+  float* x = reinterpret_cast<float*>(p);
+  p += align256(M * kWidth * 4);
+  void* emb_d = p;
+  p += align256(M * kWidth * 2);
+  const size_t enc_bytes = encoder_ws_layout(nullptr, batch, T).bytes;
+
+  const bool wave_host = !is_device_ptr(wave);
+  const bool emb_host = !is_device_ptr(emb);
+  if (wave_host) {
+    if (cudaMemcpyAsync(wave_d, wave, static_cast<size_t>(batch) * n_samples * 4, cudaMemcpyHostToDevice, s) !=
+        cudaSuccess)
+      return SAL_ECUDA;
+  } else {
+    wave_d = const_cast<float*>(wave);
+  }
+  SAL_TRY(sal_frontend(wave_d, n_samples, batch, logmel, stacked, stream));
+  SAL_TRY(sal_stack_project(stacked, batch, T, w, x, stream));
+  SAL_TRY(sal_encoder_forward(x, batch, T, w, n_layers, emb_host ? emb_d : emb, p, enc_bytes, stream));
+  if (emb_host &&
+      cudaMemcpyAsync(emb, emb_d, M * kWidth * 2, cudaMemcpyDeviceToHost, s) != cudaSuccess)
+    return SAL_ECUDA;
+  return SAL_OK;
+}
+
+sal_status sal_layernorm(const float* x, int64_t rows, const void* g, const void* b, void* y, void* stream) {
+  if (rows < 0) return SAL_EINVAL;
+  if (rows == 0) return SAL_OK;
+  if (!x || !g || !b || !y || !aligned16(x) || !aligned16(g) || !aligned16(b) || !aligned16(y)) return SAL_EINVAL;
+  SAL_TRY(check_device());
+  return layernorm_launch(x, rows, g, b, y, static_cast<cudaStream_t>(stream));
+}
+
+sal_status sal_linear(int epilogue, const void* A, int64_t M, int K, const void* W, int N, const void* bias,
+                      void* out, void* stream) {
+  if (epilogue < SAL_EPI_STORE_F32 || epilogue > SAL_EPI_RESID_F32 || M < 0) return SAL_EINVAL;
+  if (M == 0) return SAL_OK;
+  if (!A || !W || !bias || !out || !aligned16(A) || !aligned16(W) || !aligned16(bias) || !aligned16(out))
+    return SAL_EINVAL;
+  SAL_TRY(check_device());
+  return gemm_launch(epilogue, A, M, K, W, N, bias, out, nullptr, static_cast<cudaStream_t>(stream));
+}
+
+sal_status sal_qkv_rope(const void* h, int batch, int64_t T, const sal_layer* layer, void* q, void* k, void* v,
+                        float* rope_cs, void* stream) {
+  if (batch < 0 || T < 0 || !layer) return SAL_EINVAL;
+  if (T > SAL_MAX_POSITIONS) return SAL_ESHAPE;
+  if (batch == 0 || T == 0) return SAL_OK;
+  if (!h || !q || !k || !v || !rope_cs || !aligned16(h) || !aligned16(q) || !aligned16(k) || !aligned16(v) ||
+      !aligned16(rope_cs) || !layer->w_qkv || !layer->b_qkv || !layer->qn_g || !layer->kn_g ||
+      !aligned16(layer->w_qkv) || !aligned16(layer->b_qkv) || !aligned16(layer->qn_g) || !aligned16(layer->kn_g))
+    return SAL_EINVAL;
+  SAL_TRY(check_device());
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  SAL_TRY(rope_table_launch(rope_cs, T, s));
+  QkvOut qo{q, k, v, layer->qn_g, layer->kn_g, rope_cs, T};
+  return gemm_launch(kEpiQkv, h, static_cast<int64_t>(batch) * T, kWidth, layer->w_qkv, 3 * kWidth,
+                     layer->b_qkv, nullptr, &qo, s);
+}
+
+sal_status sal_attention(const void* q, const void* k, const void* v, int batch, int64_t T, void* o,
+                         void* stream) {
+  if (batch < 0 || T < 0) return SAL_EINVAL;
+  if (T > SAL_MAX_POSITIONS) return SAL_ESHAPE;
+  if (batch == 0 || T == 0) return SAL_OK;
+  if (batch > 6553) return SAL_ESHAPE;  // grid.y = 10 * batch
+  if (!q || !k || !v || !o || !aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o))
+    return SAL_EINVAL;
+  SAL_TRY(check_device());
+  return attention_launch(q, k, v, batch, T, o, static_cast<cudaStream_t>(stream));
+}
+
+}  // extern "C"

@@ -1,0 +1,58 @@
+// Host-side declarations shared by the library's translation units.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/sal.h"
+
+namespace sal {
+
+constexpr int kWin = 400;
+constexpr int kHop = 160;
+constexpr int kNfft = 512;
+constexpr int kBins = 257;
+constexpr int kMels = SAL_N_MELS;
+constexpr int kStack = SAL_STACK;
+constexpr int kWidth = SAL_WIDTH;
+constexpr int kHeads = SAL_HEADS;
+constexpr int kHeadDim = SAL_HEAD_DIM;
+constexpr int kFfn = SAL_FFN;
+
+uint64_t wait_limit_ns();
+unsigned int* device_status_ptr();  // device address of the status word (current device)
+
+// frontend.cu
+sal_status frontend_launch(const float* wave, int64_t n_samples, int batch, int64_t frames,
+                           int64_t positions, float* logmel, void* stacked, cudaStream_t s);
+
+// rowops.cu
+sal_status layernorm_launch(const float* x, int64_t rows, const void* g, const void* b, void* y,
+                            cudaStream_t s);
+sal_status rope_table_launch(float* cs, int64_t T, cudaStream_t s);
+
+// gemm.cu
+struct QkvOut {
+  void *q, *k, *v;
+  const void *qn_g, *kn_g;
+  const float* rope_cs;  // [T][64] cos then [T][64] sin
+  int64_t T;
+};
+sal_status gemm_launch(int epilogue, const void* A, int64_t M, int K, const void* W, int N,
+                       const void* bias, void* out, const QkvOut* qkv, cudaStream_t s);
+constexpr int kEpiQkv = 100;  // internal epilogue id: QK-norm + RoPE scatter
+
+// attention.cu
+sal_status attention_launch(const void* q, const void* k, const void* v, int batch, int64_t T,
+                            void* o, cudaStream_t s);
+
+// tensor maps (sal_api.cu)
+bool make_tmap_2d_bf16(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer,
+                       uint32_t box_inner, uint32_t box_outer);
+bool make_tmap_3d_bf16(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1, uint64_t d2,
+                       uint32_t b0, uint32_t b1, uint32_t b2);
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+}  // namespace sal

@@ -1,0 +1,160 @@
+"""GPU parity of the whole path (sal_stack_project, sal_encoder_forward, sal_encode)
+against the fp64 oracle.
+
+Bar: final embeddings within relative L2 2e-2 of the oracle (bf16 GEMM / attention
+operands, fp32 accumulation and residual stream). The one-layer checks compare the
+layer's update x1 - x0 (the part the kernels compute) at a tighter 1e-2.
+
+For the long workloads (16 x 60 s, 10 minutes, one hour) the oracle cannot run 32 layers
+over every position, so each check is teacher-forced: the GPU's residual stream after
+layer l (fp32, upcast) is the oracle's input, and the oracle evaluates layer l only at
+sampled positions (with keys and values from every position), which equals the same
+rows of the full layer.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+from gpu_util import rel_l2, to64, weights
+from speech_audio_encoder_b200 import synth
+
+pytestmark = pytest.mark.gpu
+
+EMB_TOL = 2e-2
+
+
+def _api():
+    from speech_audio_encoder_b200 import api
+    return api
+
+
+def _layers64(wf, idx):
+    return {k: v.astype(np.float64) for k, v in wf["layers"][idx].items()}
+
+
+def _global64(wf):
+    # float32 values of bf16 weights; the oracle upcasts each tensor to float64 exactly
+    return wf
+
+
+def test_stack_projection():
+    api = _api()
+    _, wf, dw = weights(2)
+    wave = synth.WORKLOADS["tones_1s"].audio()
+    lm, st = api.sal_frontend(torch.from_numpy(wave).cuda())
+    x = api.sal_stack_project(st, dw)
+    S = to64(st[0])  # the kernel's own bf16 stacked input
+    ref = O.stack_project(S, _global64(wf))
+    got = to64(x)
+    assert np.abs(got - ref).max() <= 1e-4 * np.sqrt(np.mean(ref ** 2)) + 1e-5 * np.abs(ref).max()
+
+
+@pytest.mark.parametrize("batch,T", [(1, 1), (2, 129), (1, 383)])
+def test_one_layer(batch, T):
+    api = _api()
+    _, wf, dw = weights(2)
+    rng = np.random.default_rng(T)
+    x0 = rng.standard_normal((batch * T, 1280)).astype(np.float32)
+    x = torch.from_numpy(x0).cuda()
+    emb = api.sal_encoder_forward(x, batch, T, dw, 1)
+    g = _global64(wf)
+    for b in range(batch):
+        xb = x0[b * T:(b + 1) * T].astype(np.float64)
+        ref1 = O.encoder_layer(xb, g["layers"][0])
+        got1 = to64(x[b * T:(b + 1) * T])
+        assert rel_l2(got1 - xb, ref1 - xb) < 1e-2
+        ref_emb = O.layer_norm(ref1, g["lnf_g"], g["lnf_b"])
+        assert rel_l2(to64(emb[b * T:(b + 1) * T]), ref_emb) < 1e-2
+
+
+def test_sharp_attention_layer():
+    """QK-norm gains of 8: logits of hundreds, attention close to one-hot."""
+    api = _api()
+    _, wf, dw = weights(1, seed=4242, qk_gain_scale=8.0)
+    T = 300
+    rng = np.random.default_rng(5)
+    x0 = rng.standard_normal((T, 1280)).astype(np.float32)
+    x = torch.from_numpy(x0).cuda()
+    api.sal_encoder_forward(x, 1, T, dw, 1)
+    ref1 = O.encoder_layer(x0.astype(np.float64), _layers64(wf, 0))
+    assert rel_l2(to64(x) - x0, ref1 - x0) < 1e-2
+
+
+def test_tones_1s_end_to_end_host_buffers():
+    """sal_encode with a pinned host waveform and a pinned host output."""
+    api = _api()
+    wl = synth.WORKLOADS["tones_1s"]
+    _, wf, dw = weights(wl.n_layers)
+    wave = torch.from_numpy(wl.audio()).pin_memory()
+    T = O.position_count(wl.n_samples)
+    emb = torch.empty((1, T, 1280), dtype=torch.bfloat16).pin_memory()
+    api.sal_encode(wave, dw, wl.n_layers, emb=emb)
+    torch.cuda.synchronize()
+    ref = O.encode(wave.numpy()[0], _global64(wf), wl.n_layers)
+    assert rel_l2(to64(emb[0]), ref) < EMB_TOL
+
+
+def test_clip_30s_32_layers():
+    api = _api()
+    wl = synth.WORKLOADS["clip_30s"]
+    _, wf, dw = weights(wl.n_layers)
+    wave = wl.audio()
+    emb = api.sal_encode(torch.from_numpy(wave).cuda(), dw, wl.n_layers)
+    ref = O.encode(wave[0], _global64(wf), wl.n_layers)
+    err = rel_l2(to64(emb[0]), ref)
+    assert err < EMB_TOL, err
+
+
+def _teacher_forced(name, layers, n_rows, seed):
+    api = _api()
+    wl = synth.WORKLOADS[name]
+    _, wf, dw = weights(wl.n_layers)
+    wave = wl.audio()
+    B, T = wl.batch, O.position_count(wl.n_samples)
+    lm, st = api.sal_frontend(torch.from_numpy(wave).cuda())
+    x0 = api.sal_stack_project(st, dw)
+    ws = api.encoder_workspace(B, T)
+    rng = np.random.default_rng(seed)
+    clips = [0] if B == 1 else [0, B - 1]
+    for l in layers:
+        x = x0.clone()
+        if l > 0:
+            api.sal_encoder_forward(x, B, T, dw, l, workspace=ws)
+        x_in = to64(x)
+        api.sal_encoder_forward(x, B, T, dw.sub(l, 1), 1, workspace=ws)
+        x_out = to64(x)
+        for b in clips:
+            rows = np.sort(rng.choice(T, size=min(n_rows, T), replace=False))
+            rows[0], rows[-1] = 0, T - 1
+            xin_b = x_in[b * T:(b + 1) * T]
+            ref = O.encoder_layer_rows(xin_b, _layers64(wf, l), rows)
+            got = x_out[b * T:(b + 1) * T][rows]
+            err = rel_l2(got - xin_b[rows], ref - xin_b[rows])
+            assert err < 1e-2, (name, l, b, err)
+
+
+def test_batch16_60s_teacher_forced():
+    _teacher_forced("batch16_60s", [0, 31], 256, 1)
+
+
+def test_rec_10min_teacher_forced():
+    _teacher_forced("rec_10min", [0, 15, 31], 256, 2)
+
+
+def test_rec_1h_teacher_forced():
+    _teacher_forced("rec_1h", [31], 128, 3)
+
+
+def test_encoder_rejects_bad_arguments():
+    api = _api()
+    _, _, dw = weights(2)
+    lib = api.lib()
+    import ctypes
+    x = torch.empty((10, 1280), device="cuda")
+    ws = api.encoder_workspace(1, 10)
+    emb = torch.empty((10, 1280), dtype=torch.bfloat16, device="cuda")
+    rec = ctypes.byref(dw.record)
+    assert lib.sal_encoder_forward(x.data_ptr(), 1, 10, rec, 3, emb.data_ptr(), ws.data_ptr(), ws.numel(), 0) == 1
+    assert lib.sal_encoder_forward(x.data_ptr(), 1, 10, rec, 1, emb.data_ptr(), ws.data_ptr(), 256, 0) == 3
+    assert lib.sal_encoder_forward(x.data_ptr(), 1, 45001, rec, 1, emb.data_ptr(), ws.data_ptr(), ws.numel(), 0) == 2

@@ -1,0 +1,158 @@
+"""GPU parity of the single-step entry points (LayerNorm, tensor-core linear layers with
+each epilogue, QKV + QK-norm + RoPE, attention) against the fp64 oracle.
+
+Inputs are bf16 values; the oracle takes the same values upcast to float64, so the only
+differences are the kernels' fp32 accumulation and their final rounding. Tolerances,
+from that arithmetic:
+  * bf16 outputs: |err| <= 2^-8 |ref| + 2e-3 rms(ref)   (one bf16 rounding is <= 2^-9 |ref|;
+    fp32 sums over K <= 5120 products add ~1e-6 relative)
+  * fp32 outputs: |err| <= 1e-4 rms(ref) + 1e-5 |ref|
+  * attention: P is rounded to bf16 before P V, so rel-L2 <= 1e-2 and every element
+    within 2^-7 |ref| + 2e-2 rms(ref).
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+from gpu_util import rand_bf16, rel_l2, to64, weights
+
+pytestmark = pytest.mark.gpu
+
+
+def _api():
+    from speech_audio_encoder_b200 import api
+    return api
+
+
+def _rms(a):
+    return float(np.sqrt(np.mean(np.square(a))))
+
+
+def _assert_bf16_close(got, ref, what):
+    err = np.abs(got - ref)
+    tol = 2.0 ** -8 * np.abs(ref) + 2e-3 * _rms(ref)
+    bad = err > tol
+    assert not bad.any(), f"{what}: {bad.sum()} of {bad.size} outside tolerance, max err {err.max()}"
+
+
+def _assert_f32_close(got, ref, what):
+    err = np.abs(got - ref)
+    tol = 1e-4 * _rms(ref) + 1e-5 * np.abs(ref)
+    bad = err > tol
+    assert not bad.any(), f"{what}: {bad.sum()} of {bad.size} outside tolerance, max err {err.max()}"
+
+
+# ---------------------------------------------------------------- LayerNorm
+
+@pytest.mark.parametrize("rows", [1, 7, 1000])
+def test_layernorm(rows):
+    api = _api()
+    rng = np.random.default_rng(rows)
+    x = (rng.standard_normal((rows, 1280)) * 2 + 0.5).astype(np.float32)
+    g, g64 = rand_bf16((1280,), 1, 0.5)
+    b, b64 = rand_bf16((1280,), 2, 0.5)
+    y = api.sal_layernorm(torch.from_numpy(x).cuda(), g.data_ptr(), b.data_ptr())
+    _assert_bf16_close(to64(y), O.layer_norm(x, g64, b64), "layernorm")
+
+
+# ---------------------------------------------------------------- linear layers
+
+SHAPES = [
+    # M, K, N : small M (narrow tiles, split-K), ragged tails, and M large enough for 256-wide tiles
+    (1, 1280, 1280), (127, 1024, 1280), (129, 1280, 3840), (300, 5120, 1280),
+    (1000, 1280, 5120), (4100, 1280, 1280), (4100, 5120, 1280),
+]
+
+
+@pytest.mark.parametrize("M,K,N", SHAPES)
+@pytest.mark.parametrize("epi", ["f32", "bf16", "gelu", "resid"])
+def test_linear(M, K, N, epi):
+    api = _api()
+    A, A64 = rand_bf16((M, K), 10 + M, 1.0)
+    W, W64 = rand_bf16((N, K), 20 + K, 0.02)
+    bias, b64 = rand_bf16((N,), 30 + N, 0.02)
+    ref = A64 @ W64.T + b64
+    if epi == "f32":
+        out = api.sal_linear(api.SAL_EPI_STORE_F32, A, W, bias)
+        _assert_f32_close(to64(out), ref, "linear f32")
+    elif epi == "bf16":
+        out = api.sal_linear(api.SAL_EPI_STORE_BF16, A, W, bias)
+        _assert_bf16_close(to64(out), ref, "linear bf16")
+    elif epi == "gelu":
+        out = api.sal_linear(api.SAL_EPI_GELU_BF16, A, W, bias)
+        _assert_bf16_close(to64(out), O.gelu(ref), "linear gelu")
+    else:
+        rng = np.random.default_rng(M + N)
+        x0 = rng.standard_normal((M, N)).astype(np.float32)
+        x = torch.from_numpy(x0).cuda()
+        api.sal_linear(api.SAL_EPI_RESID_F32, A, W, bias, out=x)
+        got = to64(x)
+        _assert_f32_close(got - x0, ref, "linear residual (update)")
+
+
+def test_linear_rejects_bad_shapes():
+    api = _api()
+    A, _ = rand_bf16((4, 100), 1)
+    W, _ = rand_bf16((64, 100), 2)
+    bias, _ = rand_bf16((64,), 3)
+    out = torch.empty((4, 64), device="cuda")
+    st = api.lib().sal_linear(0, A.data_ptr(), 4, 100, W.data_ptr(), 64, bias.data_ptr(), out.data_ptr(), 0)
+    assert st == 2  # K not a multiple of 64
+
+
+# ---------------------------------------------------------------- QKV + QK-norm + RoPE
+
+@pytest.mark.parametrize("batch,T", [(1, 1), (2, 7), (1, 129), (3, 300), (1, 3000)])
+def test_qkv_rope(batch, T):
+    api = _api()
+    w, wf, dw = weights(1)
+    lw = {k: v.astype(np.float64) for k, v in wf["layers"][0].items()}
+    h, h64 = rand_bf16((batch * T, 1280), 40 + T, 1.0)
+    q, k, v = api.sal_qkv_rope(h, batch, T, dw.layer(0))
+    qkv = O.linear(h64, lw["w_qkv"], lw["b_qkv"]).reshape(batch, T, 3, 10, 128)
+    pos = np.arange(T)
+    for b in range(batch):
+        qr = O.rope(O.rms_norm(qkv[b, :, 0].transpose(1, 0, 2), lw["qn_g"]), pos)
+        kr = O.rope(O.rms_norm(qkv[b, :, 1].transpose(1, 0, 2), lw["kn_g"]), pos)
+        vr = qkv[b, :, 2].transpose(1, 0, 2)
+        _assert_bf16_close(to64(q[b]), qr, "q")
+        _assert_bf16_close(to64(k[b]), kr, "k")
+        _assert_bf16_close(to64(v[b]), vr, "v")
+
+
+# ---------------------------------------------------------------- attention
+
+@pytest.mark.parametrize("batch,T,scale", [(1, 1, 1.0), (2, 7, 1.0), (1, 128, 1.0), (1, 129, 1.0),
+                                           (2, 383, 1.0), (1, 749, 1.0), (1, 749, 8.0), (1, 2000, 3.0)])
+def test_attention(batch, T, scale):
+    api = _api()
+    q, q64 = rand_bf16((batch, 10, T, 128), 50 + T, scale)
+    k, k64 = rand_bf16((batch, 10, T, 128), 60 + T, 1.0)
+    v, v64 = rand_bf16((batch, 10, T, 128), 70 + T, 1.0)
+    o = api.sal_attention(q, k, v)
+    got = to64(o).reshape(batch, T, 10, 128)
+    for b in range(batch):
+        ref = O.attention(q64[b], k64[b], v64[b]).transpose(1, 0, 2)
+        assert rel_l2(got[b], ref) < 1e-2
+        err = np.abs(got[b] - ref)
+        assert (err <= 2.0 ** -7 * np.abs(ref) + 2e-2 * np.sqrt(np.mean(ref ** 2))).all(), err.max()
+
+
+def test_attention_dominant_key():
+    """Sharp rows: one key aligned with each query selects its value row."""
+    api = _api()
+    T = 300
+    rng = np.random.default_rng(9)
+    qn = rng.standard_normal((1, 10, T, 128))
+    kn = rng.standard_normal((1, 10, T, 128))
+    perm = rng.permutation(T)
+    kn[0, :, perm] = qn[0] * 4.0  # key perm[t] is 4 x query t
+    from speech_audio_encoder_b200 import synth
+    from gpu_util import bf16_tensor
+    qb, kb = synth.bf16_bits(qn), synth.bf16_bits(kn)
+    vb, v64 = rand_bf16((1, 10, T, 128), 11, 1.0)
+    o = api.sal_attention(bf16_tensor(qb), bf16_tensor(kb), vb)
+    ref = O.attention(synth.bf16_to_f32(qb)[0], synth.bf16_to_f32(kb)[0], v64[0]).transpose(1, 0, 2)
+    got = to64(o).reshape(T, 10, 128)
+    assert rel_l2(got, ref) < 1e-2
