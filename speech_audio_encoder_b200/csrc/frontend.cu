@@ -4,7 +4,7 @@
 // (Page "Nemotron 3.5 Transcribe: From Recorded Speech to Dataset Audits", section
 // "How audio and speakers reach the language model", exported-frontend paragraph.)
 //
-// One CTA of 8 warps covers 64 consecutive frames of one clip. Their 160*63 + 400
+// One CTA of 8 warps covers 32 consecutive frames of one clip. Their 160*31 + 400
 // samples are staged in shared memory once (overlapping windows are never re-read from
 // HBM). Each warp then takes one frame at a time:
 //   1. the 400 windowed samples, zero-padded to 512, are packed as 256 complex values
@@ -14,8 +14,11 @@
 //   3. the split step X[k] = E[k] + e^{-2 pi i k/512} O[k], E and O the transforms of
 //      the even and odd samples recovered from Z[k] and conj(Z[256-k]); power |X[k]|^2;
 //   4. 128 sparse triangular filters (504 non-zero weights), ln(max(e, 1e-10)).
-// All arithmetic is fp32; the twiddle, window and filter tables are computed once on
-// the host in double precision.
+// The FFT, power and filter sums run in fp64: a bin 60 dB under the frame's strongest
+// component (the noise floor of a clean tone) carries an fp32 FFT error of ~1e-6 of the
+// frame norm, i.e. a few 1e-4 in its log, above the 1e-4 budget; B200's fp64 rate is half
+// its fp32 rate, so the whole transform stays in double. The twiddle, window and filter
+// tables are computed once on the host in double precision and read through L1.
 #include <cuda_bf16.h>
 #include <math.h>
 
@@ -28,40 +31,38 @@
 namespace sal {
 namespace {
 
-constexpr int kFramesPerCta = 64;
+constexpr int kFramesPerCta = 32;
 constexpr int kWarps = 8;
 constexpr int kFramesPerWarp = kFramesPerCta / kWarps;
-constexpr int kTileSamples = kHop * (kFramesPerCta - 1) + kWin;  // 10480
+constexpr int kTileSamples = kHop * (kFramesPerCta - 1) + kWin;  // 5360
 constexpr int kMelNnz = 504;
 
 struct FrontTables {
-  float2 tw256[256];  // e^{-2 pi i j / 256}
-  float2 tw512[258];  // e^{-2 pi i k / 512}, k = 0..256 (+1 pad)
-  float hann[400];
-  float mel_w[kMelNnz];
-  int mel_meta[128];  // first bin | count << 9 | weight offset << 13
+  double2 tw256[256];  // e^{-2 pi i j / 256}
+  double2 tw512[258];  // e^{-2 pi i k / 512}, k = 0..256 (+1 pad)
+  double hann[400];
+  double mel_w[kMelNnz];
+  int mel_meta[128];   // first bin | count << 9 | weight offset << 13
 };
-static_assert(sizeof(FrontTables) % 16 == 0, "table copy uses 16-byte words");
 
 __device__ FrontTables g_front_tables;
 
-// Per-warp scratch (floats): exchange A is 2 x (8 rows x 36), exchange B is 2 x (64 x 5).
+// Per-warp scratch (doubles): exchange A is 2 x (8 rows x 36), exchange B is 2 x (64 x 5).
 // The spectrum Z (2 x 256) reuses A; the power spectrum (257) reuses B.
 constexpr int kAStride = 36;
-constexpr int kAFloats = 2 * 8 * kAStride;  // 576
-constexpr int kBFloats = 2 * 64 * 5;        // 640
-constexpr int kWarpFloats = kAFloats + kBFloats;
+constexpr int kAElems = 2 * 8 * kAStride;  // 576
+constexpr int kBElems = 2 * 64 * 5;        // 640
+constexpr int kWarpElems = kAElems + kBElems;
 
-constexpr size_t kSmemBytes =
-    sizeof(FrontTables) + sizeof(float) * (kTileSamples + kWarps * kWarpFloats);
+constexpr size_t kSmemBytes = sizeof(float) * kTileSamples + sizeof(double) * kWarps * kWarpElems;
 
 struct C2 {
-  float x, y;
+  double x, y;
 };
 __device__ __forceinline__ C2 cadd(C2 a, C2 b) { return {a.x + b.x, a.y + b.y}; }
 __device__ __forceinline__ C2 csub(C2 a, C2 b) { return {a.x - b.x, a.y - b.y}; }
-__device__ __forceinline__ C2 cmul(C2 a, float2 w) {
-  return {a.x * w.x - a.y * w.y, a.x * w.y + a.y * w.x};
+__device__ __forceinline__ C2 cmul(C2 a, double2 w) {
+  return {fma(a.x, w.x, -a.y * w.y), fma(a.x, w.y, a.y * w.x)};
 }
 __device__ __forceinline__ C2 mul_neg_i(C2 a) { return {a.y, -a.x}; }  // a * (-i)
 __device__ __forceinline__ C2 mul_pos_i(C2 a) { return {-a.y, a.x}; }  // a * (+i)
@@ -81,7 +82,7 @@ __device__ __forceinline__ void dft8(C2 (&v)[8]) {
   C2 e0, e1, e2, e3, o0, o1, o2, o3;
   dft4(v[0], v[2], v[4], v[6], e0, e1, e2, e3);
   dft4(v[1], v[3], v[5], v[7], o0, o1, o2, o3);
-  const float r = 0.70710678118654752f;
+  const double r = 0.70710678118654752440;
   // twiddles e^{-2 pi i k / 8}, k = 1, 2, 3
   o1 = {(o1.x + o1.y) * r, (o1.y - o1.x) * r};
   o2 = mul_neg_i(o2);
@@ -100,9 +101,9 @@ __global__ void __launch_bounds__(256, 2)
     frontend_kernel(const float* __restrict__ wave, int64_t n_samples, int64_t F, int64_t n_stack,
                     float* __restrict__ logmel, __nv_bfloat16* __restrict__ stacked) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
-  FrontTables& tab = *reinterpret_cast<FrontTables*>(smem_raw);
-  float* tile = reinterpret_cast<float*>(smem_raw + sizeof(FrontTables));
-  float* wbuf = tile + kTileSamples;
+  double* wbuf = reinterpret_cast<double*>(smem_raw);
+  float* tile = reinterpret_cast<float*>(smem_raw + sizeof(double) * kWarps * kWarpElems);
+  const FrontTables& tab = g_front_tables;
 
   const int tid = threadIdx.x;
   const int lane = tid & 31;
@@ -112,11 +113,6 @@ __global__ void __launch_bounds__(256, 2)
   const int nf = static_cast<int>(F - f0 < kFramesPerCta ? F - f0 : kFramesPerCta);
   const int nsamp = kHop * (nf - 1) + kWin;  // a multiple of 4
 
-  {  // tables
-    const int4* src = reinterpret_cast<const int4*>(&g_front_tables);
-    int4* dst = reinterpret_cast<int4*>(smem_raw);
-    for (int i = tid; i < static_cast<int>(sizeof(FrontTables) / 16); i += blockDim.x) dst[i] = src[i];
-  }
   {  // samples [160 f0, 160 f0 + nsamp) of this clip, read once
     const int64_t g0 = clip * n_samples + kHop * f0;
     const float* src = wave + g0;
@@ -130,13 +126,13 @@ __global__ void __launch_bounds__(256, 2)
   }
   __syncthreads();
 
-  float* are = wbuf + warp * kWarpFloats;
-  float* aim = are + 8 * kAStride;
-  float* bre = are + kAFloats;
-  float* bim = bre + 64 * 5;
-  float* zre = are;        // Z[k], k < 256 (reuses exchange A)
-  float* zim = are + 256;
-  float* pw = bre;         // |X[k]|^2, k <= 256 (reuses exchange B)
+  double* are = wbuf + warp * kWarpElems;
+  double* aim = are + 8 * kAStride;
+  double* bre = are + kAElems;
+  double* bim = bre + 64 * 5;
+  double* zre = are;        // Z[k], k < 256 (reuses exchange A)
+  double* zim = are + 256;
+  double* pw = bre;         // |X[k]|^2, k <= 256 (reuses exchange B)
 
   for (int i = 0; i < kFramesPerWarp; ++i) {
     const int fl = warp * kFramesPerWarp + i;
@@ -150,16 +146,16 @@ __global__ void __launch_bounds__(256, 2)
       const int s = 64 * n1 + 2 * lane;  // sample index of the real part
       if (s < kWin) {
         const float2 xx = *reinterpret_cast<const float2*>(x + s);
-        const float2 ww = *reinterpret_cast<const float2*>(tab.hann + s);
-        v[n1] = {xx.x * ww.x, xx.y * ww.y};
+        const double2 ww = __ldg(reinterpret_cast<const double2*>(tab.hann + s));
+        v[n1] = {static_cast<double>(xx.x) * ww.x, static_cast<double>(xx.y) * ww.y};
       } else {
-        v[n1] = {0.f, 0.f};
+        v[n1] = {0.0, 0.0};
       }
     }
     dft8(v);
 #pragma unroll
     for (int k1 = 0; k1 < 8; ++k1) {
-      const C2 t = k1 ? cmul(v[k1], tab.tw256[lane * k1]) : v[0];
+      const C2 t = k1 ? cmul(v[k1], __ldg(tab.tw256 + lane * k1)) : v[0];
       are[k1 * kAStride + lane] = t.x;
       aim[k1 * kAStride + lane] = t.y;
     }
@@ -171,10 +167,9 @@ __global__ void __launch_bounds__(256, 2)
 #pragma unroll
       for (int a = 0; a < 8; ++a) v[a] = {are[k1 * kAStride + 4 * a + b], aim[k1 * kAStride + 4 * a + b]};
       dft8(v);
-      __syncwarp();
 #pragma unroll
       for (int c = 0; c < 8; ++c) {
-        const C2 t = (b && c) ? cmul(v[c], tab.tw256[8 * b * c]) : v[c];
+        const C2 t = (b && c) ? cmul(v[c], __ldg(tab.tw256 + 8 * b * c)) : v[c];
         const int p = 8 * c + k1;
         bre[p * 5 + b] = t.x;
         bim[p * 5 + b] = t.y;
@@ -202,13 +197,13 @@ __global__ void __launch_bounds__(256, 2)
       const int k = lane + 32 * h;
       if (k > 256) break;
       const int kk = k & 255, kr = (256 - k) & 255;
-      const float ar = zre[kk], ai = zim[kk], br = zre[kr], bi = -zim[kr];  // b = conj(Z[256-k])
-      const C2 e = {0.5f * (ar + br), 0.5f * (ai + bi)};
+      const double ar = zre[kk], ai = zim[kk], br = zre[kr], bi = -zim[kr];  // b = conj(Z[256-k])
+      const C2 e = {0.5 * (ar + br), 0.5 * (ai + bi)};
       // o = (Z[k] - conj(Z[256-k])) / (2 i)
-      const C2 o = {0.5f * (ai - bi), -0.5f * (ar - br)};
-      const C2 xo = cmul(o, tab.tw512[k]);
-      const float xr = e.x + xo.x, xi = e.y + xo.y;
-      pw[k] = xr * xr + xi * xi;
+      const C2 o = {0.5 * (ai - bi), -0.5 * (ar - br)};
+      const C2 xo = cmul(o, __ldg(tab.tw512 + k));
+      const double xr = e.x + xo.x, xi = e.y + xo.y;
+      pw[k] = fma(xr, xr, xi * xi);
     }
     __syncwarp();
 
@@ -219,11 +214,11 @@ __global__ void __launch_bounds__(256, 2)
 #pragma unroll
     for (int h = 0; h < 4; ++h) {
       const int m = lane + 32 * h;
-      const int meta = tab.mel_meta[m];
+      const int meta = __ldg(tab.mel_meta + m);
       const int k0 = meta & 511, cnt = (meta >> 9) & 15, off = meta >> 13;
-      float e = 0.f;
-      for (int j = 0; j < cnt; ++j) e = fmaf(tab.mel_w[off + j], pw[k0 + j], e);
-      const float lm = logf(fmaxf(e, 1e-10f));
+      double e = 0.0;
+      for (int j = 0; j < cnt; ++j) e = fma(__ldg(tab.mel_w + off + j), pw[k0 + j], e);
+      const float lm = static_cast<float>(log(fmax(e, 1e-10)));
       __stcs(out + m, lm);
       if (sout) sout[m] = __float2bfloat16_rn(lm);
     }
@@ -245,13 +240,9 @@ double mel_to_hz_slaney(double m) {
 
 bool build_tables(FrontTables* t) {
   const double pi = 3.14159265358979323846;
-  for (int j = 0; j < 256; ++j)
-    t->tw256[j] = make_float2(static_cast<float>(std::cos(2 * pi * j / 256.0)),
-                              static_cast<float>(-std::sin(2 * pi * j / 256.0)));
-  for (int k = 0; k < 258; ++k)
-    t->tw512[k] = make_float2(static_cast<float>(std::cos(2 * pi * k / 512.0)),
-                              static_cast<float>(-std::sin(2 * pi * k / 512.0)));
-  for (int n = 0; n < 400; ++n) t->hann[n] = static_cast<float>(0.5 - 0.5 * std::cos(2 * pi * n / 400.0));
+  for (int j = 0; j < 256; ++j) t->tw256[j] = make_double2(std::cos(2 * pi * j / 256.0), -std::sin(2 * pi * j / 256.0));
+  for (int k = 0; k < 258; ++k) t->tw512[k] = make_double2(std::cos(2 * pi * k / 512.0), -std::sin(2 * pi * k / 512.0));
+  for (int n = 0; n < 400; ++n) t->hann[n] = 0.5 - 0.5 * std::cos(2 * pi * n / 400.0);
   // Slaney filters: 130 points equally spaced in mel over 0..8000 Hz.
   double pts[kMels + 2];
   const double mmax = hz_to_mel_slaney(8000.0);
@@ -267,8 +258,8 @@ bool build_tables(FrontTables* t) {
       const double w = std::fmax(0.0, std::fmin(rise, fall)) * norm;
       if (w > 0.0) {
         if (first < 0) first = k;
-        if (k != first + cnt || off >= kMelNnz || cnt >= 15) return false;  // must be contiguous
-        t->mel_w[off + cnt] = static_cast<float>(w);
+        if (k != first + cnt || off + cnt >= kMelNnz || cnt >= 15) return false;  // must be contiguous
+        t->mel_w[off + cnt] = w;
         ++cnt;
       }
     }

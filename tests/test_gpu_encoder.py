@@ -68,8 +68,33 @@ def test_one_layer(batch, T):
         assert rel_l2(to64(emb[b * T:(b + 1) * T]), ref_emb) < 1e-2
 
 
+def _bf16(a):
+    return synth.bf16_to_f32(synth.bf16_bits(a)).astype(np.float64)
+
+
+def _layer_bf16_operands(x, lw):
+    """The oracle layer with every tensor-core operand rounded to bf16 where the GPU path
+    rounds it (LN outputs, q / k / v after norm and RoPE, attention output, GELU output).
+    What remains between this and the GPU is fp32 accumulation and the bf16 P."""
+    T = x.shape[0]
+    h = _bf16(O.layer_norm(x, lw["ln1_g"], lw["ln1_b"]))
+    qkv = O.linear(h, lw["w_qkv"], lw["b_qkv"]).reshape(T, 3, 10, 128).transpose(1, 2, 0, 3)
+    pos = np.arange(T)
+    q = _bf16(O.rope(O.rms_norm(qkv[0], lw["qn_g"]), pos))
+    k = _bf16(O.rope(O.rms_norm(qkv[1], lw["kn_g"]), pos))
+    v = _bf16(qkv[2])
+    o = _bf16(O.attention(q, k, v).transpose(1, 0, 2).reshape(T, 1280))
+    x = x + O.linear(o, lw["w_o"], lw["b_o"])
+    u = _bf16(O.gelu(O.linear(_bf16(O.layer_norm(x, lw["ln2_g"], lw["ln2_b"])), lw["w1"], lw["b1"])))
+    return x + O.linear(u, lw["w2"], lw["b2"])
+
+
 def test_sharp_attention_layer():
-    """QK-norm gains of 8: logits of hundreds, attention close to one-hot."""
+    """QK-norm gains of 8: logits with a standard deviation near 64, attention close to
+    one-hot. Rounding q and k to bf16 (2^-9 relative) moves such logits by ~0.2, which
+    reorders near-ties, so against the exact oracle the layer update is held to the
+    embedding bar 2e-2 (rel-L2); against the oracle with the same bf16 operand roundings
+    it is held to 1e-2."""
     api = _api()
     _, wf, dw = weights(1, seed=4242, qk_gain_scale=8.0)
     T = 300
@@ -77,8 +102,12 @@ def test_sharp_attention_layer():
     x0 = rng.standard_normal((T, 1280)).astype(np.float32)
     x = torch.from_numpy(x0).cuda()
     api.sal_encoder_forward(x, 1, T, dw, 1)
-    ref1 = O.encoder_layer(x0.astype(np.float64), _layers64(wf, 0))
-    assert rel_l2(to64(x) - x0, ref1 - x0) < 1e-2
+    lw = _layers64(wf, 0)
+    got = to64(x) - x0
+    exact = O.encoder_layer(x0.astype(np.float64), lw) - x0
+    same_rounding = _layer_bf16_operands(x0.astype(np.float64), lw) - x0
+    assert rel_l2(got, exact) < EMB_TOL
+    assert rel_l2(got, same_rounding) < 1e-2
 
 
 def test_tones_1s_end_to_end_host_buffers():

@@ -147,7 +147,7 @@ def test_attention_dominant_key():
     qn = rng.standard_normal((1, 10, T, 128))
     kn = rng.standard_normal((1, 10, T, 128))
     perm = rng.permutation(T)
-    kn[0, :, perm] = qn[0] * 4.0  # key perm[t] is 4 x query t
+    kn[0][:, perm] = qn[0] * 4.0  # key perm[t] is 4 x query t
     from speech_audio_encoder_b200 import synth
     from gpu_util import bf16_tensor
     qb, kb = synth.bf16_bits(qn), synth.bf16_bits(kn)
