@@ -1,0 +1,468 @@
+#!/usr/bin/env python
+"""Throughput of the speech front end + 32-layer ASR encoder on B200: audio seconds encoded
+per second, with the dominant kernel's roofline, an end-to-end number through the C-ABI
+with host buffers, and the fp64 oracle timed on the host cores.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl sal|reference]
+
+One step = sal_frontend + sal_stack_project + sal_encoder_forward over one batch of the
+workload's synthetic audio, inputs resident in HBM, replayed as one CUDA graph. Between
+timed steps a 256 MiB buffer (twice the 126 MB L2) is rewritten, outside the timed events.
+For N > 1 (torchrun), every rank encodes its own copy of the workload (clips are
+independent; no collective on the data path) and the job's time is the max over ranks.
+Prints ONE JSON line on rank 0.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from speech_audio_encoder_b200 import synth  # noqa: E402
+
+METRIC = "audio-sec encoded/sec (frontend+32-layer encoder, bf16) on 1 B200; % TC peak"
+UNIT = "audio-s/s"
+DEFAULT_WORKLOAD = "clip_30s"
+FLUSH_BYTES = 256 << 20
+
+GEMM_FLOPS_PER_POS_LAYER = 2 * (4 * 1280 * 1280 + 2 * 1280 * 5120)  # 39,321,600
+STACK_PROJ_FLOPS_PER_POS = 2 * 1024 * 1280
+ATTN_FLOPS_PER_T2_LAYER = 4 * 1280  # QK^T and PV over all heads: 4 T^2 * width
+
+
+def positions(n_samples: int) -> int:
+    f = 0 if n_samples < 400 else 1 + (n_samples - 400) // 160
+    return f // 8
+
+
+def frames(n_samples: int) -> int:
+    return 0 if n_samples < 400 else 1 + (n_samples - 400) // 160
+
+
+def kernel_flops(kind: str, B: int, T: int) -> float:
+    """Algorithmic flops of ONE launch of a kernel kind (all clips of the batch)."""
+    M = B * T
+    return {
+        "qkv": 2.0 * M * 1280 * 3840,
+        "out_proj": 2.0 * M * 1280 * 1280,
+        "ffn_up": 2.0 * M * 1280 * 5120,
+        "ffn_down": 2.0 * M * 5120 * 1280,
+        "attention": float(ATTN_FLOPS_PER_T2_LAYER) * T * T * B,
+    }.get(kind, 0.0)
+
+
+def kernel_bytes(kind: str, B: int, T: int) -> float:
+    """Algorithmic HBM bytes of ONE launch of a memory-bound kernel kind."""
+    M = B * T
+    return {
+        "layernorm": M * 1280 * (4 + 2) + 2 * 1280 * 2,
+        "rope_table": T * 64 * 2 * 4,
+    }.get(kind, 0.0)
+
+
+def workload_flops(B: int, T: int, L: int) -> float:
+    return (GEMM_FLOPS_PER_POS_LAYER * B * T * L + ATTN_FLOPS_PER_T2_LAYER * T * T * B * L
+            + STACK_PROJ_FLOPS_PER_POS * B * T)
+
+
+# ----------------------------------------------------------------------------- distributed
+
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def reduce_max(value: float, device=None) -> float:
+    """Max of a float over all ranks (identity when not distributed)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return value
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(audio_seconds_per_rank: float, n_ranks: int, max_seconds: float) -> float:
+    """Whole-job audio seconds per second: every rank's audio over the slowest rank's time."""
+    return audio_seconds_per_rank * n_ranks / max_seconds
+
+
+def rank_seed_offset(rank: int) -> int:
+    """Each rank encodes its own clips: audio seeds are offset by 1000 per rank."""
+    return 1000 * rank
+
+
+# ----------------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    REASONS = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+
+    def __init__(self, gpu_id: str):
+        self.gpu_id = gpu_id
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.QUERY}", "--format=csv,noheader,nounits",
+                 "-lms", "50", "-i", self.gpu_id],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        time.sleep(0.1)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        sm, smax, power, reasons = [], [], [], set()
+        for line in open(self.path):
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                smax.append(float(f[2]))
+                power.append(float(f[3]))
+            except ValueError:
+                continue
+            for name, v in zip(self.REASONS, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(name)
+        os.unlink(self.path)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": sorted(reasons), "samples": 0}
+        # samples under load: power above the midpoint of the observed range
+        pmid = (min(power) + max(power)) / 2
+        loaded = [s for s, p in zip(sm, power) if p >= pmid] or sm
+        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": max(smax),
+                "reasons": sorted(reasons), "samples": len(sm), "power_w_max": max(power)}
+
+
+# ----------------------------------------------------------------------------- oracle timing
+
+def oracle_step_estimate(wl: synth.Workload, budget_s: float, audio: np.ndarray,
+                         weights_f32: dict | None = None):
+    """Time the fp64 oracle on a bounded sample of one step and extrapolate to the whole step.
+
+    The sample: the front end on up to ``fe_frames`` frames of one clip; one encoder layer on a
+    sub-clip of ``Ts`` positions, repeated while the budget lasts (attention timed apart, so the
+    linear part scales with positions and the attention part with positions squared). Returns
+    (estimated seconds per step, description, seconds actually spent, threads used).
+    """
+    import oracle as O
+    from threadpoolctl import threadpool_info
+
+    threads = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+    t_start = time.perf_counter()
+    F, T, B, L = frames(wl.n_samples), positions(wl.n_samples), wl.batch, wl.n_layers
+    fe_frames = max(1, min(F, int(4000 * budget_s)))
+    t0 = time.perf_counter()
+    O.log_mel(audio, first=0, count=fe_frames)
+    t_fe = (time.perf_counter() - t0) * (B * F / fe_frames)
+    if weights_f32 is None:
+        weights_f32 = synth.weights_f32(synth.make_weights(1))
+    lw = weights_f32["layers"][0]
+    Ts = max(1, min(T, 374))
+    rng = np.random.default_rng(0)
+    x = rng.standard_normal((Ts, 1280))
+    q = rng.standard_normal((10, Ts, 128))
+    t_layer, t_attn, reps = [], [], 0
+    while True:
+        t0 = time.perf_counter()
+        O.encoder_layer(x, lw)
+        t_layer.append(time.perf_counter() - t0)
+        t0 = time.perf_counter()
+        O.attention(q, q, q)
+        t_attn.append(time.perf_counter() - t0)
+        reps += 1
+        if time.perf_counter() - t_start > budget_s:
+            break
+    tl, ta = float(np.median(t_layer)), float(np.median(t_attn))
+    ta = min(ta, tl)
+    t_lin = tl - ta
+    t_proj = t_lin * (STACK_PROJ_FLOPS_PER_POS / GEMM_FLOPS_PER_POS_LAYER)
+    est = t_fe + B * (T / Ts) * (L * t_lin + t_proj) + B * L * ta * (T / Ts) ** 2
+    spent = time.perf_counter() - t_start
+    desc = (f"front end on {fe_frames} of {F} frames of one clip; one encoder layer on {Ts} of {T} "
+            f"positions, {reps} run(s), attention timed apart; scaled to {B} clip(s) x {L} layers "
+            f"by flop count")
+    return est, desc, spent, threads
+
+
+# ----------------------------------------------------------------------------- reference arm
+
+def run_reference(args, wl: synth.Workload) -> dict | None:
+    world, rank, _ = dist_env()
+    if rank != 0:
+        return None
+    budget = max(0.05, 120.0 / max(1, args.steps + args.warmup))
+    wf = synth.weights_f32(synth.make_weights(1))
+    audio = synth.Workload(wl.name, 1, wl.n_samples, wl.n_layers, wl.kind, wl.seed).audio()[0]
+    for _ in range(args.warmup):
+        oracle_step_estimate(wl, budget, audio, wf)
+    ests, spent_total, desc, threads = [], 0.0, "", 1
+    for _ in range(args.steps):
+        est, desc, spent, threads = oracle_step_estimate(wl, budget, audio, wf)
+        ests.append(est)
+        spent_total += spent
+    sec = float(np.mean(ests))
+    value = wl.audio_seconds / sec
+    return {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": sec * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic",
+        "config": {"workload": wl.name, "batch": wl.batch, "n_samples": wl.n_samples,
+                   "positions": positions(wl.n_samples), "layers": wl.n_layers,
+                   "parallelism": "host cores, rank 0 only"},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
+                         "sample": desc + f"; {args.steps} samples, {spent_total:.1f} s of CPU work"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+# ----------------------------------------------------------------------------- GPU arm
+
+def run_sal(args, wl: synth.Workload) -> dict | None:
+    import torch
+    import torch.distributed as dist
+
+    from speech_audio_encoder_b200 import api
+
+    world, rank, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+
+    B, N, L = wl.batch, wl.n_samples, wl.n_layers
+    T, F = positions(N), frames(N)
+    my_wl = synth.Workload(wl.name, B, N, L, wl.kind, wl.seed + rank_seed_offset(rank))
+    audio = my_wl.audio()
+    w = synth.make_weights(L)
+    dw = api.DeviceWeights(w, device=dev)
+
+    s = torch.cuda.Stream(device=dev)
+    wave_d = torch.from_numpy(audio).to(dev)
+    logmel = torch.empty((B, F, 128), dtype=torch.float32, device=dev)
+    stacked = torch.empty((B, T, 1024), dtype=torch.bfloat16, device=dev)
+    x = torch.empty((B * T, 1280), dtype=torch.float32, device=dev)
+    emb = torch.empty((B * T, 1280), dtype=torch.bfloat16, device=dev)
+    ws = api.encoder_workspace(B, T, dev)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    lib = api.lib()
+    import ctypes
+    rec = ctypes.byref(dw.record)
+    sp = s.cuda_stream
+
+    def step(stream_ptr=sp):
+        api._check("sal_frontend", lib.sal_frontend(wave_d.data_ptr(), N, B, logmel.data_ptr(),
+                                                    stacked.data_ptr(), stream_ptr))
+        api._check("sal_stack_project", lib.sal_stack_project(stacked.data_ptr(), B, T, rec,
+                                                              x.data_ptr(), stream_ptr))
+        api._check("sal_encoder_forward", lib.sal_encoder_forward(
+            x.data_ptr(), B, T, rec, L, emb.data_ptr(), ws.data_ptr(), ws.numel(), stream_ptr))
+
+    with torch.cuda.stream(s):
+        for _ in range(max(args.warmup, 3)):
+            step()
+    s.synchronize()
+    if api.sal_last_device_status(s) != 0:
+        raise RuntimeError("device wait timed out during warm-up")
+
+    graph = torch.cuda.CUDAGraph()
+    n0 = api.sal_launch_count()
+    with torch.cuda.graph(graph, stream=s):
+        step(torch.cuda.current_stream().cuda_stream)
+    launches_per_step = api.sal_launch_count() - n0
+    for _ in range(3):
+        graph.replay()
+    torch.cuda.synchronize()
+
+    # ---- timed region
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    gpu_id = _nvsmi_id(local)
+    clocks = ClockSampler(gpu_id)
+    clocks.start()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with torch.cuda.stream(s):
+        for k in range(args.steps):
+            flush.fill_(k & 0xFF)
+            ev[k][0].record(s)
+            graph.replay()
+            ev[k][1].record(s)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clk = clocks.stop()
+    step_ms = [a.elapsed_time(b) for a, b in ev]
+    total_s = sum(step_ms) / 1e3
+    total_s = reduce_max(total_s, dev)
+    if api.sal_last_device_status(s) != 0:
+        raise RuntimeError("device wait timed out during the timed region")
+    value = job_throughput(my_wl.audio_seconds * args.steps, world, total_s)
+    flops_step = workload_flops(B, T, L)
+
+    # ---- per-kind launch durations (events around each launch, traced graph replays)
+    kinds = {}
+    k_steps = max(3, min(args.steps, 20))
+    for kind_id, kind in enumerate(api.KIND_NAMES):
+        per_step = {"rope_table": 1, "layernorm": 2 * L + 1}.get(kind, L)
+        evs = [torch.cuda.Event(enable_timing=True) for _ in range(2 * per_step)]
+        for e in evs:  # torch creates the CUDA event on its first record
+            e.record(s)
+        s.synchronize()
+        g2 = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g2, stream=s):
+            cs = torch.cuda.current_stream().cuda_stream
+            api._check("sal_frontend", lib.sal_frontend(wave_d.data_ptr(), N, B, logmel.data_ptr(),
+                                                        stacked.data_ptr(), cs))
+            api._check("sal_stack_project", lib.sal_stack_project(stacked.data_ptr(), B, T, rec,
+                                                                  x.data_ptr(), cs))
+            api.sal_encoder_forward_traced(x, B, T, dw, L, ws, emb, kind_id, evs, stream=cs)
+        durs = []
+        with torch.cuda.stream(s):
+            for _ in range(k_steps):
+                flush.fill_(1)
+                g2.replay()
+                s.synchronize()
+                durs += [evs[2 * i].elapsed_time(evs[2 * i + 1]) for i in range(per_step)]
+        kinds[kind] = {"launches_per_step": per_step, "avg_ms": float(np.mean(durs)),
+                       "ms_per_step": float(np.mean(durs)) * per_step}
+        del g2
+    step_ms_mean = total_s * 1e3 / args.steps
+    for k in kinds.values():
+        k["share"] = k["ms_per_step"] / step_ms_mean
+    tensor_kinds = ["qkv", "attention", "out_proj", "ffn_up", "ffn_down"]
+    dom = max(tensor_kinds, key=lambda k: kinds[k]["ms_per_step"])
+    peaks = _peaks()
+    achieved = kernel_flops(dom, B, T) / (kinds[dom]["avg_ms"] / 1e3) / 1e12
+    roofline = {"kernel": dom, "bound": "tensor", "achieved": achieved, "peak": peaks["tflops"],
+                "unit": "TFLOP/s", "frac": achieved / peaks["tflops"], "traffic": None,
+                "peak_source": peaks["tflops_source"],
+                "per_launch_flops": kernel_flops(dom, B, T), "avg_launch_ms": kinds[dom]["avg_ms"]}
+
+    # ---- end to end through sal_encode with pinned host buffers
+    e2e = None
+    if not args.no_e2e:
+        wave_h = torch.from_numpy(audio).pin_memory()
+        emb_h = torch.empty((B, T, 1280), dtype=torch.bfloat16).pin_memory()
+        ews = api.encode_workspace(B, N, dev)
+        with torch.cuda.stream(s):
+            for _ in range(3):
+                api.sal_encode(wave_h, dw, L, emb=emb_h, workspace=ews, stream=s)
+        s.synchronize()
+        n_e2e = max(3, min(args.steps, 50))
+        t_e2e = []
+        with torch.cuda.stream(s):
+            for _ in range(n_e2e):
+                flush.fill_(2)
+                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                a.record(s)
+                api.sal_encode(wave_h, dw, L, emb=emb_h, workspace=ews, stream=s)
+                b.record(s)
+                b.synchronize()  # the result is on the host
+                t_e2e.append(a.elapsed_time(b))
+        e2e_s = reduce_max(sum(t_e2e) / 1e3, dev)
+        e2e = {"value": job_throughput(my_wl.audio_seconds * n_e2e, world, e2e_s), "unit": UNIT,
+               "h2d_bytes_per_step": B * N * 4, "d2h_bytes_per_step": B * T * 1280 * 2,
+               "steps": n_e2e, "call": "sal_encode (pinned host wave in, pinned host embeddings out)"}
+
+    # ---- oracle on the host cores (rank 0, one GPU only)
+    cpu = None
+    if world == 1 and not args.no_cpu_baseline:
+        est, desc, spent, threads = oracle_step_estimate(wl, 15.0, audio[0])
+        cpu = {"value": wl.audio_seconds / est, "unit": UNIT, "cores": threads, "kind": "oracle",
+               "sample": desc + f"; {spent:.1f} s of CPU work"}
+
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return None
+    return {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": step_ms_mean, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": wl.name, "batch": B, "n_samples": N, "positions": T, "layers": L,
+                   "parallelism": f"dp{world} (independent clips per GPU)" if world > 1 else "single GPU",
+                   "l2": "256 MiB buffer rewritten between timed steps", "graph": "one CUDA graph per step"},
+        "tc_frac_step": flops_step / (step_ms_mean / 1e3) / 1e12 / peaks["tflops"],
+        "roofline": roofline,
+        "kernels": kinds,
+        "cpu_baseline": cpu,
+        "e2e": e2e,
+        "gpu_launches": int(launches_per_step * args.steps),
+        "clocks": clk,
+    }
+
+
+def _nvsmi_id(local: int) -> str:
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+    if vis:
+        ids = [v.strip() for v in vis.split(",") if v.strip()]
+        if local < len(ids):
+            return ids[local]
+    return str(local)
+
+
+def _peaks() -> dict:
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        p = json.load(open(path))
+        return {"tflops": float(p["bf16_tflops_sustained"]), "tflops_source": "measured (sustained bf16)",
+                "gbs": float(p["hbm_gbs"]), "gbs_source": "measured"}
+    except (OSError, KeyError, ValueError):
+        return {"tflops": 1400.0, "tflops_source": "fallback (sustained bf16)", "gbs": 6650.0,
+                "gbs_source": "fallback"}
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=300)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=synth.WORKLOAD_ORDER)
+    ap.add_argument("--impl", default="sal", choices=["sal", "reference"])
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+    wl = synth.WORKLOADS[args.workload]
+    out = run_reference(args, wl) if args.impl == "reference" else run_sal(args, wl)
+    if out is not None:
+        print(json.dumps(out), flush=True)
+
+
+if __name__ == "__main__":
+    main()

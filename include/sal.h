@@ -136,6 +136,36 @@ size_t sal_encode_workspace_bytes(int batch, int64_t n_samples);
 sal_status sal_encode(const float* wave, int64_t n_samples, int batch, const sal_weights* w,
                       int n_layers, void* emb, void* workspace, size_t ws_bytes, void* stream);
 
+/* Kinds of kernel launch, for sal_encoder_forward_traced. */
+typedef enum {
+    SAL_KIND_ROPE_TABLE = 0,
+    SAL_KIND_LAYERNORM = 1, /* LN1, LN2 and the final LN */
+    SAL_KIND_QKV = 2,       /* QKV GEMM + QK-norm + RoPE epilogue */
+    SAL_KIND_ATTENTION = 3,
+    SAL_KIND_OUT_PROJ = 4,  /* attention output projection + residual */
+    SAL_KIND_FFN_UP = 5,    /* FFN up + GELU */
+    SAL_KIND_FFN_DOWN = 6,  /* FFN down + residual */
+    SAL_KIND_COUNT = 7
+} sal_kernel_kind;
+
+/* Event trace: for the i-th launch of kind `kind` inside the call (i < n_events / 2),
+ * events[2 i] is recorded on the stream just before it and events[2 i + 1] just after.
+ * Events are cudaEvent_t handles created by the caller. */
+typedef struct {
+    int kind;
+    void* const* events;
+    int n_events;
+} sal_trace;
+
+/* sal_encoder_forward with an optional event trace (trace may be NULL). */
+sal_status sal_encoder_forward_traced(float* x, int batch, int64_t T, const sal_weights* w,
+                                      int n_layers, void* emb, void* workspace, size_t ws_bytes,
+                                      void* stream, const sal_trace* trace);
+
+/* Kernel launches this library has enqueued since the process started (all devices and
+ * streams; a launch captured into a CUDA graph counts once, at capture). */
+uint64_t sal_launch_count(void);
+
 /* Synchronises `stream` and reports (then clears) the device status word that bounded
  * waits set when they give up: SAL_OK or SAL_ETIMEOUT. */
 sal_status sal_last_device_status(void* stream);

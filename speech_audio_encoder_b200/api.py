@@ -41,6 +41,13 @@ class sal_weights(ctypes.Structure):
                 ("lnf_g", ctypes.c_void_p), ("lnf_b", ctypes.c_void_p)]
 
 
+class sal_trace(ctypes.Structure):
+    _fields_ = [("kind", ctypes.c_int), ("events", ctypes.POINTER(ctypes.c_void_p)),
+                ("n_events", ctypes.c_int)]
+
+
+KIND_NAMES = ["rope_table", "layernorm", "qkv", "attention", "out_proj", "ffn_up", "ffn_down"]
+
 EXPORTS = {
     # name: (restype, argtypes)
     "sal_frame_count": (ctypes.c_int64, [ctypes.c_int64]),
@@ -54,6 +61,11 @@ EXPORTS = {
     "sal_encoder_forward": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int, ctypes.c_int64,
                                             ctypes.POINTER(sal_weights), ctypes.c_int, ctypes.c_void_p,
                                             ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]),
+    "sal_encoder_forward_traced": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int, ctypes.c_int64,
+                                                   ctypes.POINTER(sal_weights), ctypes.c_int, ctypes.c_void_p,
+                                                   ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p,
+                                                   ctypes.POINTER(sal_trace)]),
+    "sal_launch_count": (ctypes.c_uint64, []),
     "sal_encode_workspace_bytes": (ctypes.c_size_t, [ctypes.c_int, ctypes.c_int64]),
     "sal_encode": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.POINTER(sal_weights),
                                    ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_size_t,
@@ -214,6 +226,25 @@ def sal_encoder_forward(x: torch.Tensor, batch: int, T: int, weights, n_layers: 
         _ptr(x), batch, T, ctypes.byref(rec), n_layers, _ptr(emb), _ptr(workspace),
         workspace.numel(), _stream(stream)))
     return emb
+
+
+def sal_encoder_forward_traced(x: torch.Tensor, batch: int, T: int, weights, n_layers: int,
+                               workspace: torch.Tensor, emb: torch.Tensor, kind: int, events,
+                               stream=None) -> torch.Tensor:
+    """sal_encoder_forward with torch.cuda.Event pairs recorded around each launch of ``kind``."""
+    rec = weights.record if isinstance(weights, DeviceWeights) else weights
+    if any(e.cuda_event == 0 for e in events):
+        raise ValueError("record each torch.cuda.Event once before tracing (its handle is created lazily)")
+    handles = (ctypes.c_void_p * len(events))(*[e.cuda_event for e in events])
+    tr = sal_trace(kind, ctypes.cast(handles, ctypes.POINTER(ctypes.c_void_p)), len(events))
+    _check("sal_encoder_forward_traced", lib().sal_encoder_forward_traced(
+        _ptr(x), batch, T, ctypes.byref(rec), n_layers, _ptr(emb), _ptr(workspace), workspace.numel(),
+        _stream(stream), ctypes.byref(tr)))
+    return emb
+
+
+def sal_launch_count() -> int:
+    return int(lib().sal_launch_count())
 
 
 def encode_workspace(batch: int, n_samples: int, device="cuda") -> torch.Tensor:

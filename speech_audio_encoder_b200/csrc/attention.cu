@@ -315,6 +315,7 @@ sal_status attention_launch(const void* q, const void* k, const void* v, int bat
   a.status = device_status_ptr();
   if (!a.status) return SAL_ECUDA;
   const dim3 grid(static_cast<unsigned>((T + kTile - 1) / kTile), static_cast<unsigned>(bh));
+  count_launch();
   attention_kernel<<<grid, 192, kSmem, s>>>(tq, tk, tv, a);
   return cudaGetLastError() == cudaSuccess ? SAL_OK : SAL_ECUDA;
 }

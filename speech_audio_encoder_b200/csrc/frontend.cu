@@ -301,6 +301,7 @@ sal_status frontend_launch(const float* wave, int64_t n_samples, int batch, int6
   if (st != SAL_OK) return st;
   const dim3 grid(static_cast<unsigned>((frames + kFramesPerCta - 1) / kFramesPerCta),
                   static_cast<unsigned>(batch));
+  count_launch();
   frontend_kernel<<<grid, 256, kSmemBytes, s>>>(wave, n_samples, frames,
                                                 stacked ? positions * kStack : 0, logmel,
                                                 static_cast<__nv_bfloat16*>(stacked));

@@ -384,6 +384,7 @@ sal_status launch_bn(const GemmArgs& a, const void* A, const void* W, cudaStream
   if (!make_tmap_2d_bf16(&tb, W, a.K, a.N, C::BK, BN)) return SAL_ECUDA;
   const int tiles = static_cast<int>((a.M + C::BM - 1) / C::BM) * (a.N / BN) * a.splits;
   const int grid = tiles < num_sms() ? tiles : num_sms();
+  count_launch();
   gemm_kernel<BN, EPI><<<grid, 192, C::SMEM, s>>>(ta, tb, a);
   return cudaGetLastError() == cudaSuccess ? SAL_OK : SAL_ECUDA;
 }

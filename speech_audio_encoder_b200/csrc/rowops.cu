@@ -84,6 +84,7 @@ sal_status layernorm_launch(const float* x, int64_t rows, const void* g, const v
                             cudaStream_t s) {
   if (rows == 0) return SAL_OK;
   const unsigned grid = static_cast<unsigned>((rows + kLnWarps - 1) / kLnWarps);
+  count_launch();
   layernorm_kernel<<<grid, 32 * kLnWarps, 0, s>>>(x, rows, static_cast<const __nv_bfloat16*>(g),
                                                   static_cast<const __nv_bfloat16*>(b),
                                                   static_cast<__nv_bfloat16*>(y));
@@ -93,6 +94,7 @@ sal_status layernorm_launch(const float* x, int64_t rows, const void* g, const v
 sal_status rope_table_launch(float* cs, int64_t T, cudaStream_t s) {
   if (T == 0) return SAL_OK;
   const int64_t n = T * 64;
+  count_launch();
   rope_table_kernel<<<static_cast<unsigned>((n + 255) / 256), 256, 0, s>>>(cs, T);
   return cudaGetLastError() == cudaSuccess ? SAL_OK : SAL_ECUDA;
 }

@@ -28,6 +28,7 @@ __device__ unsigned int g_status = 0;
 namespace {
 
 std::atomic<uint64_t> g_wait_limit_ns{4000000000ull};
+std::atomic<uint64_t> g_launches{0};
 
 PFN_cuTensorMapEncodeTiled_v12000 g_encode_tiled = nullptr;
 std::once_flag g_encode_once;
@@ -109,6 +110,8 @@ bool is_device_ptr(const void* p) {
 }  // namespace
 
 uint64_t wait_limit_ns() { return g_wait_limit_ns.load(); }
+
+void count_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
 
 unsigned int* device_status_ptr() {
   static std::mutex mu;
@@ -222,6 +225,41 @@ size_t sal_encoder_workspace_bytes(int batch, int64_t T) {
 
 sal_status sal_encoder_forward(float* x, int batch, int64_t T, const sal_weights* w, int n_layers, void* emb,
                                void* workspace, size_t ws_bytes, void* stream) {
+  return sal_encoder_forward_traced(x, batch, T, w, n_layers, emb, workspace, ws_bytes, stream, nullptr);
+}
+
+namespace {
+// Records trace events around the launches of one kind (as event-record nodes when the
+// stream is being captured into a CUDA graph).
+struct Tracer {
+  const sal_trace* tr;
+  cudaStream_t s;
+  int seen = 0;
+  bool before(int kind) {
+    if (!tr || tr->kind != kind || 2 * seen + 1 >= tr->n_events) return true;
+    return cudaEventRecordWithFlags(static_cast<cudaEvent_t>(tr->events[2 * seen]), s, cudaEventRecordExternal) ==
+           cudaSuccess;
+  }
+  bool after(int kind) {
+    if (!tr || tr->kind != kind || 2 * seen + 1 >= tr->n_events) return true;
+    const bool ok = cudaEventRecordWithFlags(static_cast<cudaEvent_t>(tr->events[2 * seen + 1]), s,
+                                            cudaEventRecordExternal) == cudaSuccess;
+    ++seen;
+    return ok;
+  }
+};
+}  // namespace
+
+#define SAL_TRACED(kind, expr)                              \
+  do {                                                      \
+    if (!tr.before(kind)) return SAL_ECUDA;                 \
+    SAL_TRY(expr);                                          \
+    if (!tr.after(kind)) return SAL_ECUDA;                  \
+  } while (0)
+
+sal_status sal_encoder_forward_traced(float* x, int batch, int64_t T, const sal_weights* w, int n_layers,
+                                      void* emb, void* workspace, size_t ws_bytes, void* stream,
+                                      const sal_trace* trace) {
   if (batch < 0 || T < 0 || !w || n_layers < 0 || n_layers > w->n_layers) return SAL_EINVAL;
   if (T > SAL_MAX_POSITIONS) return SAL_ESHAPE;
   if (batch == 0 || T == 0) return SAL_OK;
@@ -232,25 +270,34 @@ sal_status sal_encoder_forward(float* x, int batch, int64_t T, const sal_weights
   for (int i = 0; i < n_layers; ++i)
     if (!layer_ok(w->layers[i])) return SAL_EINVAL;
   if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u)) return SAL_EINVAL;
+  if (trace && (trace->kind < 0 || trace->kind >= SAL_KIND_COUNT || trace->n_events < 0 ||
+                (trace->n_events > 0 && !trace->events)))
+    return SAL_EINVAL;
   const EncoderWs ws = encoder_ws_layout(workspace, batch, T);
   if (ws_bytes < ws.bytes) return SAL_EWORKSPACE;
   SAL_TRY(check_device());
   cudaStream_t s = static_cast<cudaStream_t>(stream);
+  Tracer tr{trace, s};
   const int64_t M = static_cast<int64_t>(batch) * T;
-  if (n_layers > 0) SAL_TRY(rope_table_launch(ws.rope, T, s));
+  if (n_layers > 0) SAL_TRACED(SAL_KIND_ROPE_TABLE, rope_table_launch(ws.rope, T, s));
   for (int i = 0; i < n_layers; ++i) {
     const sal_layer& L = w->layers[i];
-    SAL_TRY(layernorm_launch(x, M, L.ln1_g, L.ln1_b, ws.h, s));
+    SAL_TRACED(SAL_KIND_LAYERNORM, layernorm_launch(x, M, L.ln1_g, L.ln1_b, ws.h, s));
     QkvOut qo{ws.q, ws.k, ws.v, L.qn_g, L.kn_g, ws.rope, T};
-    SAL_TRY(gemm_launch(kEpiQkv, ws.h, M, kWidth, L.w_qkv, 3 * kWidth, L.b_qkv, nullptr, &qo, s));
-    SAL_TRY(attention_launch(ws.q, ws.k, ws.v, batch, T, ws.o, s));
-    SAL_TRY(gemm_launch(SAL_EPI_RESID_F32, ws.o, M, kWidth, L.w_o, kWidth, L.b_o, x, nullptr, s));
-    SAL_TRY(layernorm_launch(x, M, L.ln2_g, L.ln2_b, ws.h, s));
-    SAL_TRY(gemm_launch(SAL_EPI_GELU_BF16, ws.h, M, kWidth, L.w1, kFfn, L.b1, ws.u, nullptr, s));
-    SAL_TRY(gemm_launch(SAL_EPI_RESID_F32, ws.u, M, kFfn, L.w2, kWidth, L.b2, x, nullptr, s));
+    SAL_TRACED(SAL_KIND_QKV, gemm_launch(kEpiQkv, ws.h, M, kWidth, L.w_qkv, 3 * kWidth, L.b_qkv, nullptr, &qo, s));
+    SAL_TRACED(SAL_KIND_ATTENTION, attention_launch(ws.q, ws.k, ws.v, batch, T, ws.o, s));
+    SAL_TRACED(SAL_KIND_OUT_PROJ,
+               gemm_launch(SAL_EPI_RESID_F32, ws.o, M, kWidth, L.w_o, kWidth, L.b_o, x, nullptr, s));
+    SAL_TRACED(SAL_KIND_LAYERNORM, layernorm_launch(x, M, L.ln2_g, L.ln2_b, ws.h, s));
+    SAL_TRACED(SAL_KIND_FFN_UP, gemm_launch(SAL_EPI_GELU_BF16, ws.h, M, kWidth, L.w1, kFfn, L.b1, ws.u, nullptr, s));
+    SAL_TRACED(SAL_KIND_FFN_DOWN,
+               gemm_launch(SAL_EPI_RESID_F32, ws.u, M, kFfn, L.w2, kWidth, L.b2, x, nullptr, s));
   }
-  return layernorm_launch(x, M, w->lnf_g, w->lnf_b, emb, s);
+  SAL_TRACED(SAL_KIND_LAYERNORM, layernorm_launch(x, M, w->lnf_g, w->lnf_b, emb, s));
+  return SAL_OK;
 }
+
+uint64_t sal_launch_count(void) { return g_launches.load(); }
 
 size_t sal_encode_workspace_bytes(int batch, int64_t n_samples) {
   if (batch <= 0 || n_samples < 0) return 0;

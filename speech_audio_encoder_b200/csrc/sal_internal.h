@@ -21,6 +21,7 @@ constexpr int kHeadDim = SAL_HEAD_DIM;
 constexpr int kFfn = SAL_FFN;
 
 uint64_t wait_limit_ns();
+void count_launch();  // one kernel enqueued
 unsigned int* device_status_ptr();  // device address of the status word (current device)
 
 // frontend.cu
