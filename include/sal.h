@@ -207,6 +207,20 @@ sal_status sal_qkv_rope(const void* h, int batch, int64_t T, const sal_layer* la
 sal_status sal_attention(const void* q, const void* k, const void* v, int batch, int64_t T,
                          void* o, void* stream);
 
+/* sal_qkv_rope without a caller-supplied scratch buffer, for callers that cannot allocate
+ * device memory when they run this step (a real-time audio callback or serving loop that
+ * must not stall or fail on cudaMalloc, a plugin host that forbids device allocations
+ * after start-up, a framework that owns the memory pool). The pages describe nothing like
+ * it: it is a deployment convenience with no counterpart in the method.
+ * Same inputs and outputs as sal_qkv_rope; the rotation table lives in a fixed 2 MiB
+ * array inside the library (held by every GPU that loads it, until exit), so T must be
+ * at most 4096 (SAL_ESHAPE otherwise). No allocation of any kind. Every call shares that
+ * array and fully rewrites the part it reads; calls whose kernels overlap on the GPU
+ * (e.g. on two streams) race on it. The first call on a device looks up the array's
+ * address; make it before any stream capture. */
+sal_status sal_qkv_rope_noalloc(const void* h, int batch, int64_t T, const sal_layer* layer,
+                                void* q, void* k, void* v, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -79,6 +79,9 @@ EXPORTS = {
     "sal_qkv_rope": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.POINTER(sal_layer),
                                      ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
                                      ctypes.c_void_p]),
+    "sal_qkv_rope_noalloc": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int, ctypes.c_int64,
+                                             ctypes.POINTER(sal_layer), ctypes.c_void_p, ctypes.c_void_p,
+                                             ctypes.c_void_p, ctypes.c_void_p]),
     "sal_attention": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int,
                                       ctypes.c_int64, ctypes.c_void_p, ctypes.c_void_p]),
 }
@@ -292,6 +295,14 @@ def sal_qkv_rope(h: torch.Tensor, batch: int, T: int, layer: sal_layer, stream=N
     cs = torch.empty((2, T, 64), dtype=torch.float32, device=h.device)
     _check("sal_qkv_rope", lib().sal_qkv_rope(_ptr(h), batch, T, ctypes.byref(layer), _ptr(q), _ptr(k), _ptr(v),
                                               _ptr(cs), _stream(stream)))
+    return q, k, v
+
+
+def sal_qkv_rope_noalloc(h: torch.Tensor, batch: int, T: int, layer: sal_layer, q: torch.Tensor,
+                         k: torch.Tensor, v: torch.Tensor, stream=None):
+    """sal_qkv_rope into caller-provided q, k, v [batch, 10, T, 128] bf16; allocates nothing."""
+    _check("sal_qkv_rope_noalloc", lib().sal_qkv_rope_noalloc(_ptr(h), batch, T, ctypes.byref(layer), _ptr(q),
+                                                              _ptr(k), _ptr(v), _stream(stream)))
     return q, k, v
 
 
