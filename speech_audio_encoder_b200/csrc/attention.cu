@@ -96,6 +96,8 @@ __global__ void __launch_bounds__(192, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  pdl_wait();
+  pdl_trigger();
   const uint32_t tmem = *tmem_slot;
   const WaitGuard guard{abort_flag, args.limit_ns, args.status};
 
@@ -315,9 +317,8 @@ sal_status attention_launch(const void* q, const void* k, const void* v, int bat
   a.status = device_status_ptr();
   if (!a.status) return SAL_ECUDA;
   const dim3 grid(static_cast<unsigned>((T + kTile - 1) / kTile), static_cast<unsigned>(bh));
-  count_launch();
-  attention_kernel<<<grid, 192, kSmem, s>>>(tq, tk, tv, a);
-  return cudaGetLastError() == cudaSuccess ? SAL_OK : SAL_ECUDA;
+  return launch_kernel(attention_kernel, grid, dim3(192), kSmem, s, tq, tk, tv, a) == cudaSuccess ? SAL_OK
+                                                                                        : SAL_ECUDA;
 }
 
 }  // namespace sal

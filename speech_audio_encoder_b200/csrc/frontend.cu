@@ -112,6 +112,8 @@ __global__ void __launch_bounds__(256, 2)
   const int64_t f0 = static_cast<int64_t>(blockIdx.x) * kFramesPerCta;
   const int nf = static_cast<int>(F - f0 < kFramesPerCta ? F - f0 : kFramesPerCta);
   const int nsamp = kHop * (nf - 1) + kWin;  // a multiple of 4
+  pdl_wait();
+  pdl_trigger();
 
   {  // samples [160 f0, 160 f0 + nsamp) of this clip, read once
     const int64_t g0 = clip * n_samples + kHop * f0;
@@ -301,11 +303,11 @@ sal_status frontend_launch(const float* wave, int64_t n_samples, int batch, int6
   if (st != SAL_OK) return st;
   const dim3 grid(static_cast<unsigned>((frames + kFramesPerCta - 1) / kFramesPerCta),
                   static_cast<unsigned>(batch));
-  count_launch();
-  frontend_kernel<<<grid, 256, kSmemBytes, s>>>(wave, n_samples, frames,
-                                                stacked ? positions * kStack : 0, logmel,
-                                                static_cast<__nv_bfloat16*>(stacked));
-  return cudaGetLastError() == cudaSuccess ? SAL_OK : SAL_ECUDA;
+  const int64_t n_stack = stacked ? positions * kStack : 0;
+  return launch_kernel(frontend_kernel, grid, dim3(256), kSmemBytes, s, wave, n_samples, frames, n_stack, logmel,
+                       static_cast<__nv_bfloat16*>(stacked)) == cudaSuccess
+             ? SAL_OK
+             : SAL_ECUDA;
 }
 
 }  // namespace sal

@@ -45,56 +45,66 @@ struct GemmArgs {
   unsigned int* status;
 };
 
-template <int BN>
+template <int BN, int EPI>
 struct Cfg {
   static constexpr int BM = 128, BK = 64;
-  static constexpr int STAGES = BN == 256 ? 4 : (BN == 128 ? 6 : 8);
+  static constexpr bool QKV = EPI == kEpiQkv;
+  static constexpr bool F32_OUT = EPI == SAL_EPI_STORE_F32 || EPI == SAL_EPI_RESID_F32;
+  // epilogue shared memory: QKV stages a whole head per warp (32 rows x 128 fp32); the
+  // other kinds stage 128-byte-wide output boxes for TMA, two per warp
+  static constexpr int CW = F32_OUT ? 32 : 64;  // output columns per 128-byte box row
+  static constexpr int SCR_BYTES = QKV ? 4 * 32 * 128 * 4 + 4 * 32 * 4 : 4 * 2 * 4096;
+  static constexpr int STAGES = QKV ? 4 : (BN == 256 ? 4 : (BN == 128 ? 6 : 8));
   static constexpr int A_BYTES = BM * BK * 2;
   static constexpr int B_BYTES = BN * BK * 2;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
   static constexpr int TMEM_COLS = 2 * BN;
-  static constexpr size_t SMEM = 1024 + static_cast<size_t>(STAGES) * STAGE_BYTES + 256;
+  static constexpr size_t SMEM = 1024 + static_cast<size_t>(STAGES) * STAGE_BYTES + SCR_BYTES + 256;
+  static_assert(SMEM <= 232448, "shared memory budget");
 };
-
-__device__ __forceinline__ void load_bias32(const __nv_bfloat16* p, float (&b)[32]) {
-  const uint4* p4 = reinterpret_cast<const uint4*>(p);
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const uint4 u = __ldg(p4 + i);
-    b[8 * i + 0] = bf16_lo(u.x); b[8 * i + 1] = bf16_hi(u.x);
-    b[8 * i + 2] = bf16_lo(u.y); b[8 * i + 3] = bf16_hi(u.y);
-    b[8 * i + 4] = bf16_lo(u.z); b[8 * i + 5] = bf16_hi(u.z);
-    b[8 * i + 6] = bf16_lo(u.w); b[8 * i + 7] = bf16_hi(u.w);
-  }
-}
-
-__device__ __forceinline__ void store_bf16x32(__nv_bfloat16* dst, const float (&v)[32]) {
-  uint4* d4 = reinterpret_cast<uint4*>(dst);
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    uint4 u;
-    u.x = pack_bf16x2(v[8 * i + 0], v[8 * i + 1]);
-    u.y = pack_bf16x2(v[8 * i + 2], v[8 * i + 3]);
-    u.z = pack_bf16x2(v[8 * i + 4], v[8 * i + 5]);
-    u.w = pack_bf16x2(v[8 * i + 6], v[8 * i + 7]);
-    d4[i] = u;
-  }
-}
 
 __device__ __forceinline__ float gelu_erf(float x) {
   return 0.5f * x * (1.0f + erff(x * 0.70710678118654752f));
 }
 
+__device__ __forceinline__ float bf16_at(const __nv_bfloat16* p, int i) { return __bfloat162float(p[i]); }
+
+// Warp scratch: 32 rows x W fp32 columns, row r at r * W floats; the 16-byte chunk j of a
+// row sits at chunk position (j & ~7) | ((j ^ r) & 7), so a thread-per-row store of 8
+// consecutive chunks and a row read by the whole warp are both free of bank conflicts.
+template <int W>
+__device__ __forceinline__ int scr_chunk(int r, int j) {
+  return r * (W / 4) + ((j & ~7) | ((j ^ r) & 7));
+}
+
+// Thread `lane` (= row) copies 32 accumulator columns [32 cc, 32 cc + 32) of its TMEM lane
+// into the warp scratch.
+template <int W>
+__device__ __forceinline__ void stage_chunk(float4* scr, int lane, int cc, const uint32_t (&r)[32]) {
+#pragma unroll
+  for (int i = 0; i < 8; ++i)
+    scr[scr_chunk<W>(lane, cc * 8 + i)] =
+        make_float4(__uint_as_float(r[4 * i]), __uint_as_float(r[4 * i + 1]), __uint_as_float(r[4 * i + 2]),
+                    __uint_as_float(r[4 * i + 3]));
+}
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
 template <int BN, int EPI>
 __global__ void __launch_bounds__(192, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                const GemmArgs args) {
-  using C = Cfg<BN>;
+                const __grid_constant__ CUtensorMap tmC, const GemmArgs args) {
+  using C = Cfg<BN, EPI>;
   extern __shared__ unsigned char smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem;
   uint8_t* sB = smem + C::STAGES * C::A_BYTES;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sB + C::STAGES * C::B_BYTES);
+  float4* scratch = reinterpret_cast<float4*>(sB + C::STAGES * C::B_BYTES);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(scratch) + C::SCR_BYTES);
   uint64_t* full = bars;
   uint64_t* empty = bars + C::STAGES;
   uint64_t* tfull = bars + 2 * C::STAGES;
@@ -120,6 +130,7 @@ __global__ void __launch_bounds__(192, 1)
     fence_mbar_init();
     tma_prefetch_desc(&tmA);
     tma_prefetch_desc(&tmB);
+    if constexpr (!C::QKV) tma_prefetch_desc(&tmC);
   }
   if (warp == 1) {
     tmem_alloc(tmem_slot, C::TMEM_COLS);
@@ -128,6 +139,8 @@ __global__ void __launch_bounds__(192, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  pdl_wait();
+  pdl_trigger();
   const uint32_t tmem_base = *tmem_slot;
   const WaitGuard guard{abort_flag, args.limit_ns, args.status};
 
@@ -206,136 +219,205 @@ __global__ void __launch_bounds__(192, 1)
     }
   } else {
     // ------------------------------------------------------------ epilogue warps 2..5
+    // Each warp owns TMEM lanes (= tile rows) 32 q .. 32 q + 31, one row per thread.
     const int quarter = warp & 3;
-    const int row_in_tile = quarter * 32 + lane;
     uint32_t acc = 0, acc_phase = 0;
-    for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
-      const int sp = tile % args.splits;
-      const int rest = tile / args.splits;
-      const int n = rest % num_n, m = rest / num_n;
-      if (!mbar_wait_warp(&tfull[acc], acc_phase, guard)) break;
-      tc_fence_after();
-      const int64_t row = static_cast<int64_t>(m) * C::BM + row_in_tile;
-      const bool valid = row < args.M;
-      const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + acc * BN;
-
-      if constexpr (EPI == kEpiQkv) {
-        const int64_t b = valid ? row / args.T : 0;
-        const int64_t t = valid ? row - b * args.T : 0;
+    if constexpr (C::QKV) {
+      // Per head: stage the 32 x 128 accumulator block in shared memory, then walk its
+      // rows with the lanes across the columns (lane l holds columns 4l .. 4l + 3): the
+      // RMS norm is a warp sum, the RoPE partner column i +- 64 sits 16 lanes away, and
+      // cos / sin of t * theta_i advance row by row by one rotation through theta_i, so
+      // the loop issues no global load besides one table row per 32-row block.
+      float4* scr = scratch + (warp - 2) * (32 * 128 / 4);
+      float* inv_row = reinterpret_cast<float*>(scratch + 4 * (32 * 128 / 4)) + (warp - 2) * 32;
+      const int q4 = lane & 15;
+      const float sg = lane >= 16 ? 1.f : -1.f;  // i < 64: a c - b s;  i >= 64: b c + a s
+      float4 c1 = make_float4(1.f, 1.f, 1.f, 1.f), s1 = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (args.T > 1) {  // table row t = 1 holds cos / sin of theta_i itself
+        c1 = __ldg(reinterpret_cast<const float4*>(args.rope_cs + 64) + q4);
+        s1 = __ldg(reinterpret_cast<const float4*>(args.rope_cs + (args.T + 1) * 64) + q4);
+      }
+      for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
+        const int rest = tile / args.splits;
+        const int n = rest % num_n, m = rest / num_n;
+        if (!mbar_wait_warp(&tfull[acc], acc_phase, guard)) break;
+        tc_fence_after();
+        const int64_t row0 = static_cast<int64_t>(m) * C::BM + quarter * 32;
+        const int nrows = static_cast<int>(args.M - row0 < 32 ? (args.M - row0 > 0 ? args.M - row0 : 0) : 32);
+        const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + acc * BN;
 #pragma unroll 1
         for (int hb = 0; hb < BN / 128; ++hb) {
           const int col0 = n * BN + hb * 128;
           const int sec = col0 / kWidth;
           const int head = (col0 % kWidth) / kHeadDim;
+          // thread-per-row: add the bias, stage the row, and (q, k) take its RMS factor
+          float ss = 0.f;
+#pragma unroll 1
+          for (int cc = 0; cc < 4; ++cc) {
+            uint32_t r[32];
+            tmem_ld32(taddr + hb * 128 + cc * 32, r);
+            tmem_wait_ld();
+            const uint4* b8 = reinterpret_cast<const uint4*>(args.bias + col0 + cc * 32);
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              const uint4 bb = __ldg(b8 + j);
+              const uint32_t bw[4] = {bb.x, bb.y, bb.z, bb.w};
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                const float lo = __uint_as_float(r[8 * j + 2 * e]) + bf16_lo(bw[e]);
+                const float hi = __uint_as_float(r[8 * j + 2 * e + 1]) + bf16_hi(bw[e]);
+                ss = fmaf(lo, lo, fmaf(hi, hi, ss));
+                r[8 * j + 2 * e] = __float_as_uint(lo);
+                r[8 * j + 2 * e + 1] = __float_as_uint(hi);
+              }
+            }
+            stage_chunk<128>(scr, lane, cc, r);
+          }
+          if (hb == BN / 128 - 1) {  // accumulator no longer needed
+            tc_fence_before();
+            mbar_arrive(&tempty[acc]);
+          }
+          inv_row[lane] = 1.0f / sqrtf(ss * (1.0f / kHeadDim) + 1e-6f);
+          __syncwarp();
           __nv_bfloat16* base = sec == 0 ? args.q : (sec == 1 ? args.k : args.v);
-          __nv_bfloat16* dst = base + ((b * kHeads + head) * args.T + t) * kHeadDim;
-          const uint32_t ta = taddr + hb * 128;
-          if (sec == 2) {
-#pragma unroll 1
-            for (int c = 0; c < 128; c += 32) {
-              uint32_t r[32];
-              float bias[32], vv[32];
-              tmem_ld32(ta + c, r);
-              tmem_wait_ld();
-              load_bias32(args.bias + col0 + c, bias);
-#pragma unroll
-              for (int j = 0; j < 32; ++j) vv[j] = __uint_as_float(r[j]) + bias[j];
-              if (valid) store_bf16x32(dst + c, vv);
-            }
-          } else {
-            float ss = 0.f;
-#pragma unroll 1
-            for (int c = 0; c < 128; c += 32) {
-              uint32_t r[32];
-              float bias[32];
-              tmem_ld32(ta + c, r);
-              tmem_wait_ld();
-              load_bias32(args.bias + col0 + c, bias);
-#pragma unroll
-              for (int j = 0; j < 32; ++j) {
-                const float x = __uint_as_float(r[j]) + bias[j];
-                ss = fmaf(x, x, ss);
-              }
-            }
-            const float inv = 1.0f / sqrtf(ss * (1.0f / kHeadDim) + 1e-6f);
-            const __nv_bfloat16* g = sec == 0 ? args.qn_g : args.kn_g;
-            const float* cosr = args.rope_cs + t * 64;
-            const float* sinr = args.rope_cs + args.T * 64 + t * 64;
-#pragma unroll 1
-            for (int i0 = 0; i0 < 64; i0 += 32) {
-              uint32_t ra[32], rb[32];
-              float ba[32], bb[32], ga[32], gb[32], oa[32], ob[32];
-              tmem_ld32(ta + i0, ra);
-              tmem_ld32(ta + i0 + 64, rb);
-              tmem_wait_ld();
-              load_bias32(args.bias + col0 + i0, ba);
-              load_bias32(args.bias + col0 + i0 + 64, bb);
-              load_bias32(g + i0, ga);
-              load_bias32(g + i0 + 64, gb);
-              if (valid) {
-#pragma unroll
-                for (int j = 0; j < 32; ++j) {
-                  const float av = (__uint_as_float(ra[j]) + ba[j]) * inv * ga[j];
-                  const float bv = (__uint_as_float(rb[j]) + bb[j]) * inv * gb[j];
-                  const float cs = __ldg(cosr + i0 + j), sn = __ldg(sinr + i0 + j);
-                  oa[j] = av * cs - bv * sn;
-                  ob[j] = bv * cs + av * sn;
+          if (nrows > 0) {
+            int64_t b = row0 / args.T, t = row0 - b * args.T;
+            __nv_bfloat16* dst = base + ((b * kHeads + head) * args.T + t) * kHeadDim;
+            if (sec == 2) {
+#pragma unroll 4
+              for (int r = 0; r < nrows; ++r) {
+                const float4 v = scr[scr_chunk<128>(r, lane)];
+                uint2 o;
+                o.x = pack_bf16x2(v.x, v.y);
+                o.y = pack_bf16x2(v.z, v.w);
+                reinterpret_cast<uint2*>(dst)[lane] = o;
+                dst += kHeadDim;
+                if (++t == args.T) {  // next clip
+                  t = 0;
+                  ++b;
+                  dst = base + (b * kHeads + head) * args.T * kHeadDim;
                 }
-                store_bf16x32(dst + i0, oa);
-                store_bf16x32(dst + i0 + 64, ob);
               }
-            }
-          }
-        }
-      } else {
-#pragma unroll 1
-        for (int c = 0; c < BN; c += 32) {
-          uint32_t r[32];
-          float bias[32], vv[32];
-          tmem_ld32(taddr + c, r);
-          tmem_wait_ld();
-          const int col0 = n * BN + c;
-          if (EPI == SAL_EPI_RESID_F32 && sp != 0) {
-#pragma unroll
-            for (int j = 0; j < 32; ++j) bias[j] = 0.f;
-          } else {
-            load_bias32(args.bias + col0, bias);
-          }
-#pragma unroll
-          for (int j = 0; j < 32; ++j) vv[j] = __uint_as_float(r[j]) + bias[j];
-          if (valid) {
-            if constexpr (EPI == SAL_EPI_STORE_F32) {
-              float4* o4 = reinterpret_cast<float4*>(static_cast<float*>(args.out) + row * args.N + col0);
-#pragma unroll
-              for (int i = 0; i < 8; ++i) o4[i] = make_float4(vv[4 * i], vv[4 * i + 1], vv[4 * i + 2], vv[4 * i + 3]);
-            } else if constexpr (EPI == SAL_EPI_STORE_BF16) {
-              store_bf16x32(static_cast<__nv_bfloat16*>(args.out) + row * args.N + col0, vv);
-            } else if constexpr (EPI == SAL_EPI_GELU_BF16) {
-#pragma unroll
-              for (int j = 0; j < 32; ++j) vv[j] = gelu_erf(vv[j]);
-              store_bf16x32(static_cast<__nv_bfloat16*>(args.out) + row * args.N + col0, vv);
-            } else {  // residual add into the fp32 stream
-              float4* o4 = reinterpret_cast<float4*>(static_cast<float*>(args.out) + row * args.N + col0);
-              if (args.splits == 1) {
-#pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                  float4 x = o4[i];
-                  x.x += vv[4 * i]; x.y += vv[4 * i + 1]; x.z += vv[4 * i + 2]; x.w += vv[4 * i + 3];
-                  o4[i] = x;
+            } else {
+              const __nv_bfloat16* gp = (sec == 0 ? args.qn_g : args.kn_g) + 4 * lane;
+              const float4 g4 = make_float4(bf16_at(gp, 0), bf16_at(gp, 1), bf16_at(gp, 2), bf16_at(gp, 3));
+              float4 c = __ldg(reinterpret_cast<const float4*>(args.rope_cs + t * 64) + q4);
+              float4 sn = __ldg(reinterpret_cast<const float4*>(args.rope_cs + (args.T + t) * 64) + q4);
+#pragma unroll 4
+              for (int r = 0; r < nrows; ++r) {
+                float4 v = scr[scr_chunk<128>(r, lane)];
+                const float inv = inv_row[r];
+                v.x *= inv * g4.x; v.y *= inv * g4.y; v.z *= inv * g4.z; v.w *= inv * g4.w;
+                float4 p;  // the partner half: column i +- 64
+                p.x = __shfl_xor_sync(0xffffffffu, v.x, 16);
+                p.y = __shfl_xor_sync(0xffffffffu, v.y, 16);
+                p.z = __shfl_xor_sync(0xffffffffu, v.z, 16);
+                p.w = __shfl_xor_sync(0xffffffffu, v.w, 16);
+                uint2 o;
+                o.x = pack_bf16x2(fmaf(sg * p.x, sn.x, v.x * c.x), fmaf(sg * p.y, sn.y, v.y * c.y));
+                o.y = pack_bf16x2(fmaf(sg * p.z, sn.z, v.z * c.z), fmaf(sg * p.w, sn.w, v.w * c.w));
+                reinterpret_cast<uint2*>(dst)[lane] = o;
+                dst += kHeadDim;
+                if (++t == args.T) {  // next clip: positions restart at 0
+                  t = 0;
+                  ++b;
+                  dst = base + (b * kHeads + head) * args.T * kHeadDim;
+                  c = make_float4(1.f, 1.f, 1.f, 1.f);
+                  sn = make_float4(0.f, 0.f, 0.f, 0.f);
+                } else {  // rotate by theta_i: angle (t + 1) theta_i
+                  const float4 cc = c;
+                  c.x = fmaf(cc.x, c1.x, -sn.x * s1.x); sn.x = fmaf(sn.x, c1.x, cc.x * s1.x);
+                  c.y = fmaf(cc.y, c1.y, -sn.y * s1.y); sn.y = fmaf(sn.y, c1.y, cc.y * s1.y);
+                  c.z = fmaf(cc.z, c1.z, -sn.z * s1.z); sn.z = fmaf(sn.z, c1.z, cc.z * s1.z);
+                  c.w = fmaf(cc.w, c1.w, -sn.w * s1.w); sn.w = fmaf(sn.w, c1.w, cc.w * s1.w);
                 }
-              } else {
-#pragma unroll
-                for (int i = 0; i < 8; ++i)
-                  atomicAdd(o4 + i, make_float4(vv[4 * i], vv[4 * i + 1], vv[4 * i + 2], vv[4 * i + 3]));
               }
             }
           }
+          __syncwarp();
         }
+        acc ^= 1;
+        if (acc == 0) acc_phase ^= 1;
       }
-      tc_fence_before();
-      mbar_arrive(&tempty[acc]);
-      acc ^= 1;
-      if (acc == 0) acc_phase ^= 1;
+    } else {
+      // Per 128-byte-wide column chunk: each thread converts its row's values and writes
+      // them into a 128B-swizzled 32-row box in shared memory (two boxes per warp, used in
+      // turn); one lane then issues a TMA store of the box, or a TMA reduce-add into the
+      // fp32 residual stream, while the warp moves on to the next chunk.
+      uint8_t* stg = reinterpret_cast<uint8_t*>(scratch) + (warp - 2) * 8192;
+      uint32_t kbuf = 0;
+      for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
+        const int sp = tile % args.splits;
+        const int rest = tile / args.splits;
+        const int n = rest % num_n, m = rest / num_n;
+        if (!mbar_wait_warp(&tfull[acc], acc_phase, guard)) break;
+        tc_fence_after();
+        const int y = m * C::BM + quarter * 32;
+        const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + acc * BN;
+#pragma unroll 1
+        for (int c = 0; c < BN; c += C::CW) {
+          uint8_t* buf = stg + (kbuf & 1) * 4096;
+          if (kbuf >= 2) {  // the store issued from this box two chunks ago has read it
+            if (lane == 0) bulk_wait_read<1>();
+            __syncwarp();
+          }
+          uint32_t r[C::CW];
+          tmem_ld32(taddr + c, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
+          if constexpr (C::CW == 64) tmem_ld32(taddr + c + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
+          tmem_wait_ld();
+          if (c + C::CW == BN) {  // accumulator no longer needed
+            tc_fence_before();
+            mbar_arrive(&tempty[acc]);
+          }
+          const int col0 = n * BN + c;
+          const bool add_bias = !(EPI == SAL_EPI_RESID_F32 && sp != 0);
+          const uint4* bias8 = reinterpret_cast<const uint4*>(args.bias + col0);
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {  // 16-byte chunk j of this row
+            uint4 word;
+            if constexpr (C::F32_OUT) {
+              float v[4];
+              const uint2 bb = add_bias ? __ldg(reinterpret_cast<const uint2*>(bias8) + j) : make_uint2(0, 0);
+              v[0] = __uint_as_float(r[4 * j + 0]) + bf16_lo(bb.x);
+              v[1] = __uint_as_float(r[4 * j + 1]) + bf16_hi(bb.x);
+              v[2] = __uint_as_float(r[4 * j + 2]) + bf16_lo(bb.y);
+              v[3] = __uint_as_float(r[4 * j + 3]) + bf16_hi(bb.y);
+              word = make_uint4(__float_as_uint(v[0]), __float_as_uint(v[1]), __float_as_uint(v[2]),
+                                __float_as_uint(v[3]));
+            } else {
+              const uint4 bb = __ldg(bias8 + j);
+              const uint32_t bw[4] = {bb.x, bb.y, bb.z, bb.w};
+              uint32_t o[4];
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                float lo = __uint_as_float(r[8 * j + 2 * e]) + bf16_lo(bw[e]);
+                float hi = __uint_as_float(r[8 * j + 2 * e + 1]) + bf16_hi(bw[e]);
+                if constexpr (EPI == SAL_EPI_GELU_BF16) {
+                  lo = gelu_erf(lo);
+                  hi = gelu_erf(hi);
+                }
+                o[e] = pack_bf16x2(lo, hi);
+              }
+              word = make_uint4(o[0], o[1], o[2], o[3]);
+            }
+            *reinterpret_cast<uint4*>(buf + lane * 128 + ((j ^ (lane & 7)) << 4)) = word;
+          }
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            if constexpr (EPI == SAL_EPI_RESID_F32)
+              tma_reduce_add_2d(&tmC, buf, col0, y);
+            else
+              tma_store_2d(&tmC, buf, col0, y);
+            bulk_commit();
+          }
+          ++kbuf;
+        }
+        acc ^= 1;
+        if (acc == 0) acc_phase ^= 1;
+      }
+      if (lane == 0) bulk_wait_all();  // every store of this warp has landed
+      __syncwarp();
     }
   }
 
@@ -366,7 +448,7 @@ int num_sms() {
 
 template <int BN, int EPI>
 sal_status launch_bn(const GemmArgs& a, const void* A, const void* W, cudaStream_t s) {
-  using C = Cfg<BN>;
+  using C = Cfg<BN, EPI>;
   static bool attr_done[64] = {};
   int dev = 0;
   cudaGetDevice(&dev);
@@ -379,29 +461,39 @@ sal_status launch_bn(const GemmArgs& a, const void* A, const void* W, cudaStream
       attr_done[dev] = true;
     }
   }
-  CUtensorMap ta, tb;
+  CUtensorMap ta, tb, tc;
   if (!make_tmap_2d_bf16(&ta, A, a.K, a.M, C::BK, C::BM)) return SAL_ECUDA;
   if (!make_tmap_2d_bf16(&tb, W, a.K, a.N, C::BK, BN)) return SAL_ECUDA;
+  if constexpr (C::QKV) {
+    tc = ta;  // unused
+  } else if constexpr (C::F32_OUT) {
+    if (!make_tmap_2d_f32(&tc, a.out, a.N, a.M, C::CW, 32)) return SAL_ECUDA;
+  } else {
+    if (!make_tmap_2d_bf16(&tc, a.out, a.N, a.M, C::CW, 32)) return SAL_ECUDA;
+  }
   const int tiles = static_cast<int>((a.M + C::BM - 1) / C::BM) * (a.N / BN) * a.splits;
   const int grid = tiles < num_sms() ? tiles : num_sms();
-  count_launch();
-  gemm_kernel<BN, EPI><<<grid, 192, C::SMEM, s>>>(ta, tb, a);
-  return cudaGetLastError() == cudaSuccess ? SAL_OK : SAL_ECUDA;
+  return launch_kernel(gemm_kernel<BN, EPI>, dim3(grid), dim3(192), C::SMEM, s, ta, tb, tc, a) == cudaSuccess
+             ? SAL_OK
+             : SAL_ECUDA;
 }
 
 template <int EPI>
 sal_status launch_epi(int BN, const GemmArgs& a, const void* A, const void* W, cudaStream_t s) {
-  switch (BN) {
-    case 256: return launch_bn<256, EPI>(a, A, W, s);
-    case 128: return launch_bn<128, EPI>(a, A, W, s);
-    default:
-      if constexpr (EPI == kEpiQkv) return SAL_ESHAPE;
-      else return launch_bn<64, EPI>(a, A, W, s);
+  if constexpr (EPI == kEpiQkv) {  // one head per tile
+    return BN == 128 ? launch_bn<128, EPI>(a, A, W, s) : SAL_ESHAPE;
+  } else {
+    switch (BN) {
+      case 256: return launch_bn<256, EPI>(a, A, W, s);
+      case 128: return launch_bn<128, EPI>(a, A, W, s);
+      default: return launch_bn<64, EPI>(a, A, W, s);
+    }
   }
 }
 
 // Largest tile width whose tile count fills the GPU; the narrowest otherwise.
 int pick_bn(int64_t M, int N, bool qkv) {
+  if (qkv) return 128;
   const int64_t mt = (M + 127) / 128;
   const int sms = num_sms();
   if (N % 256 == 0 && mt * (N / 256) >= sms) return 256;

@@ -11,6 +11,7 @@
 #include <math.h>
 
 #include "sal_internal.h"
+#include "sal_ptx.cuh"
 
 namespace sal {
 namespace {
@@ -30,6 +31,8 @@ __global__ void __launch_bounds__(256) layernorm_kernel(const float* __restrict_
                                                         __nv_bfloat16* __restrict__ y) {
   const int lane = threadIdx.x & 31;
   const int64_t row = static_cast<int64_t>(blockIdx.x) * kLnWarps + (threadIdx.x >> 5);
+  pdl_wait();
+  pdl_trigger();
   if (row >= rows) return;
   const float4* xr = reinterpret_cast<const float4*>(x + row * kWidth);
   float4 v[kVec];
@@ -68,6 +71,8 @@ __global__ void __launch_bounds__(256) layernorm_kernel(const float* __restrict_
 
 __global__ void rope_table_kernel(float* __restrict__ cs, int64_t T) {
   const int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  pdl_wait();
+  pdl_trigger();
   if (idx >= T * 64) return;
   const int64_t t = idx >> 6;
   const int i = static_cast<int>(idx & 63);
@@ -84,19 +89,20 @@ sal_status layernorm_launch(const float* x, int64_t rows, const void* g, const v
                             cudaStream_t s) {
   if (rows == 0) return SAL_OK;
   const unsigned grid = static_cast<unsigned>((rows + kLnWarps - 1) / kLnWarps);
-  count_launch();
-  layernorm_kernel<<<grid, 32 * kLnWarps, 0, s>>>(x, rows, static_cast<const __nv_bfloat16*>(g),
-                                                  static_cast<const __nv_bfloat16*>(b),
-                                                  static_cast<__nv_bfloat16*>(y));
-  return cudaGetLastError() == cudaSuccess ? SAL_OK : SAL_ECUDA;
+  return launch_kernel(layernorm_kernel, dim3(grid), dim3(32 * kLnWarps), 0, s, x, rows,
+                       static_cast<const __nv_bfloat16*>(g), static_cast<const __nv_bfloat16*>(b),
+                       static_cast<__nv_bfloat16*>(y)) == cudaSuccess
+             ? SAL_OK
+             : SAL_ECUDA;
 }
 
 sal_status rope_table_launch(float* cs, int64_t T, cudaStream_t s) {
   if (T == 0) return SAL_OK;
   const int64_t n = T * 64;
-  count_launch();
-  rope_table_kernel<<<static_cast<unsigned>((n + 255) / 256), 256, 0, s>>>(cs, T);
-  return cudaGetLastError() == cudaSuccess ? SAL_OK : SAL_ECUDA;
+  return launch_kernel(rope_table_kernel, dim3(static_cast<unsigned>((n + 255) / 256)), dim3(256), 0, s, cs, T) ==
+                 cudaSuccess
+             ? SAL_OK
+             : SAL_ECUDA;
 }
 
 }  // namespace sal

@@ -5,6 +5,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <utility>
+
 #include "../../include/sal.h"
 
 namespace sal {
@@ -21,6 +23,7 @@ constexpr int kHeadDim = SAL_HEAD_DIM;
 constexpr int kFfn = SAL_FFN;
 
 uint64_t wait_limit_ns();
+bool pdl_enabled();  // programmatic dependent launch (env SAL_PDL=0 turns it off)
 void count_launch();  // one kernel enqueued
 unsigned int* device_status_ptr();  // device address of the status word (current device)
 
@@ -51,8 +54,31 @@ sal_status attention_launch(const void* q, const void* k, const void* v, int bat
 // tensor maps (sal_api.cu)
 bool make_tmap_2d_bf16(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer,
                        uint32_t box_inner, uint32_t box_outer);
+bool make_tmap_2d_f32(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer,
+                      uint32_t box_inner, uint32_t box_outer);
 bool make_tmap_3d_bf16(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1, uint64_t d2,
                        uint32_t b0, uint32_t b1, uint32_t b2);
+
+// Launches `kernel` on `s` with programmatic dependent launch allowed: the kernel may be
+// scheduled while its predecessor on the stream is still running, runs its prologue, and
+// waits in griddepcontrol.wait (every kernel of this library does so before touching
+// global memory) until the predecessor has completed.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_kernel(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                          Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl_enabled() ? 1 : 0;
+  count_launch();
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
 
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 

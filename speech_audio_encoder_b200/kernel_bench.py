@@ -2,9 +2,11 @@
 
     python -m speech_audio_encoder_b200.kernel_bench KIND [--batch B] [--T T] [--reps R]
 
-KIND is one of frontend, stack_proj, layernorm, qkv, attention, out_proj, ffn_up, ffn_down.
-Each repetition is one launch (qkv also launches the small RoPE-table kernel); times come
-from CUDA events on the launching stream after warm-up. Prints one JSON line with the
+KIND is one of frontend, stack_proj, layernorm, qkv, attention, out_proj, ffn_up, ffn_down,
+linear (any --N, --K, --epi).
+Each repetition is one launch (qkv also launches the small RoPE-table kernel). The
+repetitions are captured once as a CUDA graph and the replay is timed with CUDA events on
+the launching stream after warm-up (eager launches from Python would measure the host). Prints one JSON line with the
 average launch time and the achieved rate against the algorithmic flops or bytes. Small
 cases of this command are what the committed ncu summaries capture.
 """
@@ -31,6 +33,9 @@ def main():
     ap.add_argument("--T", type=int, default=374)
     ap.add_argument("--reps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--N", type=int, default=1280, help="linear: output width")
+    ap.add_argument("--K", type=int, default=1280, help="linear: reduction length")
+    ap.add_argument("--epi", type=int, default=1, help="linear: sal_epilogue value")
     a = ap.parse_args()
     B, T = a.batch, a.T
     M = B * T
@@ -65,6 +70,16 @@ def main():
 
         def run():
             api.sal_attention(q, k, v)
+    elif a.kind == "linear":
+        K, N, epi = a.K, a.N, a.epi
+        A = _bf16((M, K), 4, 1.0)
+        W = _bf16((N, K), 5, 0.02)
+        bias = _bf16((N,), 6, 0.02)
+        out = torch.zeros((M, N), dtype=torch.float32 if epi in (0, 3) else torch.bfloat16, device="cuda")
+        flops = 2.0 * M * N * K
+
+        def run():
+            api.sal_linear(epi, A, W, bias, out=out)
     else:
         K, N, epi = {"stack_proj": (1024, 1280, api.SAL_EPI_STORE_F32),
                      "out_proj": (1280, 1280, api.SAL_EPI_RESID_F32),
@@ -82,15 +97,20 @@ def main():
     for _ in range(a.warmup):
         run()
     torch.cuda.synchronize()
-    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(a.reps)]
-    for e0, e1 in evs:
-        e0.record(s)
-        run()
-        e1.record(s)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        for _ in range(a.reps):
+            run()
+    graph.replay()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(s)
+    graph.replay()
+    e1.record(s)
     torch.cuda.synchronize()
     if api.sal_last_device_status() != 0:
         raise RuntimeError("a device wait timed out")
-    ms = float(np.mean([e0.elapsed_time(e1) for e0, e1 in evs]))
+    ms = e0.elapsed_time(e1) / a.reps
     out = {"kind": a.kind, "batch": B, "T": T, "avg_ms": ms}
     if flops:
         out["tflops"] = flops / (ms / 1e3) / 1e12
