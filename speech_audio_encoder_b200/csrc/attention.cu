@@ -19,6 +19,7 @@
 #include <cuda_bf16.h>
 #include <math.h>
 
+#include <cstdlib>
 #include <mutex>
 
 #include "sal_internal.h"
@@ -35,6 +36,15 @@ __device__ __forceinline__ uint32_t col_s(int s) { return s ? 128u : 0u; }    //
 __device__ __forceinline__ uint32_t col_p(int s) { return s ? 448u : 384u; }  // bf16 P buffers
 constexpr size_t kSmem = 1024 + 5 * kTileBytes + 256;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
+
+// The two-tile kernel can be turned off with SAL_ATTN_PP=0 (to compare the two designs).
+bool attention_pp_enabled() {
+  static const bool on = [] {
+    const char* e = std::getenv("SAL_ATTN_PP");
+    return !(e && e[0] == '0');
+  }();
+  return on;
+}
 
 struct AttnArgs {
   int64_t T;
@@ -284,8 +294,290 @@ __global__ void __launch_bounds__(192, 1)
   }
 }
 
+// ---------------------------------------------------------------------------------
+// Ping-pong variant for long clips: one CTA owns TWO 128-row query tiles of one
+// (clip, head), so each K / V tile loaded serves 256 queries, and two softmax warpgroups
+// alternate with the tensor core: while warpgroup 0 runs the softmax of S0_j, the
+// tensor core computes O1 += P1_{j-1} V_{j-1} and S1_j, and the other way round.
+//   warp 0: TMA loads (Q0 and Q1 once; K_j and V_j through two-stage rings released
+//           separately: K after both S products, V after both P V products)
+//   warp 1: tcgen05.mma issue, in the order S0_0 S1_0 | PV0_j S0_{j+1} PV1_j S1_{j+1} ...
+//   warps 2-5 / 6-9: softmax of query tile 0 / 1, one row per thread
+// TMEM: S0 [0,128) S1 [128,256) O0 [256,384) O1 [384,512); P_i (bf16 pairs) overwrites
+// the first 64 columns of S_i once the row has been read. Because tcgen05.mma operations
+// of one thread complete in issue order, S_i(j) completing implies P_i(j-1) V_{j-1} has
+// completed, so the softmax may rescale O_i as soon as S_i(j) is ready.
+// The softmax makes two passes over S in TMEM (row maximum, then exponentials), which
+// keeps register use low enough for ten warps.
+constexpr size_t kSmemPP = 1024 + 6 * kTileBytes + 256;
+
+__global__ void __launch_bounds__(320, 1)
+    attention_pp_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                        const __grid_constant__ CUtensorMap tmV, const AttnArgs args) {
+  extern __shared__ unsigned char smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sQ = smem;                       // Q0, Q1
+  uint8_t* sK = smem + 2 * kTileBytes;      // K stage 0, 1
+  uint8_t* sV = smem + 4 * kTileBytes;      // V stage 0, 1
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + 6 * kTileBytes);
+  uint64_t* q_full = bars + 0;
+  uint64_t* k_full = bars + 1;    // [2]
+  uint64_t* v_full = bars + 3;    // [2]
+  uint64_t* k_empty = bars + 5;   // [2]
+  uint64_t* v_empty = bars + 7;   // [2]
+  uint64_t* s_full = bars + 9;    // [2] one per query tile
+  uint64_t* p_full = bars + 11;   // [2]
+  uint64_t* o_final = bars + 13;  // [2]
+  uint64_t* drain = bars + 15;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 16);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int64_t T = args.T;
+  const int bh = blockIdx.y;
+  const int qt2 = blockIdx.x;  // 256-row query block
+  const int n_kv = static_cast<int>((T + kTile - 1) / kTile);
+
+  if (threadIdx.x == 0) {
+    mbar_init(q_full, 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&k_full[s], 1);
+      mbar_init(&v_full[s], 1);
+      mbar_init(&k_empty[s], 1);
+      mbar_init(&v_empty[s], 1);
+      mbar_init(&s_full[s], 1);
+      mbar_init(&p_full[s], 128);
+      mbar_init(&o_final[s], 1);
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+    tma_prefetch_desc(&tmQ);
+    tma_prefetch_desc(&tmK);
+    tma_prefetch_desc(&tmV);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  pdl_wait();
+  pdl_trigger();
+  const uint32_t tmem = *tmem_slot;
+  const WaitGuard guard{abort_flag, args.limit_ns, args.status};
+
+  if (warp == 0) {
+    if (lane == 0) {
+      uint32_t issued_k = 0, issued_v = 0, par_k = 0, par_v = 0;
+      mbar_arrive_expect_tx(q_full, 2 * kTileBytes);
+      for (int i = 0; i < 2; ++i) {
+        tma_load_3d(sQ + i * kTileBytes, &tmQ, q_full, 0, (2 * qt2 + i) * kTile, bh);
+        tma_load_3d(sQ + i * kTileBytes + kBox, &tmQ, q_full, 64, (2 * qt2 + i) * kTile, bh);
+      }
+      for (int j = 0; j < n_kv; ++j) {
+        const int s = j & 1;
+        const uint32_t use_par = (j >> 1) & 1;
+        if (!mbar_wait(&k_empty[s], use_par ^ 1, guard)) break;
+        mbar_arrive_expect_tx(&k_full[s], kTileBytes);
+        tma_load_3d(sK + s * kTileBytes, &tmK, &k_full[s], 0, j * kTile, bh);
+        tma_load_3d(sK + s * kTileBytes + kBox, &tmK, &k_full[s], 64, j * kTile, bh);
+        issued_k |= 1u << s;
+        par_k = (par_k & ~(1u << s)) | (use_par << s);
+        if (!mbar_wait(&v_empty[s], use_par ^ 1, guard)) break;
+        mbar_arrive_expect_tx(&v_full[s], kTileBytes);
+        tma_load_3d(sV + s * kTileBytes, &tmV, &v_full[s], 0, j * kTile, bh);
+        tma_load_3d(sV + s * kTileBytes + kBox, &tmV, &v_full[s], 64, j * kTile, bh);
+        issued_v |= 1u << s;
+        par_v = (par_v & ~(1u << s)) | (use_par << s);
+      }
+      if (*abort_flag) {
+        drain_wait(q_full, 0, args.limit_ns);
+        for (int s = 0; s < 2; ++s) {
+          if (issued_k & (1u << s)) drain_wait(&k_full[s], (par_k >> s) & 1, args.limit_ns);
+          if (issued_v & (1u << s)) drain_wait(&v_full[s], (par_v >> s) & 1, args.limit_ns);
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      constexpr uint32_t IDESC_S = idesc_bf16(128, 128, false, false);
+      constexpr uint32_t IDESC_O = idesc_bf16(128, 128, false, true);
+      bool any_mma = false;
+      auto issue_s = [&](int i, int j) -> bool {  // S_i = Q_i K_j^T
+        const int s = j & 1;
+        if (!mbar_wait(&k_full[s], (j >> 1) & 1, guard)) return false;
+        tc_fence_after();
+        const uint32_t q0 = smem_u32(sQ + i * kTileBytes), k0 = smem_u32(sK + s * kTileBytes);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint32_t off = (kk >> 2) * kBox + (kk & 3) * 32;
+          umma_ss(tmem + 128 * i, sdesc_kmajor_sw128(q0 + off), sdesc_kmajor_sw128(k0 + off), IDESC_S, kk > 0);
+        }
+        umma_commit(&s_full[i]);
+        if (i == 1) umma_commit(&k_empty[s]);  // both products with K_j issued
+        any_mma = true;
+        return true;
+      };
+      auto issue_pv = [&](int i, int j) -> bool {  // O_i += P_i V_j
+        const int s = j & 1;
+        if (!mbar_wait(&p_full[i], j & 1, guard)) return false;
+        if (!mbar_wait(&v_full[s], (j >> 1) & 1, guard)) return false;
+        tc_fence_after();
+        const uint32_t v0 = smem_u32(sV + s * kTileBytes);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          umma_ts(tmem + 256 + 128 * i, tmem + 128 * i + kk * 8, sdesc_mnmajor_sw128(v0 + kk * 2048, kBox), IDESC_O,
+                  (j > 0 || kk > 0));
+        if (i == 1) umma_commit(&v_empty[s]);
+        return true;
+      };
+      bool ok = mbar_wait(q_full, 0, guard) && issue_s(0, 0) && issue_s(1, 0);
+      for (int j = 0; ok && j < n_kv; ++j) {
+        ok = issue_pv(0, j);
+        if (!ok) break;
+        if (j + 1 < n_kv) {
+          ok = issue_s(0, j + 1);
+        } else {
+          umma_commit(&o_final[0]);
+        }
+        if (!ok) break;
+        ok = issue_pv(1, j);
+        if (!ok) break;
+        if (j + 1 < n_kv) {
+          ok = issue_s(1, j + 1);
+        } else {
+          umma_commit(&o_final[1]);
+        }
+      }
+      if (*abort_flag && any_mma) {
+        umma_commit(drain);
+        drain_wait(drain, 0, args.limit_ns);
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ softmax warpgroups
+    const int wg = (warp - 2) >> 2;  // query tile 0 or 1
+    const int quarter = warp & 3;
+    const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
+    const uint32_t colS = 128u * wg, colO = 256u + 128u * wg;
+    const int row = quarter * 32 + lane;
+    const float sl2 = args.scale_log2;
+    float m_ref = -INFINITY, l = 0.f;
+    bool ok = true;
+    for (int j = 0; j < n_kv; ++j) {
+      if (!mbar_wait_warp(&s_full[wg], j & 1, guard)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const int64_t rem = T - static_cast<int64_t>(j) * kTile;
+      const int valid = static_cast<int>(rem < kTile ? rem : kTile);
+      // pass 1: row maximum
+      float mx = -INFINITY;
+#pragma unroll
+      for (int c = 0; c < 4; c += 2) {
+        uint32_t ra[32], rb[32];
+        tmem_ld32(tmem + lane_base + colS + 32 * c, ra);
+        tmem_ld32(tmem + lane_base + colS + 32 * c + 32, rb);
+        tmem_wait_ld();
+        if (valid == kTile) {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) mx = fmaxf(mx, fmaxf(__uint_as_float(ra[i]), __uint_as_float(rb[i])));
+        } else {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            if (32 * c + i < valid) mx = fmaxf(mx, __uint_as_float(ra[i]));
+            if (32 * c + 32 + i < valid) mx = fmaxf(mx, __uint_as_float(rb[i]));
+          }
+        }
+      }
+      mx *= sl2;
+      float alpha = 1.f;
+      bool rescale = false;
+      if (j == 0) {
+        m_ref = mx;
+      } else if (mx > m_ref + kRescaleThreshold) {
+        alpha = fast_exp2(m_ref - mx);
+        m_ref = mx;
+        rescale = true;
+      }
+      // O_i(j-1) is complete (it was issued before S_i(j)); rescale it if the max moved
+      if (j > 0 && __any_sync(0xffffffffu, rescale)) {
+#pragma unroll 1
+        for (int c = 0; c < 4; ++c) {
+          uint32_t o[32];
+          tmem_ld32(tmem + lane_base + colO + 32 * c, o);
+          tmem_wait_ld();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+          tmem_st32(tmem + lane_base + colO + 32 * c, o);
+        }
+      }
+      // pass 2: exponentials, row sum, bf16 P over the first 64 columns of S
+      float sum = 0.f;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        uint32_t r[32];
+        tmem_ld32(tmem + lane_base + colS + 32 * c, r);
+        tmem_wait_ld();
+        uint32_t p[16];
+#pragma unroll
+        for (int i = 0; i < 32; i += 2) {
+          const int col = 32 * c + i;
+          const float e0 = col < valid ? fast_exp2(fmaf(__uint_as_float(r[i]), sl2, -m_ref)) : 0.f;
+          const float e1 = col + 1 < valid ? fast_exp2(fmaf(__uint_as_float(r[i + 1]), sl2, -m_ref)) : 0.f;
+          sum += e0 + e1;
+          p[i >> 1] = pack_bf16x2(e0, e1);
+        }
+        tmem_st16(tmem + lane_base + colS + 16 * c, p);
+      }
+      l = l * alpha + sum;
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(&p_full[wg]);
+    }
+    if (ok && mbar_wait_warp(&o_final[wg], 0, guard)) {
+      tc_fence_after();
+      const int64_t t = static_cast<int64_t>(2 * qt2 + wg) * kTile + row;
+      const int b = bh / args.heads, h = bh % args.heads;
+      const float inv_l = 1.0f / l;
+      __nv_bfloat16* dst = args.o + (static_cast<int64_t>(b) * T + t) * (args.heads * kHeadDim) + h * kHeadDim;
+#pragma unroll 1
+      for (int c = 0; c < 4; ++c) {
+        uint32_t o[32];
+        tmem_ld32(tmem + lane_base + colO + 32 * c, o);
+        tmem_wait_ld();
+        if (t < T) {
+          uint4* d4 = reinterpret_cast<uint4*>(dst + 32 * c);
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            uint4 u;
+            u.x = pack_bf16x2(__uint_as_float(o[8 * i + 0]) * inv_l, __uint_as_float(o[8 * i + 1]) * inv_l);
+            u.y = pack_bf16x2(__uint_as_float(o[8 * i + 2]) * inv_l, __uint_as_float(o[8 * i + 3]) * inv_l);
+            u.z = pack_bf16x2(__uint_as_float(o[8 * i + 4]) * inv_l, __uint_as_float(o[8 * i + 5]) * inv_l);
+            u.w = pack_bf16x2(__uint_as_float(o[8 * i + 6]) * inv_l, __uint_as_float(o[8 * i + 7]) * inv_l);
+            d4[i] = u;
+          }
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
 std::mutex g_mu;
 bool g_attr[64] = {};
+bool g_attr_pp[64] = {};
 
 }  // namespace
 
@@ -298,7 +590,9 @@ sal_status attention_launch(const void* q, const void* k, const void* v, int bat
     std::lock_guard<std::mutex> lk(g_mu);
     if (dev >= 0 && dev < 64 && !g_attr[dev]) {
       if (cudaFuncSetAttribute(attention_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               static_cast<int>(kSmem)) != cudaSuccess)
+                               static_cast<int>(kSmem)) != cudaSuccess ||
+          cudaFuncSetAttribute(attention_pp_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               static_cast<int>(kSmemPP)) != cudaSuccess)
         return SAL_ECUDA;
       g_attr[dev] = true;
     }
@@ -316,6 +610,20 @@ sal_status attention_launch(const void* q, const void* k, const void* v, int bat
   a.limit_ns = wait_limit_ns();
   a.status = device_status_ptr();
   if (!a.status) return SAL_ECUDA;
+  // Pick the kernel by waves of CTAs over the SMs: a two-tile CTA costs about 1.6 one-tile
+  // CTAs (measured), so it wins unless its coarser grain leaves a mostly empty last wave.
+  int sms = 148;
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const uint64_t ctas_pp = static_cast<uint64_t>((T + 2 * kTile - 1) / (2 * kTile)) * bh;
+  const uint64_t ctas_1 = static_cast<uint64_t>((T + kTile - 1) / kTile) * bh;
+  const double waves_pp = static_cast<double>((ctas_pp + sms - 1) / sms) * 1.6;
+  const double waves_1 = static_cast<double>((ctas_1 + sms - 1) / sms);
+  if (ctas_pp >= 120 && waves_pp < waves_1 && attention_pp_enabled()) {
+    const dim3 grid(static_cast<unsigned>((T + 2 * kTile - 1) / (2 * kTile)), static_cast<unsigned>(bh));
+    return launch_kernel(attention_pp_kernel, grid, dim3(320), kSmemPP, s, tq, tk, tv, a) == cudaSuccess
+               ? SAL_OK
+               : SAL_ECUDA;
+  }
   const dim3 grid(static_cast<unsigned>((T + kTile - 1) / kTile), static_cast<unsigned>(bh));
   return launch_kernel(attention_kernel, grid, dim3(192), kSmem, s, tq, tk, tv, a) == cudaSuccess ? SAL_OK
                                                                                         : SAL_ECUDA;

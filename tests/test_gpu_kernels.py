@@ -123,10 +123,23 @@ def test_qkv_rope(batch, T):
 
 # ---------------------------------------------------------------- attention
 
+def _two_tile_kernel(batch, T, sms=148):
+    """Which attention kernel the library picks: the two-tile ping-pong one when its CTAs
+    (256 query rows each) need fewer 'waves' over the SMs, at 1.6 one-tile CTAs apiece."""
+    bh = 10 * batch
+    pp, one = -(-T // 256) * bh, -(-T // 128) * bh
+    return pp >= 120 and -(-pp // sms) * 1.6 < -(-one // sms)
+
+
+# The first eight cases run the one-tile kernel, the last four the two-tile kernel
+# (checked below), including T = 129: a second query tile with one valid row and a last
+# key tile with one valid column.
 @pytest.mark.parametrize("batch,T,scale", [(1, 1, 1.0), (2, 7, 1.0), (1, 128, 1.0), (1, 129, 1.0),
-                                           (2, 383, 1.0), (1, 749, 1.0), (1, 749, 8.0), (1, 2000, 3.0)])
+                                           (2, 383, 1.0), (1, 749, 1.0), (1, 749, 8.0), (1, 2000, 3.0),
+                                           (30, 129, 1.0), (8, 1000, 1.0), (1, 3000, 8.0), (16, 749, 1.0)])
 def test_attention(batch, T, scale):
     api = _api()
+    assert _two_tile_kernel(batch, T) == (batch, T) in [(30, 129), (8, 1000), (1, 3000), (16, 749)]
     q, q64 = rand_bf16((batch, 10, T, 128), 50 + T, scale)
     k, k64 = rand_bf16((batch, 10, T, 128), 60 + T, 1.0)
     v, v64 = rand_bf16((batch, 10, T, 128), 70 + T, 1.0)
