@@ -20,6 +20,9 @@ Audits", flozi.net):
   seconds, nominally 375 per 30 s and 45,000 per hour, ignoring rounding at the ends.
 * [SERVE] section "Serving choices that change the audit": an hour of 16 kHz mono audio
   decodes to about 230.4 MB of float32.
+* [CHUNK] section "Local encoder windows, recording-wide language context": in training the
+  encoder runs on independent 30-second post-feature chunks with no attention across
+  their borders, and the chunk outputs are concatenated in order; pairs scale as T w.
 
 Readings where the pages are silent (each one is listed in the design notes):
 
@@ -71,7 +74,8 @@ __all__ = [
     "log_mel", "stack_frames", "linear", "layer_norm", "rms_norm", "rope_angles",
     "rope", "attention_probs", "attention", "gelu", "encoder_layer",
     "encoder_layer_rows", "encoder_forward", "stack_project", "encode",
-    "param_count", "rel_l2",
+    "param_count", "rel_l2", "chunk_bounds", "encoder_layer_chunked",
+    "encoder_layer_rows_chunked", "encoder_forward_chunked",
 ]
 
 
@@ -312,6 +316,39 @@ def encoder_layer_rows(x, lw, rows, dims: EncoderDims = DIMS):
     xr = x[rows] + linear(o, lw["w_o"], lw["b_o"])
     u = gelu(linear(layer_norm(xr, lw["ln2_g"], lw["ln2_b"]), lw["w1"], lw["b1"]))
     return xr + linear(u, lw["w2"], lw["b2"])
+
+
+def chunk_bounds(T: int, chunk: int):
+    """[(start, end)] of consecutive chunks of ``chunk`` positions; the last may be shorter."""
+    chunk = T if chunk <= 0 else chunk
+    return [(s, min(s + chunk, T)) for s in range(0, T, chunk)]
+
+
+def encoder_layer_chunked(x, lw, chunk: int, dims: EncoderDims = DIMS):
+    """One layer where each chunk of ``chunk`` positions is an independent sequence
+    ([CHUNK]): attention stays inside the chunk and RoPE positions restart at its start."""
+    x = _f64(x)
+    return np.concatenate([encoder_layer(x[a:b], lw, dims) for a, b in chunk_bounds(len(x), chunk)])
+
+
+def encoder_layer_rows_chunked(x, lw, rows, chunk: int, dims: EncoderDims = DIMS):
+    """:func:`encoder_layer_chunked` evaluated only at the positions ``rows``."""
+    x = _f64(x)
+    rows = np.asarray(rows)
+    out = np.empty((len(rows), x.shape[1]))
+    for a, b in chunk_bounds(len(x), chunk):
+        sel = np.nonzero((rows >= a) & (rows < b))[0]
+        if len(sel):
+            out[sel] = encoder_layer_rows(x[a:b], lw, rows[sel] - a, dims)
+    return out
+
+
+def encoder_forward_chunked(x0, weights, n_layers: int, chunk: int, dims: EncoderDims = DIMS):
+    """Chunked encoder: every chunk runs all layers on its own; final LayerNorm per position."""
+    x = _f64(x0)
+    for i in range(n_layers):
+        x = encoder_layer_chunked(x, weights["layers"][i], chunk, dims)
+    return layer_norm(x, weights["lnf_g"], weights["lnf_b"])
 
 
 def stack_project(stacked, weights):

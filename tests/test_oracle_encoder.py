@@ -234,3 +234,53 @@ def test_workload_shapes():
     assert O.position_count(wl["rec_1h"].n_samples) == 44999
     a = synth.WORKLOADS["tones_1s"].audio()
     assert a.shape == (1, 16000) and a.dtype == np.float32
+
+
+# ---------------------------------------------------------------- chunked encoder
+
+def test_chunk_bounds():
+    assert O.chunk_bounds(10, 4) == [(0, 4), (4, 8), (8, 10)]
+    assert O.chunk_bounds(10, 0) == [(0, 10)] and O.chunk_bounds(10, 10) == [(0, 10)]
+    assert O.chunk_bounds(44999, 375)[-1] == (44625, 44999) and len(O.chunk_bounds(44999, 375)) == 120
+
+
+def _small_layer(seed):
+    dims = O.EncoderDims(width=16, heads=2, head_dim=8, ffn=64, stack_in=32)
+    w = synth.weights_f32(synth.make_weights(1, seed=seed, width=16, ffn=64, head_dim=8,
+                                             stack_in=32, std=0.3, gain_std=0.3))
+    return dims, {k: np.asarray(v, np.float64) for k, v in w["layers"][0].items()}
+
+
+def test_chunk_equal_to_length_is_the_full_layer():
+    dims, lw = _small_layer(5)
+    x = np.random.default_rng(0).standard_normal((9, 16))
+    full = O.encoder_layer(x, lw, dims)
+    assert np.array_equal(O.encoder_layer_chunked(x, lw, 9, dims), full)
+    assert np.array_equal(O.encoder_layer_chunked(x, lw, 50, dims), full)
+
+
+def test_chunk_of_one_attends_to_itself():
+    """With one position per chunk the softmax has one key: the attention output is v, and
+    RoPE (position 0) is the identity."""
+    dims, lw = _small_layer(6)
+    x = np.random.default_rng(1).standard_normal((5, 16))
+    got = O.encoder_layer_chunked(x, lw, 1, dims)
+    h = O.layer_norm(x, lw["ln1_g"], lw["ln1_b"])
+    v = O.linear(h, lw["w_qkv"], lw["b_qkv"])[:, 32:]
+    x1 = x + O.linear(v, lw["w_o"], lw["b_o"])
+    ref = x1 + O.linear(O.gelu(O.linear(O.layer_norm(x1, lw["ln2_g"], lw["ln2_b"]), lw["w1"], lw["b1"])),
+                        lw["w2"], lw["b2"])
+    assert np.allclose(got, ref, rtol=1e-12, atol=1e-12)
+
+
+def test_chunks_are_independent_and_shift_invariant():
+    """A chunk's output depends only on its own positions (re-indexed from 0)."""
+    dims, lw = _small_layer(7)
+    x = np.random.default_rng(2).standard_normal((11, 16))
+    got = O.encoder_layer_chunked(x, lw, 4, dims)
+    assert np.allclose(got[4:8], O.encoder_layer(x[4:8], lw, dims), rtol=1e-12, atol=1e-12)
+    y = x.copy()
+    y[:4] += 1.0  # change the first chunk only
+    assert np.array_equal(O.encoder_layer_chunked(y, lw, 4, dims)[4:], got[4:])
+    rows = np.array([0, 3, 4, 10])
+    assert np.allclose(O.encoder_layer_rows_chunked(x, lw, rows, 4, dims), got[rows], rtol=1e-12, atol=1e-12)
