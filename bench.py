@@ -51,7 +51,16 @@ def frames(n_samples: int) -> int:
     return 0 if n_samples < 400 else 1 + (n_samples - 400) // 160
 
 
-def kernel_flops(kind: str, B: int, T: int) -> float:
+def attention_pairs(T: int, chunk: int = 0) -> int:
+    """Query-key pairs of one clip: T^2, or the sum of squared chunk lengths when attention
+    stays inside chunks of ``chunk`` positions."""
+    if chunk <= 0 or chunk >= T:
+        return T * T
+    full, rest = divmod(T, chunk)
+    return full * chunk * chunk + rest * rest
+
+
+def kernel_flops(kind: str, B: int, T: int, chunk: int = 0) -> float:
     """Algorithmic flops of ONE launch of a kernel kind (all clips of the batch)."""
     M = B * T
     return {
@@ -59,7 +68,7 @@ def kernel_flops(kind: str, B: int, T: int) -> float:
         "out_proj": 2.0 * M * 1280 * 1280,
         "ffn_up": 2.0 * M * 1280 * 5120,
         "ffn_down": 2.0 * M * 5120 * 1280,
-        "attention": float(ATTN_FLOPS_PER_T2_LAYER) * T * T * B,
+        "attention": float(ATTN_FLOPS_PER_T2_LAYER) * attention_pairs(T, chunk) * B,
     }.get(kind, 0.0)
 
 
@@ -72,8 +81,8 @@ def kernel_bytes(kind: str, B: int, T: int) -> float:
     }.get(kind, 0.0)
 
 
-def workload_flops(B: int, T: int, L: int) -> float:
-    return (GEMM_FLOPS_PER_POS_LAYER * B * T * L + ATTN_FLOPS_PER_T2_LAYER * T * T * B * L
+def workload_flops(B: int, T: int, L: int, chunk: int = 0) -> float:
+    return (GEMM_FLOPS_PER_POS_LAYER * B * T * L + ATTN_FLOPS_PER_T2_LAYER * attention_pairs(T, chunk) * B * L
             + STACK_PROJ_FLOPS_PER_POS * B * T)
 
 
@@ -282,13 +291,16 @@ def run_sal(args, wl: synth.Workload) -> dict | None:
     rec = ctypes.byref(dw.record)
     sp = s.cuda_stream
 
+    opts = api.sal_forward_options(args.chunk, None)
+
     def step(stream_ptr=sp):
         api._check("sal_frontend", lib.sal_frontend(wave_d.data_ptr(), N, B, logmel.data_ptr(),
                                                     stacked.data_ptr(), stream_ptr))
         api._check("sal_stack_project", lib.sal_stack_project(stacked.data_ptr(), B, T, rec,
                                                               x.data_ptr(), stream_ptr))
-        api._check("sal_encoder_forward", lib.sal_encoder_forward(
-            x.data_ptr(), B, T, rec, L, emb.data_ptr(), ws.data_ptr(), ws.numel(), stream_ptr))
+        api._check("sal_encoder_forward_ex", lib.sal_encoder_forward_ex(
+            x.data_ptr(), B, T, rec, L, emb.data_ptr(), ws.data_ptr(), ws.numel(), stream_ptr,
+            ctypes.byref(opts)))
 
     with torch.cuda.stream(s):
         for _ in range(max(args.warmup, 3)):
@@ -330,7 +342,7 @@ def run_sal(args, wl: synth.Workload) -> dict | None:
     if api.sal_last_device_status(s) != 0:
         raise RuntimeError("device wait timed out during the timed region")
     value = job_throughput(my_wl.audio_seconds * args.steps, world, total_s)
-    flops_step = workload_flops(B, T, L)
+    flops_step = workload_flops(B, T, L, args.chunk)
 
     # ---- per-kind launch durations (events around each launch, traced graph replays)
     kinds = {}
@@ -348,7 +360,8 @@ def run_sal(args, wl: synth.Workload) -> dict | None:
                                                         stacked.data_ptr(), cs))
             api._check("sal_stack_project", lib.sal_stack_project(stacked.data_ptr(), B, T, rec,
                                                                   x.data_ptr(), cs))
-            api.sal_encoder_forward_traced(x, B, T, dw, L, ws, emb, kind_id, evs, stream=cs)
+            api.sal_encoder_forward_ex(x, B, T, dw, L, workspace=ws, emb=emb, chunk=args.chunk, kind=kind_id,
+                                       events=evs, stream=cs)
         durs = []
         with torch.cuda.stream(s):
             for _ in range(k_steps):
@@ -365,15 +378,15 @@ def run_sal(args, wl: synth.Workload) -> dict | None:
     tensor_kinds = ["qkv", "attention", "out_proj", "ffn_up", "ffn_down"]
     dom = max(tensor_kinds, key=lambda k: kinds[k]["ms_per_step"])
     peaks = _peaks()
-    achieved = kernel_flops(dom, B, T) / (kinds[dom]["avg_ms"] / 1e3) / 1e12
+    achieved = kernel_flops(dom, B, T, args.chunk) / (kinds[dom]["avg_ms"] / 1e3) / 1e12
     roofline = {"kernel": dom, "bound": "tensor", "achieved": achieved, "peak": peaks["tflops"],
                 "unit": "TFLOP/s", "frac": achieved / peaks["tflops"], "traffic": None,
                 "peak_source": peaks["tflops_source"],
-                "per_launch_flops": kernel_flops(dom, B, T), "avg_launch_ms": kinds[dom]["avg_ms"]}
+                "per_launch_flops": kernel_flops(dom, B, T, args.chunk), "avg_launch_ms": kinds[dom]["avg_ms"]}
 
     # ---- end to end through sal_encode with pinned host buffers
     e2e = None
-    if not args.no_e2e:
+    if not args.no_e2e and args.chunk == 0:
         wave_h = torch.from_numpy(audio).pin_memory()
         emb_h = torch.empty((B, T, 1280), dtype=torch.bfloat16).pin_memory()
         ews = api.encode_workspace(B, N, dev)
@@ -414,6 +427,7 @@ def run_sal(args, wl: synth.Workload) -> dict | None:
         "warmup": args.warmup, "ms_per_step": step_ms_mean, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": {"workload": wl.name, "batch": B, "n_samples": N, "positions": T, "layers": L,
+                   "attention": f"chunks of {args.chunk} positions" if 0 < args.chunk < T else "whole clip",
                    "parallelism": f"dp{world} (independent clips per GPU)" if world > 1 else "single GPU",
                    "l2": "256 MiB buffer rewritten between timed steps", "graph": "one CUDA graph per step"},
         "tc_frac_step": flops_step / (step_ms_mean / 1e3) / 1e12 / peaks["tflops"],
@@ -453,6 +467,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=synth.WORKLOAD_ORDER)
     ap.add_argument("--impl", default="sal", choices=["sal", "reference"])
+    ap.add_argument("--chunk", type=int, default=0,
+                    help="attention within chunks of this many positions (0: whole clip)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()

@@ -136,7 +136,7 @@ size_t sal_encode_workspace_bytes(int batch, int64_t n_samples);
 sal_status sal_encode(const float* wave, int64_t n_samples, int batch, const sal_weights* w,
                       int n_layers, void* emb, void* workspace, size_t ws_bytes, void* stream);
 
-/* Kinds of kernel launch, for sal_encoder_forward_traced. */
+/* Kinds of kernel launch, for the event trace of sal_encoder_forward_ex. */
 typedef enum {
     SAL_KIND_ROPE_TABLE = 0,
     SAL_KIND_LAYERNORM = 1, /* LN1, LN2 and the final LN */
@@ -150,17 +150,32 @@ typedef enum {
 
 /* Event trace: for the i-th launch of kind `kind` inside the call (i < n_events / 2),
  * events[2 i] is recorded on the stream just before it and events[2 i + 1] just after.
- * Events are cudaEvent_t handles created by the caller. */
+ * Events are cudaEvent_t handles created (and recorded at least once) by the caller. */
 typedef struct {
     int kind;
     void* const* events;
     int n_events;
 } sal_trace;
 
-/* sal_encoder_forward with an optional event trace (trace may be NULL). */
-sal_status sal_encoder_forward_traced(float* x, int batch, int64_t T, const sal_weights* w,
-                                      int n_layers, void* emb, void* workspace, size_t ws_bytes,
-                                      void* stream, const sal_trace* trace);
+/* Options of sal_encoder_forward_ex.
+ *   chunk: attention and RoPE positions work per chunk of `chunk` positions of each clip
+ *          (the last chunk of a clip may be shorter); no attention crosses a chunk border
+ *          and positions restart at 0 in every chunk, so every chunk is encoded as an
+ *          independent sequence and the outputs come out concatenated in order. This is
+ *          the training-time scheme of the page "Nemotron 3.5 Transcribe: From Recorded
+ *          Speech to Dataset Audits", section "Local encoder windows, recording-wide
+ *          language context" (independent 30-second post-feature chunks = 375 positions).
+ *          chunk <= 0 or chunk >= T: attention over the whole clip (sal_encoder_forward).
+ *   trace: optional event trace (may be NULL). */
+typedef struct {
+    int64_t chunk;
+    const sal_trace* trace;
+} sal_forward_options;
+
+/* sal_encoder_forward with options (opts may be NULL: whole-clip attention, no trace). */
+sal_status sal_encoder_forward_ex(float* x, int batch, int64_t T, const sal_weights* w,
+                                  int n_layers, void* emb, void* workspace, size_t ws_bytes,
+                                  void* stream, const sal_forward_options* opts);
 
 /* Kernel launches this library has enqueued since the process started (all devices and
  * streams; a launch captured into a CUDA graph counts once, at capture). */
@@ -206,6 +221,11 @@ sal_status sal_qkv_rope(const void* h, int batch, int64_t T, const sal_layer* la
  * o [batch * T, 1280] bf16, o[b*T + t][128 h + d] = softmax(q k^T / sqrt(128)) v. */
 sal_status sal_attention(const void* q, const void* k, const void* v, int batch, int64_t T,
                          void* o, void* stream);
+
+/* sal_attention restricted to chunks of `chunk` positions of each clip (block-diagonal:
+ * row t attends to the keys of its own chunk only; chunk <= 0 or >= T: whole clip). */
+sal_status sal_attention_chunked(const void* q, const void* k, const void* v, int batch, int64_t T,
+                                 int64_t chunk, void* o, void* stream);
 
 /* sal_qkv_rope without a caller-supplied scratch buffer, for callers that cannot allocate
  * device memory when they run this step (a real-time audio callback or serving loop that

@@ -46,6 +46,10 @@ class sal_trace(ctypes.Structure):
                 ("n_events", ctypes.c_int)]
 
 
+class sal_forward_options(ctypes.Structure):
+    _fields_ = [("chunk", ctypes.c_int64), ("trace", ctypes.POINTER(sal_trace))]
+
+
 KIND_NAMES = ["rope_table", "layernorm", "qkv", "attention", "out_proj", "ffn_up", "ffn_down"]
 
 EXPORTS = {
@@ -61,10 +65,10 @@ EXPORTS = {
     "sal_encoder_forward": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int, ctypes.c_int64,
                                             ctypes.POINTER(sal_weights), ctypes.c_int, ctypes.c_void_p,
                                             ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]),
-    "sal_encoder_forward_traced": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int, ctypes.c_int64,
-                                                   ctypes.POINTER(sal_weights), ctypes.c_int, ctypes.c_void_p,
-                                                   ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p,
-                                                   ctypes.POINTER(sal_trace)]),
+    "sal_encoder_forward_ex": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int, ctypes.c_int64,
+                                               ctypes.POINTER(sal_weights), ctypes.c_int, ctypes.c_void_p,
+                                               ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p,
+                                               ctypes.POINTER(sal_forward_options)]),
     "sal_launch_count": (ctypes.c_uint64, []),
     "sal_encode_workspace_bytes": (ctypes.c_size_t, [ctypes.c_int, ctypes.c_int64]),
     "sal_encode": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.POINTER(sal_weights),
@@ -84,6 +88,8 @@ EXPORTS = {
                                              ctypes.c_void_p, ctypes.c_void_p]),
     "sal_attention": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int,
                                       ctypes.c_int64, ctypes.c_void_p, ctypes.c_void_p]),
+    "sal_attention_chunked": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int,
+                                              ctypes.c_int64, ctypes.c_int64, ctypes.c_void_p, ctypes.c_void_p]),
 }
 
 _lib = None
@@ -231,18 +237,27 @@ def sal_encoder_forward(x: torch.Tensor, batch: int, T: int, weights, n_layers: 
     return emb
 
 
-def sal_encoder_forward_traced(x: torch.Tensor, batch: int, T: int, weights, n_layers: int,
-                               workspace: torch.Tensor, emb: torch.Tensor, kind: int, events,
-                               stream=None) -> torch.Tensor:
-    """sal_encoder_forward with torch.cuda.Event pairs recorded around each launch of ``kind``."""
+def sal_encoder_forward_ex(x: torch.Tensor, batch: int, T: int, weights, n_layers: int,
+                           workspace: torch.Tensor | None = None, emb: torch.Tensor | None = None,
+                           chunk: int = 0, kind: int | None = None, events=None, stream=None) -> torch.Tensor:
+    """sal_encoder_forward with chunked attention (``chunk`` positions per chunk, 0 = whole
+    clip) and, optionally, torch.cuda.Event pairs recorded around each launch of ``kind``."""
     rec = weights.record if isinstance(weights, DeviceWeights) else weights
-    if any(e.cuda_event == 0 for e in events):
-        raise ValueError("record each torch.cuda.Event once before tracing (its handle is created lazily)")
-    handles = (ctypes.c_void_p * len(events))(*[e.cuda_event for e in events])
-    tr = sal_trace(kind, ctypes.cast(handles, ctypes.POINTER(ctypes.c_void_p)), len(events))
-    _check("sal_encoder_forward_traced", lib().sal_encoder_forward_traced(
+    if workspace is None:
+        workspace = encoder_workspace(batch, T, x.device)
+    if emb is None:
+        emb = torch.empty((batch * T, WIDTH), dtype=torch.bfloat16, device=x.device)
+    trace_p = None
+    if events:
+        if any(e.cuda_event == 0 for e in events):
+            raise ValueError("record each torch.cuda.Event once before tracing (its handle is created lazily)")
+        handles = (ctypes.c_void_p * len(events))(*[e.cuda_event for e in events])
+        tr = sal_trace(kind, ctypes.cast(handles, ctypes.POINTER(ctypes.c_void_p)), len(events))
+        trace_p = ctypes.pointer(tr)
+    opts = sal_forward_options(chunk, trace_p)
+    _check("sal_encoder_forward_ex", lib().sal_encoder_forward_ex(
         _ptr(x), batch, T, ctypes.byref(rec), n_layers, _ptr(emb), _ptr(workspace), workspace.numel(),
-        _stream(stream), ctypes.byref(tr)))
+        _stream(stream), ctypes.byref(opts)))
     return emb
 
 
@@ -310,6 +325,14 @@ def sal_attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, stream=None
     batch, H, T, hd = q.shape
     o = torch.empty((batch * T, H * hd), dtype=torch.bfloat16, device=q.device)
     _check("sal_attention", lib().sal_attention(_ptr(q), _ptr(k), _ptr(v), batch, T, _ptr(o), _stream(stream)))
+    return o
+
+
+def sal_attention_chunked(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, chunk: int, stream=None) -> torch.Tensor:
+    batch, H, T, hd = q.shape
+    o = torch.empty((batch * T, H * hd), dtype=torch.bfloat16, device=q.device)
+    _check("sal_attention_chunked", lib().sal_attention_chunked(_ptr(q), _ptr(k), _ptr(v), batch, T, chunk,
+                                                                _ptr(o), _stream(stream)))
     return o
 
 

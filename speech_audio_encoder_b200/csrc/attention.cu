@@ -48,12 +48,50 @@ bool attention_pp_enabled() {
 
 struct AttnArgs {
   int64_t T;
+  int64_t chunk;  // attention stays inside chunks of this many positions (T: whole clip)
   int heads;
   __nv_bfloat16* o;
   float scale_log2;
   uint64_t limit_ns;
   unsigned int* status;
 };
+
+// Key tiles [j0, j0 + n) that the query rows [q_lo, q_hi) can see: the union of their
+// chunks [floor(t / chunk) chunk, next chunk start) clipped to T.
+__device__ __forceinline__ void kv_tile_range(int64_t q_lo, int64_t q_hi, int64_t T, int64_t chunk, int& j0,
+                                              int& n) {
+  const int64_t kv_lo = (q_lo / chunk) * chunk;
+  int64_t kv_hi = ((q_hi - 1) / chunk + 1) * chunk;
+  if (kv_hi > T) kv_hi = T;
+  j0 = static_cast<int>(kv_lo / 128);
+  n = static_cast<int>((kv_hi + 127) / 128) - j0;
+}
+
+// Keys [lo, hi) that row t may attend to: its own chunk (empty for rows t >= T). Positions
+// fit in 32 bits (T <= 45000).
+__device__ __forceinline__ void row_range(int t, int T, int chunk, int& lo, int& hi) {
+  if (t >= T) {
+    lo = hi = 0;
+    return;
+  }
+  lo = (t / chunk) * chunk;
+  hi = lo + chunk < T ? lo + chunk : T;
+}
+
+// Columns [c_lo, c_hi) of key tile jt inside [lo, hi).
+__device__ __forceinline__ void tile_cols(int lo, int hi, int jt, int& c_lo, int& c_hi) {
+  const int base = jt * 128;
+  c_lo = min(max(lo - base, 0), 128);
+  c_hi = min(max(hi - base, 0), 128);
+}
+
+// Scores outside [c_lo, c_hi) of this 32-column chunk become -inf, so the unmasked softmax
+// that follows gives them weight 0 (run only on tiles that need a mask).
+__device__ __forceinline__ void mask_chunk(uint32_t (&r)[32], int col0, int c_lo, int c_hi) {
+#pragma unroll
+  for (int i = 0; i < 32; ++i)
+    if (col0 + i < c_lo || col0 + i >= c_hi) r[i] = 0xff800000u;  // -inf
+}
 
 __global__ void __launch_bounds__(192, 1)
     attention_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -80,7 +118,10 @@ __global__ void __launch_bounds__(192, 1)
   const int64_t T = args.T;
   const int bh = blockIdx.y;
   const int qt = blockIdx.x;
-  const int n_kv = static_cast<int>((T + kTile - 1) / kTile);
+  int j0, n_kv;
+  kv_tile_range(static_cast<int64_t>(qt) * kTile,
+                static_cast<int64_t>(qt) * kTile + kTile < T ? static_cast<int64_t>(qt) * kTile + kTile : T, T,
+                args.chunk, j0, n_kv);
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
@@ -123,11 +164,11 @@ __global__ void __launch_bounds__(192, 1)
         const uint32_t use_par = (j >> 1) & 1;
         if (!mbar_wait(&kv_empty[s], use_par ^ 1, guard)) break;
         mbar_arrive_expect_tx(&k_full[s], kTileBytes);
-        tma_load_3d(sK[s], &tmK, &k_full[s], 0, j * kTile, bh);
-        tma_load_3d(sK[s] + kBox, &tmK, &k_full[s], 64, j * kTile, bh);
+        tma_load_3d(sK[s], &tmK, &k_full[s], 0, (j0 + j) * kTile, bh);
+        tma_load_3d(sK[s] + kBox, &tmK, &k_full[s], 64, (j0 + j) * kTile, bh);
         mbar_arrive_expect_tx(&v_full[s], kTileBytes);
-        tma_load_3d(sV[s], &tmV, &v_full[s], 0, j * kTile, bh);
-        tma_load_3d(sV[s] + kBox, &tmV, &v_full[s], 64, j * kTile, bh);
+        tma_load_3d(sV[s], &tmV, &v_full[s], 0, (j0 + j) * kTile, bh);
+        tma_load_3d(sV[s] + kBox, &tmV, &v_full[s], 64, (j0 + j) * kTile, bh);
         issued |= 1u << s;
         par_k = (par_k & ~(1u << s)) | (use_par << s);
       }
@@ -191,6 +232,8 @@ __global__ void __launch_bounds__(192, 1)
     const float sl2 = args.scale_log2;
     float m_ref = -INFINITY, l = 0.f;
     bool ok = true;
+    int row_lo, row_hi;
+    row_range(qt * kTile + row, static_cast<int>(T), static_cast<int>(args.chunk), row_lo, row_hi);
     for (int j = 0; j < n_kv; ++j) {
       const int s = j & 1;
       if (!mbar_wait_warp(&s_full[s], (j >> 1) & 1, guard)) {
@@ -202,14 +245,17 @@ __global__ void __launch_bounds__(192, 1)
 #pragma unroll
       for (int c = 0; c < 4; ++c) tmem_ld32(tmem + lane_base + col_s(s) + 32 * c, r[c]);
       tmem_wait_ld();
-      const int64_t rem = T - static_cast<int64_t>(j) * kTile;
-      const int valid = static_cast<int>(rem < kTile ? rem : kTile);
+      int c_lo, c_hi;
+      tile_cols(row_lo, row_hi, j0 + j, c_lo, c_hi);
+      if (!__all_sync(0xffffffffu, c_lo == 0 && c_hi == kTile)) {
+#pragma unroll
+        for (int c = 0; c < 4; ++c) mask_chunk(r[c], 32 * c, c_lo, c_hi);
+      }
       float mx = -INFINITY;
 #pragma unroll
       for (int c = 0; c < 4; ++c)
 #pragma unroll
-        for (int i = 0; i < 32; ++i)
-          if (32 * c + i < valid) mx = fmaxf(mx, __uint_as_float(r[c][i]));
+        for (int i = 0; i < 32; ++i) mx = fmaxf(mx, __uint_as_float(r[c][i]));
       mx *= sl2;
       float alpha = 1.f;
       bool rescale = false;
@@ -220,15 +266,16 @@ __global__ void __launch_bounds__(192, 1)
         m_ref = mx;
         rescale = true;
       }
+      // a row that has seen no key yet keeps m_ref = -inf; its masked scores still give 0
+      const float m_use = m_ref == -INFINITY ? 0.f : m_ref;
       float sum = 0.f;
       uint32_t p[2][32];
 #pragma unroll
       for (int c = 0; c < 4; ++c)
 #pragma unroll
         for (int i = 0; i < 32; i += 2) {
-          const int col = 32 * c + i;
-          const float e0 = col < valid ? fast_exp2(fmaf(__uint_as_float(r[c][i]), sl2, -m_ref)) : 0.f;
-          const float e1 = col + 1 < valid ? fast_exp2(fmaf(__uint_as_float(r[c][i + 1]), sl2, -m_ref)) : 0.f;
+          const float e0 = fast_exp2(fmaf(__uint_as_float(r[c][i]), sl2, -m_use));
+          const float e1 = fast_exp2(fmaf(__uint_as_float(r[c][i + 1]), sl2, -m_use));
           sum += e0 + e1;
           p[c >> 1][(c & 1) * 16 + (i >> 1)] = pack_bf16x2(e0, e1);
         }
@@ -337,7 +384,11 @@ __global__ void __launch_bounds__(320, 1)
   const int64_t T = args.T;
   const int bh = blockIdx.y;
   const int qt2 = blockIdx.x;  // 256-row query block
-  const int n_kv = static_cast<int>((T + kTile - 1) / kTile);
+  int j0, n_kv;
+  kv_tile_range(static_cast<int64_t>(qt2) * 2 * kTile,
+                static_cast<int64_t>(qt2) * 2 * kTile + 2 * kTile < T ? static_cast<int64_t>(qt2) * 2 * kTile + 2 * kTile
+                                                                      : T,
+                T, args.chunk, j0, n_kv);
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
@@ -382,14 +433,14 @@ __global__ void __launch_bounds__(320, 1)
         const uint32_t use_par = (j >> 1) & 1;
         if (!mbar_wait(&k_empty[s], use_par ^ 1, guard)) break;
         mbar_arrive_expect_tx(&k_full[s], kTileBytes);
-        tma_load_3d(sK + s * kTileBytes, &tmK, &k_full[s], 0, j * kTile, bh);
-        tma_load_3d(sK + s * kTileBytes + kBox, &tmK, &k_full[s], 64, j * kTile, bh);
+        tma_load_3d(sK + s * kTileBytes, &tmK, &k_full[s], 0, (j0 + j) * kTile, bh);
+        tma_load_3d(sK + s * kTileBytes + kBox, &tmK, &k_full[s], 64, (j0 + j) * kTile, bh);
         issued_k |= 1u << s;
         par_k = (par_k & ~(1u << s)) | (use_par << s);
         if (!mbar_wait(&v_empty[s], use_par ^ 1, guard)) break;
         mbar_arrive_expect_tx(&v_full[s], kTileBytes);
-        tma_load_3d(sV + s * kTileBytes, &tmV, &v_full[s], 0, j * kTile, bh);
-        tma_load_3d(sV + s * kTileBytes + kBox, &tmV, &v_full[s], 64, j * kTile, bh);
+        tma_load_3d(sV + s * kTileBytes, &tmV, &v_full[s], 0, (j0 + j) * kTile, bh);
+        tma_load_3d(sV + s * kTileBytes + kBox, &tmV, &v_full[s], 64, (j0 + j) * kTile, bh);
         issued_v |= 1u << s;
         par_v = (par_v & ~(1u << s)) | (use_par << s);
       }
@@ -467,31 +518,39 @@ __global__ void __launch_bounds__(320, 1)
     const float sl2 = args.scale_log2;
     float m_ref = -INFINITY, l = 0.f;
     bool ok = true;
+    int row_lo, row_hi;
+    row_range((2 * qt2 + wg) * kTile + row, static_cast<int>(T), static_cast<int>(args.chunk), row_lo, row_hi);
     for (int j = 0; j < n_kv; ++j) {
       if (!mbar_wait_warp(&s_full[wg], j & 1, guard)) {
         ok = false;
         break;
       }
       tc_fence_after();
-      const int64_t rem = T - static_cast<int64_t>(j) * kTile;
-      const int valid = static_cast<int>(rem < kTile ? rem : kTile);
-      // pass 1: row maximum
+      int c_lo, c_hi;
+      tile_cols(row_lo, row_hi, j0 + j, c_lo, c_hi);
+      const bool masked = !__all_sync(0xffffffffu, c_lo == 0 && c_hi == kTile);
+      // pass 1: row maximum (tiles that need a mask take a compact separate loop, so the
+      // common unmasked body carries no mask code)
       float mx = -INFINITY;
+      if (!masked) {
 #pragma unroll
-      for (int c = 0; c < 4; c += 2) {
-        uint32_t ra[32], rb[32];
-        tmem_ld32(tmem + lane_base + colS + 32 * c, ra);
-        tmem_ld32(tmem + lane_base + colS + 32 * c + 32, rb);
-        tmem_wait_ld();
-        if (valid == kTile) {
+        for (int c = 0; c < 4; c += 2) {
+          uint32_t ra[32], rb[32];
+          tmem_ld32(tmem + lane_base + colS + 32 * c, ra);
+          tmem_ld32(tmem + lane_base + colS + 32 * c + 32, rb);
+          tmem_wait_ld();
 #pragma unroll
           for (int i = 0; i < 32; ++i) mx = fmaxf(mx, fmaxf(__uint_as_float(ra[i]), __uint_as_float(rb[i])));
-        } else {
+        }
+      } else {
+#pragma unroll 1
+        for (int c = 0; c < 4; ++c) {
+          uint32_t r[32];
+          tmem_ld32(tmem + lane_base + colS + 32 * c, r);
+          tmem_wait_ld();
+          mask_chunk(r, 32 * c, c_lo, c_hi);
 #pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            if (32 * c + i < valid) mx = fmaxf(mx, __uint_as_float(ra[i]));
-            if (32 * c + 32 + i < valid) mx = fmaxf(mx, __uint_as_float(rb[i]));
-          }
+          for (int i = 0; i < 32; ++i) mx = fmaxf(mx, __uint_as_float(r[i]));
         }
       }
       mx *= sl2;
@@ -517,22 +576,41 @@ __global__ void __launch_bounds__(320, 1)
         }
       }
       // pass 2: exponentials, row sum, bf16 P over the first 64 columns of S
+      const float m_use = m_ref == -INFINITY ? 0.f : m_ref;  // a row with no key seen yet
       float sum = 0.f;
+      if (!masked) {
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        uint32_t r[32];
-        tmem_ld32(tmem + lane_base + colS + 32 * c, r);
-        tmem_wait_ld();
-        uint32_t p[16];
+        for (int c = 0; c < 4; ++c) {
+          uint32_t r[32];
+          tmem_ld32(tmem + lane_base + colS + 32 * c, r);
+          tmem_wait_ld();
+          uint32_t p[16];
 #pragma unroll
-        for (int i = 0; i < 32; i += 2) {
-          const int col = 32 * c + i;
-          const float e0 = col < valid ? fast_exp2(fmaf(__uint_as_float(r[i]), sl2, -m_ref)) : 0.f;
-          const float e1 = col + 1 < valid ? fast_exp2(fmaf(__uint_as_float(r[i + 1]), sl2, -m_ref)) : 0.f;
-          sum += e0 + e1;
-          p[i >> 1] = pack_bf16x2(e0, e1);
+          for (int i = 0; i < 32; i += 2) {
+            const float e0 = fast_exp2(fmaf(__uint_as_float(r[i]), sl2, -m_use));
+            const float e1 = fast_exp2(fmaf(__uint_as_float(r[i + 1]), sl2, -m_use));
+            sum += e0 + e1;
+            p[i >> 1] = pack_bf16x2(e0, e1);
+          }
+          tmem_st16(tmem + lane_base + colS + 16 * c, p);
         }
-        tmem_st16(tmem + lane_base + colS + 16 * c, p);
+      } else {
+#pragma unroll 1
+        for (int c = 0; c < 4; ++c) {
+          uint32_t r[32];
+          tmem_ld32(tmem + lane_base + colS + 32 * c, r);
+          tmem_wait_ld();
+          mask_chunk(r, 32 * c, c_lo, c_hi);
+          uint32_t p[16];
+#pragma unroll
+          for (int i = 0; i < 32; i += 2) {
+            const float e0 = fast_exp2(fmaf(__uint_as_float(r[i]), sl2, -m_use));
+            const float e1 = fast_exp2(fmaf(__uint_as_float(r[i + 1]), sl2, -m_use));
+            sum += e0 + e1;
+            p[i >> 1] = pack_bf16x2(e0, e1);
+          }
+          tmem_st16(tmem + lane_base + colS + 16 * c, p);
+        }
       }
       l = l * alpha + sum;
       tmem_wait_st();
@@ -582,7 +660,7 @@ bool g_attr_pp[64] = {};
 }  // namespace
 
 sal_status attention_launch(const void* q, const void* k, const void* v, int batch, int64_t T,
-                            void* o, cudaStream_t s) {
+                            int64_t chunk, void* o, cudaStream_t s) {
   if (T == 0 || batch == 0) return SAL_OK;
   int dev = 0;
   cudaGetDevice(&dev);
@@ -604,6 +682,7 @@ sal_status attention_launch(const void* q, const void* k, const void* v, int bat
   if (!make_tmap_3d_bf16(&tv, v, kHeadDim, T, bh, 64, kTile, 1)) return SAL_ECUDA;
   AttnArgs a;
   a.T = T;
+  a.chunk = chunk > 0 && chunk < T ? chunk : T;
   a.heads = kHeads;
   a.o = static_cast<__nv_bfloat16*>(o);
   a.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(128.0));

@@ -39,8 +39,10 @@ struct GemmArgs {
   // QKV epilogue
   __nv_bfloat16 *q, *k, *v;
   const __nv_bfloat16 *qn_g, *kn_g;
-  const float* rope_cs;
+  const float* rope_cs;  // [2][rope_rows][64]: cos rows, then sin rows
   int64_t T;
+  int64_t chunk;         // positions restart every `chunk` positions of a clip
+  int64_t rope_rows;     // rows of the table = min(T, chunk)
   uint64_t limit_ns;
   unsigned int* status;
 };
@@ -233,9 +235,9 @@ __global__ void __launch_bounds__(192, 1)
       const int q4 = lane & 15;
       const float sg = lane >= 16 ? 1.f : -1.f;  // i < 64: a c - b s;  i >= 64: b c + a s
       float4 c1 = make_float4(1.f, 1.f, 1.f, 1.f), s1 = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (args.T > 1) {  // table row t = 1 holds cos / sin of theta_i itself
+      if (args.rope_rows > 1) {  // table row 1 holds cos / sin of theta_i itself
         c1 = __ldg(reinterpret_cast<const float4*>(args.rope_cs + 64) + q4);
-        s1 = __ldg(reinterpret_cast<const float4*>(args.rope_cs + (args.T + 1) * 64) + q4);
+        s1 = __ldg(reinterpret_cast<const float4*>(args.rope_cs + (args.rope_rows + 1) * 64) + q4);
       }
       for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
         const int rest = tile / args.splits;
@@ -282,6 +284,7 @@ __global__ void __launch_bounds__(192, 1)
           __nv_bfloat16* base = sec == 0 ? args.q : (sec == 1 ? args.k : args.v);
           if (nrows > 0) {
             int64_t b = row0 / args.T, t = row0 - b * args.T;
+            int64_t pos = t % args.chunk;  // RoPE position: restarts at every chunk
             __nv_bfloat16* dst = base + ((b * kHeads + head) * args.T + t) * kHeadDim;
             if (sec == 2) {
 #pragma unroll 4
@@ -301,8 +304,8 @@ __global__ void __launch_bounds__(192, 1)
             } else {
               const __nv_bfloat16* gp = (sec == 0 ? args.qn_g : args.kn_g) + 4 * lane;
               const float4 g4 = make_float4(bf16_at(gp, 0), bf16_at(gp, 1), bf16_at(gp, 2), bf16_at(gp, 3));
-              float4 c = __ldg(reinterpret_cast<const float4*>(args.rope_cs + t * 64) + q4);
-              float4 sn = __ldg(reinterpret_cast<const float4*>(args.rope_cs + (args.T + t) * 64) + q4);
+              float4 c = __ldg(reinterpret_cast<const float4*>(args.rope_cs + pos * 64) + q4);
+              float4 sn = __ldg(reinterpret_cast<const float4*>(args.rope_cs + (args.rope_rows + pos) * 64) + q4);
 #pragma unroll 4
               for (int r = 0; r < nrows; ++r) {
                 float4 v = scr[scr_chunk<128>(r, lane)];
@@ -318,13 +321,18 @@ __global__ void __launch_bounds__(192, 1)
                 o.y = pack_bf16x2(fmaf(sg * p.z, sn.z, v.z * c.z), fmaf(sg * p.w, sn.w, v.w * c.w));
                 reinterpret_cast<uint2*>(dst)[lane] = o;
                 dst += kHeadDim;
+                ++pos;
                 if (++t == args.T) {  // next clip: positions restart at 0
                   t = 0;
+                  pos = 0;
                   ++b;
                   dst = base + (b * kHeads + head) * args.T * kHeadDim;
+                }
+                if (pos == args.chunk || pos == 0) {  // a new clip or chunk starts at position 0
+                  pos = 0;
                   c = make_float4(1.f, 1.f, 1.f, 1.f);
                   sn = make_float4(0.f, 0.f, 0.f, 0.f);
-                } else {  // rotate by theta_i: angle (t + 1) theta_i
+                } else {  // rotate by theta_i: angle (pos + 1) theta_i
                   const float4 cc = c;
                   c.x = fmaf(cc.x, c1.x, -sn.x * s1.x); sn.x = fmaf(sn.x, c1.x, cc.x * s1.x);
                   c.y = fmaf(cc.y, c1.y, -sn.y * s1.y); sn.y = fmaf(sn.y, c1.y, cc.y * s1.y);
@@ -528,6 +536,8 @@ sal_status gemm_launch(int epilogue, const void* A, int64_t M, int K, const void
     a.kn_g = static_cast<const __nv_bfloat16*>(qkv->kn_g);
     a.rope_cs = qkv->rope_cs;
     a.T = qkv->T;
+    a.chunk = qkv->chunk > 0 && qkv->chunk < qkv->T ? qkv->chunk : qkv->T;
+    a.rope_rows = a.chunk;
   }
   const int BN = pick_bn(M, N, is_qkv);
   if (epilogue == SAL_EPI_RESID_F32) {

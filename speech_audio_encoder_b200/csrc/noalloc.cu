@@ -68,7 +68,7 @@ extern "C" sal_status sal_qkv_rope_noalloc(const void* h, int batch, int64_t T, 
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const sal_status st = rope_table_launch(cs, T, s);
   if (st != SAL_OK) return st;
-  QkvOut qo{q, k, v, layer->qn_g, layer->kn_g, cs, T};
+  QkvOut qo{q, k, v, layer->qn_g, layer->kn_g, cs, T, 0};
   return gemm_launch(kEpiQkv, h, static_cast<int64_t>(batch) * T, kWidth, layer->w_qkv, 3 * kWidth,
                      layer->b_qkv, nullptr, &qo, s);
 }

@@ -247,7 +247,7 @@ size_t sal_encoder_workspace_bytes(int batch, int64_t T) {
 
 sal_status sal_encoder_forward(float* x, int batch, int64_t T, const sal_weights* w, int n_layers, void* emb,
                                void* workspace, size_t ws_bytes, void* stream) {
-  return sal_encoder_forward_traced(x, batch, T, w, n_layers, emb, workspace, ws_bytes, stream, nullptr);
+  return sal_encoder_forward_ex(x, batch, T, w, n_layers, emb, workspace, ws_bytes, stream, nullptr);
 }
 
 namespace {
@@ -279,9 +279,10 @@ struct Tracer {
     if (!tr.after(kind)) return SAL_ECUDA;                  \
   } while (0)
 
-sal_status sal_encoder_forward_traced(float* x, int batch, int64_t T, const sal_weights* w, int n_layers,
-                                      void* emb, void* workspace, size_t ws_bytes, void* stream,
-                                      const sal_trace* trace) {
+sal_status sal_encoder_forward_ex(float* x, int batch, int64_t T, const sal_weights* w, int n_layers, void* emb,
+                                  void* workspace, size_t ws_bytes, void* stream, const sal_forward_options* opts) {
+  const sal_trace* trace = opts ? opts->trace : nullptr;
+  const int64_t chunk = (opts && opts->chunk > 0 && opts->chunk < T) ? opts->chunk : T;
   if (batch < 0 || T < 0 || !w || n_layers < 0 || n_layers > w->n_layers) return SAL_EINVAL;
   if (T > SAL_MAX_POSITIONS) return SAL_ESHAPE;
   if (batch == 0 || T == 0) return SAL_OK;
@@ -301,13 +302,13 @@ sal_status sal_encoder_forward_traced(float* x, int batch, int64_t T, const sal_
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   Tracer tr{trace, s};
   const int64_t M = static_cast<int64_t>(batch) * T;
-  if (n_layers > 0) SAL_TRACED(SAL_KIND_ROPE_TABLE, rope_table_launch(ws.rope, T, s));
+  if (n_layers > 0) SAL_TRACED(SAL_KIND_ROPE_TABLE, rope_table_launch(ws.rope, chunk, s));
   for (int i = 0; i < n_layers; ++i) {
     const sal_layer& L = w->layers[i];
     SAL_TRACED(SAL_KIND_LAYERNORM, layernorm_launch(x, M, L.ln1_g, L.ln1_b, ws.h, s));
-    QkvOut qo{ws.q, ws.k, ws.v, L.qn_g, L.kn_g, ws.rope, T};
+    QkvOut qo{ws.q, ws.k, ws.v, L.qn_g, L.kn_g, ws.rope, T, chunk};
     SAL_TRACED(SAL_KIND_QKV, gemm_launch(kEpiQkv, ws.h, M, kWidth, L.w_qkv, 3 * kWidth, L.b_qkv, nullptr, &qo, s));
-    SAL_TRACED(SAL_KIND_ATTENTION, attention_launch(ws.q, ws.k, ws.v, batch, T, ws.o, s));
+    SAL_TRACED(SAL_KIND_ATTENTION, attention_launch(ws.q, ws.k, ws.v, batch, T, chunk, ws.o, s));
     SAL_TRACED(SAL_KIND_OUT_PROJ,
                gemm_launch(SAL_EPI_RESID_F32, ws.o, M, kWidth, L.w_o, kWidth, L.b_o, x, nullptr, s));
     SAL_TRACED(SAL_KIND_LAYERNORM, layernorm_launch(x, M, L.ln2_g, L.ln2_b, ws.h, s));
@@ -406,13 +407,18 @@ sal_status sal_qkv_rope(const void* h, int batch, int64_t T, const sal_layer* la
   SAL_TRY(check_device());
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   SAL_TRY(rope_table_launch(rope_cs, T, s));
-  QkvOut qo{q, k, v, layer->qn_g, layer->kn_g, rope_cs, T};
+  QkvOut qo{q, k, v, layer->qn_g, layer->kn_g, rope_cs, T, 0};
   return gemm_launch(kEpiQkv, h, static_cast<int64_t>(batch) * T, kWidth, layer->w_qkv, 3 * kWidth,
                      layer->b_qkv, nullptr, &qo, s);
 }
 
 sal_status sal_attention(const void* q, const void* k, const void* v, int batch, int64_t T, void* o,
                          void* stream) {
+  return sal_attention_chunked(q, k, v, batch, T, 0, o, stream);
+}
+
+sal_status sal_attention_chunked(const void* q, const void* k, const void* v, int batch, int64_t T,
+                                 int64_t chunk, void* o, void* stream) {
   if (batch < 0 || T < 0) return SAL_EINVAL;
   if (T > SAL_MAX_POSITIONS) return SAL_ESHAPE;
   if (batch == 0 || T == 0) return SAL_OK;
@@ -420,7 +426,7 @@ sal_status sal_attention(const void* q, const void* k, const void* v, int batch,
   if (!q || !k || !v || !o || !aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o))
     return SAL_EINVAL;
   SAL_TRY(check_device());
-  return attention_launch(q, k, v, batch, T, o, static_cast<cudaStream_t>(stream));
+  return attention_launch(q, k, v, batch, T, chunk, o, static_cast<cudaStream_t>(stream));
 }
 
 }  // extern "C"

@@ -40,8 +40,9 @@ sal_status rope_table_launch(float* cs, int64_t T, cudaStream_t s);
 struct QkvOut {
   void *q, *k, *v;
   const void *qn_g, *kn_g;
-  const float* rope_cs;  // [T][64] cos then [T][64] sin
+  const float* rope_cs;  // [min(T, chunk)][64] cos then the same rows of sin
   int64_t T;
+  int64_t chunk;         // positions restart every `chunk` positions (<= 0: whole clip)
 };
 sal_status gemm_launch(int epilogue, const void* A, int64_t M, int K, const void* W, int N,
                        const void* bias, void* out, const QkvOut* qkv, cudaStream_t s);
@@ -49,7 +50,7 @@ constexpr int kEpiQkv = 100;  // internal epilogue id: QK-norm + RoPE scatter
 
 // attention.cu
 sal_status attention_launch(const void* q, const void* k, const void* v, int batch, int64_t T,
-                            void* o, cudaStream_t s);
+                            int64_t chunk, void* o, cudaStream_t s);
 
 // tensor maps (sal_api.cu)
 bool make_tmap_2d_bf16(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer,

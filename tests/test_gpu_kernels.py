@@ -139,7 +139,7 @@ def _two_tile_kernel(batch, T, sms=148):
                                            (30, 129, 1.0), (8, 1000, 1.0), (1, 3000, 8.0), (16, 749, 1.0)])
 def test_attention(batch, T, scale):
     api = _api()
-    assert _two_tile_kernel(batch, T) == (batch, T) in [(30, 129), (8, 1000), (1, 3000), (16, 749)]
+    assert _two_tile_kernel(batch, T) == ((batch, T) in [(30, 129), (8, 1000), (1, 3000), (16, 749)])
     q, q64 = rand_bf16((batch, 10, T, 128), 50 + T, scale)
     k, k64 = rand_bf16((batch, 10, T, 128), 60 + T, 1.0)
     v, v64 = rand_bf16((batch, 10, T, 128), 70 + T, 1.0)
