@@ -499,14 +499,16 @@ sal_status launch_epi(int BN, const GemmArgs& a, const void* A, const void* W, c
   }
 }
 
-// Largest tile width whose tile count fills the GPU; the narrowest otherwise.
+// Tile width: 256 when those tiles alone fill the GPU; otherwise 128. At small M (a 30 s
+// clip is 374 rows) every GEMM is one short wave bound by the L2 -> SM traffic of
+// re-reading A for every column tile and W for every row tile; measured at M = 374,
+// 128-wide tiles beat 64 (fewer A re-reads) and 256 (too few CTAs).
 int pick_bn(int64_t M, int N, bool qkv) {
   if (qkv) return 128;
   const int64_t mt = (M + 127) / 128;
-  const int sms = num_sms();
-  if (N % 256 == 0 && mt * (N / 256) >= sms) return 256;
-  if (N % 128 == 0 && (qkv || mt * (N / 128) >= sms)) return 128;
-  return qkv ? 128 : 64;
+  if (N % 256 == 0 && mt * (N / 256) >= num_sms()) return 256;
+  if (N % 128 == 0) return 128;
+  return 64;
 }
 
 }  // namespace
@@ -541,11 +543,14 @@ sal_status gemm_launch(int epilogue, const void* A, int64_t M, int K, const void
   }
   const int BN = pick_bn(M, N, is_qkv);
   if (epilogue == SAL_EPI_RESID_F32) {
-    // split K when the output tiles alone leave most SMs idle (partial sums are added
-    // atomically into the residual stream; the bias goes in with split 0)
+    // split K when the output tiles alone leave most SMs idle: up to 8 splits while the
+    // work units stay within two waves and each split keeps >= 4 k-blocks (partial sums
+    // are reduced into the residual stream by the TMA reduce-add; the bias goes in with
+    // split 0)
     const int64_t tiles = (M + 127) / 128 * (N / BN);
     const int kb = K / 64;
-    while (tiles * a.splits * 2 <= num_sms() && kb % (a.splits * 2) == 0 && a.splits < 8)
+    while (tiles * a.splits * 2 <= 2 * num_sms() && kb % (a.splits * 2) == 0 && kb / (a.splits * 2) >= 4 &&
+           a.splits < 8)
       a.splits *= 2;
   }
   switch (epilogue) {
