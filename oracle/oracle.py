@@ -20,6 +20,13 @@ Audits", flozi.net):
   seconds, nominally 375 per 30 s and 45,000 per hour, ignoring rounding at the ends.
 * [SERVE] section "Serving choices that change the audit": an hour of 16 kHz mono audio
   decodes to about 230.4 MB of float32.
+* [FUSE]  section "How audio and speakers reach the language model", the paragraphs after
+  the frontend one: speaker activity for eight slots, aligned to the ASR grid, thresholded
+  at 0.5, a learned LayerNorm over the speaker dimension, a fixed sinusoidal speaker kernel
+  (scale 1) mapping the eight slot indicators to width 1,280, summed into the ASR states;
+  then one learned linear projection (the identity connector) to the language width 2,688
+  (the width of the language backbone's block input, section on the released backbone).
+  The fusion equation itself is missing from the page text; readings 13-16 below.
 * [CHUNK] section "Local encoder windows, recording-wide language context": in training the
   encoder runs on independent 30-second post-feature chunks with no attention across
   their borders, and the chunk outputs are concatenated in order; pairs scale as T w.
@@ -42,6 +49,13 @@ Readings where the pages are silent (each one is listed in the design notes):
 10. RoPE rotates the pairs (i, i + 64) by t * 10000^(-2 i / 128), t = 0..T-1 per clip.
 11. attention is softmax(q k^T / sqrt(128)) v over the whole clip, no mask.
 12. GELU is the exact erf form; the FFN has two matrices (1280 -> 5120 -> 1280).
+13. speaker activity arrives already on the 80 ms ASR grid, P [T, 8] in [0, 1]; the
+    indicator is P > 0.5 (strict).
+14. the speaker LayerNorm normalises the 8 indicators of a position (eps 1e-5, gain and
+    bias of length 8).
+15. the speaker kernel is the sinusoidal table K[s, 2i] = sin(s w_i), K[s, 2i+1] = cos(s w_i),
+    w_i = 10000^(-2i/1280), s = 0..7; fused = H + 1 * LN(indicators) K.
+16. the connector is x W^T + b with W [2688, 1280].
 """
 from __future__ import annotations
 
@@ -65,6 +79,8 @@ LN_EPS = 1e-5        # reading 8
 QK_EPS = 1e-6        # reading 9
 ROPE_BASE = 10000.0  # reading 10
 MAX_POSITIONS = 45000  # one hour at 12.5 positions/s [POS]
+N_SLOTS = 8            # speaker slots [FUSE]
+LLM_WIDTH = 2688       # language width [FUSE]
 
 __all__ = [
     "SAMPLE_RATE", "WIN", "HOP", "NFFT", "NBINS", "NMEL", "STACK", "LOG_FLOOR",
@@ -75,7 +91,8 @@ __all__ = [
     "rope", "attention_probs", "attention", "gelu", "encoder_layer",
     "encoder_layer_rows", "encoder_forward", "stack_project", "encode",
     "param_count", "rel_l2", "chunk_bounds", "encoder_layer_chunked",
-    "encoder_layer_rows_chunked", "encoder_forward_chunked",
+    "encoder_layer_rows_chunked", "encoder_forward_chunked", "N_SLOTS", "LLM_WIDTH",
+    "speaker_kernel", "speaker_fuse", "connector",
 ]
 
 
@@ -349,6 +366,27 @@ def encoder_forward_chunked(x0, weights, n_layers: int, chunk: int, dims: Encode
     for i in range(n_layers):
         x = encoder_layer_chunked(x, weights["layers"][i], chunk, dims)
     return layer_norm(x, weights["lnf_g"], weights["lnf_b"])
+
+
+def speaker_kernel(n_slots: int = N_SLOTS, width: int = 1280) -> np.ndarray:
+    """Fixed sinusoidal speaker kernel K [n_slots, width] (reading 15)."""
+    s = np.arange(n_slots, dtype=np.float64)[:, None]
+    w = ROPE_BASE ** (-2.0 * np.arange(width // 2, dtype=np.float64) / width)[None, :]
+    K = np.empty((n_slots, width), dtype=np.float64)
+    K[:, 0::2] = np.sin(s * w)
+    K[:, 1::2] = np.cos(s * w)
+    return K
+
+
+def speaker_fuse(H, P, g, b, scale: float = 1.0):
+    """H + scale * LN_slots(P > 0.5) K ([FUSE], readings 13-15). H [T, 1280], P [T, 8]."""
+    A = (np.asarray(P, dtype=np.float64) > 0.5).astype(np.float64)
+    return _f64(H) + scale * layer_norm(A, g, b) @ speaker_kernel(A.shape[1], H.shape[1])
+
+
+def connector(x, w, b):
+    """The identity connector: one linear projection to the language width ([FUSE], 16)."""
+    return linear(x, w, b)
 
 
 def stack_project(stacked, weights):

@@ -284,3 +284,48 @@ def test_chunks_are_independent_and_shift_invariant():
     assert np.array_equal(O.encoder_layer_chunked(y, lw, 4, dims)[4:], got[4:])
     rows = np.array([0, 3, 4, 10])
     assert np.allclose(O.encoder_layer_rows_chunked(x, lw, rows, 4, dims), got[rows], rtol=1e-12, atol=1e-12)
+
+
+# ---------------------------------------------------------------- speaker fusion and connector
+
+def test_speaker_kernel_closed_forms():
+    K = O.speaker_kernel()
+    assert K.shape == (8, 1280)
+    assert np.array_equal(K[0, 0::2], np.zeros(640)) and np.array_equal(K[0, 1::2], np.ones(640))
+    assert np.allclose(K[:, 0::2] ** 2 + K[:, 1::2] ** 2, 1.0, atol=1e-15)
+    for s_ in (1, 3, 7):
+        assert K[s_, 0] == pytest.approx(math.sin(s_)) and K[s_, 1] == pytest.approx(math.cos(s_))
+        i = 300
+        w = 10000.0 ** (-2.0 * i / 1280)
+        assert K[s_, 2 * i] == pytest.approx(math.sin(s_ * w)) and K[s_, 2 * i + 1] == pytest.approx(math.cos(s_ * w))
+
+
+def test_speaker_fuse_brute_force_and_special_cases():
+    rng = np.random.default_rng(3)
+    H = rng.standard_normal((6, 1280))
+    P = rng.uniform(0, 1, (6, 8))
+    P[0] = 0.5  # exactly at the threshold: inactive (strict)
+    g, b = 1 + 0.1 * rng.standard_normal(8), 0.1 * rng.standard_normal(8)
+    got = O.speaker_fuse(H, P, g, b)
+    for t in range(6):
+        a = [1.0 if P[t, s_] > 0.5 else 0.0 for s_ in range(8)]
+        mu = sum(a) / 8
+        var = sum((v - mu) ** 2 for v in a) / 8
+        ah = [(a[s_] - mu) / math.sqrt(var + 1e-5) * g[s_] + b[s_] for s_ in range(8)]
+        for c in (0, 1, 2, 639, 1278, 1279):
+            i = c // 2
+            w = 10000.0 ** (-2.0 * i / 1280)
+            k = [math.sin(s_ * w) if c % 2 == 0 else math.cos(s_ * w) for s_ in range(8)]
+            assert got[t, c] == pytest.approx(H[t, c] + sum(ah[s_] * k[s_] for s_ in range(8)), abs=1e-12)
+    # no active slot (or all active): LayerNorm of a constant is beta, so H + beta K
+    K = O.speaker_kernel()
+    assert np.allclose(O.speaker_fuse(H, np.zeros((6, 8)), g, b), H + b @ K, atol=1e-12)
+    assert np.allclose(O.speaker_fuse(H, np.ones((6, 8)), g, b), H + b @ K, atol=1e-12)
+
+
+def test_connector_is_a_linear_map_to_the_language_width():
+    rng = np.random.default_rng(4)
+    x, W, b = rng.standard_normal((3, 1280)), rng.standard_normal((2688, 1280)), rng.standard_normal(2688)
+    y = O.connector(x, W, b)
+    assert y.shape == (3, O.LLM_WIDTH)
+    assert np.allclose(y[1, 7], sum(x[1, i] * W[7, i] for i in range(1280)) + b[7])
