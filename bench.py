@@ -380,7 +380,8 @@ def run_sal(args, wl: synth.Workload) -> dict | None:
     peaks = _peaks()
     achieved = kernel_flops(dom, B, T, args.chunk) / (kinds[dom]["avg_ms"] / 1e3) / 1e12
     roofline = {"kernel": dom, "bound": "tensor", "achieved": achieved, "peak": peaks["tflops"],
-                "unit": "TFLOP/s", "frac": achieved / peaks["tflops"], "traffic": None,
+                "unit": "TFLOP/s", "frac": achieved / peaks["tflops"],
+                "traffic": _traffic(dom, wl.name) if args.chunk == 0 else None,
                 "peak_source": peaks["tflops_source"],
                 "per_launch_flops": kernel_flops(dom, B, T, args.chunk), "avg_launch_ms": kinds[dom]["avg_ms"]}
 
@@ -438,6 +439,20 @@ def run_sal(args, wl: synth.Workload) -> dict | None:
         "gpu_launches": int(launches_per_step * args.steps),
         "clocks": clk,
     }
+
+
+def _traffic(kind: str, workload: str):
+    """DRAM bytes per launch of `kind` from the committed ncu summary, or None when the
+    kernel's source changed since that capture or the capture was of another workload."""
+    import hashlib
+    try:
+        rec = json.load(open(os.path.join(ROOT, "profiles", "roofline_traffic.json")))[kind]
+        src = open(os.path.join(ROOT, rec["source"]), "rb").read()
+    except (OSError, KeyError, ValueError):
+        return None
+    if rec.get("workload") != workload or hashlib.sha256(src).hexdigest()[:16] != rec.get("sha256_16"):
+        return None
+    return rec["dram_bytes_per_launch"]
 
 
 def _nvsmi_id(local: int) -> str:

@@ -227,6 +227,29 @@ sal_status sal_attention(const void* q, const void* k, const void* v, int batch,
 sal_status sal_attention_chunked(const void* q, const void* k, const void* v, int batch, int64_t T,
                                  int64_t chunk, void* o, void* stream);
 
+/* ---------------------------------------------------------------------------------
+ * After the encoder (page "Nemotron 3.5 Transcribe: From Recorded Speech to Dataset
+ * Audits", section "How audio and speakers reach the language model"): speaker-activity
+ * fusion into the encoder states, then the identity connector to the language width.
+ * --------------------------------------------------------------------------------- */
+
+#define SAL_SPEAKER_SLOTS 8
+#define SAL_LLM_WIDTH 2688
+
+/* out = H + LN_8(P > 0.5) K, per position: P [rows, 8] float32 slot activities already on
+ * the 80 ms ASR grid; the indicators P > 0.5 are normalised over the 8 slots (LayerNorm,
+ * eps 1e-5, gain g [8] and bias b [8] bf16) and mapped to width 1280 by the fixed
+ * sinusoidal speaker kernel K[s, 2i] = sin(s w_i), K[s, 2i+1] = cos(s w_i),
+ * w_i = 10000^(-2i/1280), scale 1. H and out are [rows, 1280] bf16 (may alias). The page
+ * states the steps but its equation is missing from the text; this is the reading. */
+sal_status sal_speaker_fuse(const void* H, const float* P, int64_t rows, const void* g, const void* b,
+                            void* out, void* stream);
+
+/* The identity connector: out [rows, 2688] bf16 = x [rows, 1280] bf16 W^T + bias, with
+ * W [2688, 1280] and bias [2688] bf16 (one learned linear projection, no downsampling). */
+sal_status sal_connector(const void* x, int64_t rows, const void* W, const void* bias, void* out,
+                         void* stream);
+
 /* sal_qkv_rope without a caller-supplied scratch buffer, for callers that cannot allocate
  * device memory when they run this step (a real-time audio callback or serving loop that
  * must not stall or fail on cudaMalloc, a plugin host that forbids device allocations

@@ -86,6 +86,10 @@ EXPORTS = {
     "sal_qkv_rope_noalloc": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int, ctypes.c_int64,
                                              ctypes.POINTER(sal_layer), ctypes.c_void_p, ctypes.c_void_p,
                                              ctypes.c_void_p, ctypes.c_void_p]),
+    "sal_speaker_fuse": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64, ctypes.c_void_p,
+                                         ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p]),
+    "sal_connector": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int64, ctypes.c_void_p, ctypes.c_void_p,
+                                      ctypes.c_void_p, ctypes.c_void_p]),
     "sal_attention": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int,
                                       ctypes.c_int64, ctypes.c_void_p, ctypes.c_void_p]),
     "sal_attention_chunked": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int,
@@ -334,6 +338,24 @@ def sal_attention_chunked(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, chu
     _check("sal_attention_chunked", lib().sal_attention_chunked(_ptr(q), _ptr(k), _ptr(v), batch, T, chunk,
                                                                 _ptr(o), _stream(stream)))
     return o
+
+
+def sal_speaker_fuse(H: torch.Tensor, P: torch.Tensor, g: torch.Tensor, b: torch.Tensor,
+                     out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """H [rows, 1280] bf16, P [rows, 8] f32 -> H + LN_8(P > 0.5) K (bf16)."""
+    if out is None:
+        out = torch.empty_like(H)
+    _check("sal_speaker_fuse", lib().sal_speaker_fuse(_ptr(H), _ptr(P), H.shape[0], _ptr(g), _ptr(b), _ptr(out),
+                                                      _stream(stream)))
+    return out
+
+
+def sal_connector(x: torch.Tensor, W: torch.Tensor, bias: torch.Tensor, stream=None) -> torch.Tensor:
+    """x [rows, 1280] bf16 -> [rows, 2688] bf16."""
+    out = torch.empty((x.shape[0], 2688), dtype=torch.bfloat16, device=x.device)
+    _check("sal_connector", lib().sal_connector(_ptr(x), x.shape[0], _ptr(W), _ptr(bias), _ptr(out),
+                                                _stream(stream)))
+    return out
 
 
 def sal_last_device_status(stream=None) -> int:

@@ -7,8 +7,19 @@
 // RoPE table: cos and sin of t * 10000^(-2 i / 128), i < 64, t < T. The angle reaches
 // 4.5e4 rad at one hour, where fp32 would lose ~3 digits, so it is formed and reduced in
 // fp64 before the fp32 table entry is written.
+//
+// Speaker-activity fusion (page "Nemotron 3.5 Transcribe: From Recorded Speech to Dataset
+// Audits", section "How audio and speakers reach the language model", the paragraph on
+// Sortformer activity): per position, the eight slot activities are thresholded at 0.5,
+// normalised by a LayerNorm over the slots, mapped to width 1280 by the fixed sinusoidal
+// speaker kernel K[s, 2i] = sin(s w_i), K[s, 2i+1] = cos(s w_i), w_i = 10000^(-2i/1280)
+// (scale 1), and added to the encoder state. One warp per position; K (40 KB, built in
+// fp64 on the host) sits in shared memory.
 #include <cuda_bf16.h>
 #include <math.h>
+
+#include <cmath>
+#include <mutex>
 
 #include "sal_internal.h"
 #include "sal_ptx.cuh"
@@ -83,7 +94,112 @@ __global__ void rope_table_kernel(float* __restrict__ cs, int64_t T) {
   cs[T * 64 + idx] = static_cast<float>(s);
 }
 
+constexpr int kSlots = 8;
+struct SpeakerKernel {
+  float k[kSlots][kWidth];
+};
+__device__ SpeakerKernel g_speaker_kernel;
+
+__global__ void __launch_bounds__(256) speaker_fuse_kernel(const __nv_bfloat16* __restrict__ H,
+                                                           const float* __restrict__ P, int64_t rows,
+                                                           const __nv_bfloat16* __restrict__ g,
+                                                           const __nv_bfloat16* __restrict__ b,
+                                                           __nv_bfloat16* __restrict__ out) {
+  extern __shared__ __align__(16) float sk[];  // [8][1280]
+  {
+    const float4* src = reinterpret_cast<const float4*>(&g_speaker_kernel);
+    float4* dst = reinterpret_cast<float4*>(sk);
+    for (int i = threadIdx.x; i < kSlots * kWidth / 4; i += blockDim.x) dst[i] = src[i];
+  }
+  __syncthreads();
+  pdl_wait();
+  pdl_trigger();
+  const int lane = threadIdx.x & 31;
+  const int s = lane & 7;
+  const float gs = __bfloat162float(g[s]), bs = __bfloat162float(b[s]);
+  const int64_t warps = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
+  for (int64_t row = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5); row < rows;
+       row += warps) {
+    // every group of 8 lanes holds the 8 slots of this position
+    const float a = P[row * kSlots + s] > 0.5f ? 1.f : 0.f;
+    float sum = a;
+#pragma unroll
+    for (int o = 1; o < kSlots; o <<= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+    const float mu = sum * (1.0f / kSlots);
+    float q = (a - mu) * (a - mu);
+#pragma unroll
+    for (int o = 1; o < kSlots; o <<= 1) q += __shfl_xor_sync(0xffffffffu, q, o);
+    const float ah = (a - mu) / sqrtf(q * (1.0f / kSlots) + 1e-5f) * gs + bs;
+    float w[kSlots];
+#pragma unroll
+    for (int t = 0; t < kSlots; ++t) w[t] = __shfl_sync(0xffffffffu, ah, t);
+    const uint2* hr = reinterpret_cast<const uint2*>(H + row * kWidth);
+    uint2* orow = reinterpret_cast<uint2*>(out + row * kWidth);
+#pragma unroll
+    for (int i = 0; i < kWidth / 128; ++i) {
+      const int c4 = lane + 32 * i;  // columns 4 c4 .. 4 c4 + 3
+      const uint2 hv = hr[c4];
+      float o0 = __uint_as_float(hv.x << 16), o1 = __uint_as_float(hv.x & 0xFFFF0000u);
+      float o2 = __uint_as_float(hv.y << 16), o3 = __uint_as_float(hv.y & 0xFFFF0000u);
+#pragma unroll
+      for (int t = 0; t < kSlots; ++t) {
+        const float4 kv = reinterpret_cast<const float4*>(sk + t * kWidth)[c4];
+        o0 = fmaf(w[t], kv.x, o0);
+        o1 = fmaf(w[t], kv.y, o1);
+        o2 = fmaf(w[t], kv.z, o2);
+        o3 = fmaf(w[t], kv.w, o3);
+      }
+      __nv_bfloat162 p0 = __floats2bfloat162_rn(o0, o1), p1 = __floats2bfloat162_rn(o2, o3);
+      uint2 ov;
+      ov.x = *reinterpret_cast<uint32_t*>(&p0);
+      ov.y = *reinterpret_cast<uint32_t*>(&p1);
+      orow[c4] = ov;
+    }
+  }
+}
+
+std::mutex g_spk_mu;
+bool g_spk_done[64] = {};
+
+sal_status ensure_speaker_kernel() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return SAL_ECUDA;
+  std::lock_guard<std::mutex> lk(g_spk_mu);
+  if (g_spk_done[dev]) return SAL_OK;
+  static SpeakerKernel host;
+  for (int s = 0; s < kSlots; ++s)
+    for (int i = 0; i < kWidth / 2; ++i) {
+      const double w = std::pow(10000.0, -2.0 * i / kWidth);
+      host.k[s][2 * i] = static_cast<float>(std::sin(s * w));
+      host.k[s][2 * i + 1] = static_cast<float>(std::cos(s * w));
+    }
+  if (cudaMemcpyToSymbol(g_speaker_kernel, &host, sizeof(host)) != cudaSuccess) return SAL_ECUDA;
+  if (cudaFuncSetAttribute(speaker_fuse_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(sizeof(SpeakerKernel))) != cudaSuccess)
+    return SAL_ECUDA;
+  g_spk_done[dev] = true;
+  return SAL_OK;
+}
+
 }  // namespace
+
+sal_status speaker_fuse_launch(const void* H, const float* P, int64_t rows, const void* g, const void* b, void* out,
+                               cudaStream_t s) {
+  if (rows == 0) return SAL_OK;
+  const sal_status st = ensure_speaker_kernel();
+  if (st != SAL_OK) return st;
+  int sms = 148;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int64_t want = (rows + 7) / 8;
+  const unsigned grid = static_cast<unsigned>(want < 4 * sms ? want : 4 * sms);
+  return launch_kernel(speaker_fuse_kernel, dim3(grid), dim3(256), sizeof(SpeakerKernel), s,
+                       static_cast<const __nv_bfloat16*>(H), P, rows, static_cast<const __nv_bfloat16*>(g),
+                       static_cast<const __nv_bfloat16*>(b), static_cast<__nv_bfloat16*>(out)) == cudaSuccess
+             ? SAL_OK
+             : SAL_ECUDA;
+}
 
 sal_status layernorm_launch(const float* x, int64_t rows, const void* g, const void* b, void* y,
                             cudaStream_t s) {

@@ -412,6 +412,27 @@ sal_status sal_qkv_rope(const void* h, int batch, int64_t T, const sal_layer* la
                      layer->b_qkv, nullptr, &qo, s);
 }
 
+sal_status sal_speaker_fuse(const void* H, const float* P, int64_t rows, const void* g, const void* b, void* out,
+                            void* stream) {
+  if (rows < 0) return SAL_EINVAL;
+  if (rows == 0) return SAL_OK;
+  if (!H || !P || !g || !b || !out || !aligned16(H) || !aligned16(P) || !aligned16(g) || !aligned16(b) ||
+      !aligned16(out))
+    return SAL_EINVAL;
+  SAL_TRY(check_device());
+  return speaker_fuse_launch(H, P, rows, g, b, out, static_cast<cudaStream_t>(stream));
+}
+
+sal_status sal_connector(const void* x, int64_t rows, const void* W, const void* bias, void* out, void* stream) {
+  if (rows < 0) return SAL_EINVAL;
+  if (rows == 0) return SAL_OK;
+  if (!x || !W || !bias || !out || !aligned16(x) || !aligned16(W) || !aligned16(bias) || !aligned16(out))
+    return SAL_EINVAL;
+  SAL_TRY(check_device());
+  return gemm_launch(SAL_EPI_STORE_BF16, x, rows, kWidth, W, SAL_LLM_WIDTH, bias, out, nullptr,
+                     static_cast<cudaStream_t>(stream));
+}
+
 sal_status sal_attention(const void* q, const void* k, const void* v, int batch, int64_t T, void* o,
                          void* stream) {
   return sal_attention_chunked(q, k, v, batch, T, 0, o, stream);

@@ -35,6 +35,8 @@ sal_status frontend_launch(const float* wave, int64_t n_samples, int batch, int6
 sal_status layernorm_launch(const float* x, int64_t rows, const void* g, const void* b, void* y,
                             cudaStream_t s);
 sal_status rope_table_launch(float* cs, int64_t T, cudaStream_t s);
+sal_status speaker_fuse_launch(const void* H, const float* P, int64_t rows, const void* g, const void* b, void* out,
+                               cudaStream_t s);
 
 // gemm.cu
 struct QkvOut {

@@ -3,7 +3,7 @@
     python -m speech_audio_encoder_b200.kernel_bench KIND [--batch B] [--T T] [--reps R]
 
 KIND is one of frontend, stack_proj, layernorm, qkv, attention, out_proj, ffn_up, ffn_down,
-linear (any --N, --K, --epi).
+speaker_fuse, connector, linear (any --N, --K, --epi).
 Each repetition is one launch (qkv also launches the small RoPE-table kernel). The
 repetitions are captured once as a CUDA graph and the replay is timed with CUDA events on
 the launching stream after warm-up (eager launches from Python would measure the host). Prints one JSON line with the
@@ -70,6 +70,22 @@ def main():
 
         def run():
             api.sal_attention(q, k, v)
+    elif a.kind == "speaker_fuse":
+        H = _bf16((M, 1280), 7, 1.0)
+        P = torch.from_numpy(synth.speaker_activity(M, 1)).cuda()
+        g, b = _bf16((8,), 8, 1.0), _bf16((8,), 9, 0.1)
+        out = torch.empty_like(H)
+        bytes_ = M * (1280 * 2 * 2 + 8 * 4)
+
+        def run():
+            api.sal_speaker_fuse(H, P, g, b, out=out)
+    elif a.kind == "connector":
+        x = _bf16((M, 1280), 10, 1.0)
+        W, bias = _bf16((2688, 1280), 11, 0.02), _bf16((2688,), 12, 0.02)
+        flops = 2.0 * M * 2688 * 1280
+
+        def run():
+            api.sal_connector(x, W, bias)
     elif a.kind == "linear":
         K, N, epi = a.K, a.N, a.epi
         A = _bf16((M, K), 4, 1.0)

@@ -186,3 +186,37 @@ def random_bf16(shape, seed: int, std: float = 1.0):
     """N(0, std^2) values rounded to bf16: (bits, float32 values)."""
     b = bf16_bits(np.random.default_rng(seed).normal(0.0, std, shape))
     return b, bf16_to_f32(b)
+
+
+# ----------------------------------------------------------------------------- speaker fusion inputs
+
+def speaker_activity(T: int, seed: int, n_slots: int = 8, n_speakers: int = 3) -> np.ndarray:
+    """[T, n_slots] float32 activities on the 80 ms grid: speakers take turns of 1-10 s
+    (12-125 positions) with some overlap, plus N(0, 0.2) noise clipped to [0, 1]; unused
+    slots stay near 0. A few entries are exactly 0.5 (the threshold)."""
+    rng = np.random.default_rng(seed)
+    P = np.zeros((T, n_slots))
+    t = 0
+    while t < T:
+        n = int(rng.integers(12, 126))
+        spk = int(rng.integers(0, n_speakers))
+        P[t:t + n, spk] = 1.0
+        if rng.uniform() < 0.2:  # an overlapping second speaker
+            P[t + n // 2:t + n, (spk + 1) % n_speakers] = 1.0
+        t += n
+    P = np.clip(P + rng.normal(0.0, 0.2, P.shape), 0.0, 1.0)
+    P[rng.integers(0, T, max(1, T // 50)), rng.integers(0, n_slots, max(1, T // 50))] = 0.5
+    return P.astype(np.float32)
+
+
+def make_fusion_weights(seed: int = 5000, width: int = 1280, llm_width: int = 2688, n_slots: int = 8,
+                        std: float = 0.02, gain_std: float = 0.02) -> dict:
+    """Speaker LayerNorm (gain 1 + N(0, 0.02), bias N(0, 0.02)) and the connector
+    (N(0, 0.02) weights and bias), bf16-rounded: {name: (bits, float32)}."""
+    out = {}
+    for i, (name, shape, kind) in enumerate([("spk_g", (n_slots,), "gain"), ("spk_b", (n_slots,), "normal"),
+                                              ("w_conn", (llm_width, width), "normal"),
+                                              ("b_conn", (llm_width,), "normal")]):
+        b = bf16_bits(_draw(shape, kind, seed + i, std, gain_std))
+        out[name] = (b, bf16_to_f32(b))
+    return out
