@@ -255,7 +255,7 @@ __global__ void __launch_bounds__(192, 1)
 #pragma unroll
       for (int c = 0; c < 4; ++c)
 #pragma unroll
-        for (int i = 0; i < 32; ++i) mx = fmaxf(mx, __uint_as_float(r[c][i]));
+        for (int i = 0; i < 32; i += 2) mx = max3f(mx, __uint_as_float(r[c][i]), __uint_as_float(r[c][i + 1]));
       mx *= sl2;
       float alpha = 1.f;
       bool rescale = false;
@@ -268,17 +268,23 @@ __global__ void __launch_bounds__(192, 1)
       }
       // a row that has seen no key yet keeps m_ref = -inf; its masked scores still give 0
       const float m_use = m_ref == -INFINITY ? 0.f : m_ref;
-      float sum = 0.f;
+      // two scores per instruction: x = s * scale - m (packed fma), the row sum (packed add)
+      const uint64_t sl2_2 = f2_pack(sl2, sl2), negm_2 = f2_pack(-m_use, -m_use);
+      uint64_t sum2 = f2_pack(0.f, 0.f);
       uint32_t p[2][32];
 #pragma unroll
       for (int c = 0; c < 4; ++c)
 #pragma unroll
         for (int i = 0; i < 32; i += 2) {
-          const float e0 = fast_exp2(fmaf(__uint_as_float(r[c][i]), sl2, -m_use));
-          const float e1 = fast_exp2(fmaf(__uint_as_float(r[c][i + 1]), sl2, -m_use));
-          sum += e0 + e1;
+          float x0, x1;
+          f2_unpack(f2_fma(f2_pack(__uint_as_float(r[c][i]), __uint_as_float(r[c][i + 1])), sl2_2, negm_2), x0, x1);
+          const float e0 = fast_exp2(x0), e1 = fast_exp2(x1);
+          sum2 = f2_add(sum2, f2_pack(e0, e1));
           p[c >> 1][(c & 1) * 16 + (i >> 1)] = pack_bf16x2(e0, e1);
         }
+      float sum_lo, sum_hi;
+      f2_unpack(sum2, sum_lo, sum_hi);
+      const float sum = sum_lo + sum_hi;
       if (j > 0) {
         // PV_{j-1} must be complete before O is rescaled or P buffer s is overwritten
         if (!mbar_wait_warp(o_done, (j - 1) & 1, guard)) {
@@ -540,7 +546,7 @@ __global__ void __launch_bounds__(320, 1)
           tmem_ld32(tmem + lane_base + colS + 32 * c + 32, rb);
           tmem_wait_ld();
 #pragma unroll
-          for (int i = 0; i < 32; ++i) mx = fmaxf(mx, fmaxf(__uint_as_float(ra[i]), __uint_as_float(rb[i])));
+          for (int i = 0; i < 32; ++i) mx = max3f(mx, __uint_as_float(ra[i]), __uint_as_float(rb[i]));
         }
       } else {
 #pragma unroll 1
@@ -577,7 +583,8 @@ __global__ void __launch_bounds__(320, 1)
       }
       // pass 2: exponentials, row sum, bf16 P over the first 64 columns of S
       const float m_use = m_ref == -INFINITY ? 0.f : m_ref;  // a row with no key seen yet
-      float sum = 0.f;
+      const uint64_t sl2_2 = f2_pack(sl2, sl2), negm_2 = f2_pack(-m_use, -m_use);
+      uint64_t sum2 = f2_pack(0.f, 0.f);
       if (!masked) {
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
@@ -587,9 +594,10 @@ __global__ void __launch_bounds__(320, 1)
           uint32_t p[16];
 #pragma unroll
           for (int i = 0; i < 32; i += 2) {
-            const float e0 = fast_exp2(fmaf(__uint_as_float(r[i]), sl2, -m_use));
-            const float e1 = fast_exp2(fmaf(__uint_as_float(r[i + 1]), sl2, -m_use));
-            sum += e0 + e1;
+            float x0, x1;
+            f2_unpack(f2_fma(f2_pack(__uint_as_float(r[i]), __uint_as_float(r[i + 1])), sl2_2, negm_2), x0, x1);
+            const float e0 = fast_exp2(x0), e1 = fast_exp2(x1);
+            sum2 = f2_add(sum2, f2_pack(e0, e1));
             p[i >> 1] = pack_bf16x2(e0, e1);
           }
           tmem_st16(tmem + lane_base + colS + 16 * c, p);
@@ -604,15 +612,18 @@ __global__ void __launch_bounds__(320, 1)
           uint32_t p[16];
 #pragma unroll
           for (int i = 0; i < 32; i += 2) {
-            const float e0 = fast_exp2(fmaf(__uint_as_float(r[i]), sl2, -m_use));
-            const float e1 = fast_exp2(fmaf(__uint_as_float(r[i + 1]), sl2, -m_use));
-            sum += e0 + e1;
+            float x0, x1;
+            f2_unpack(f2_fma(f2_pack(__uint_as_float(r[i]), __uint_as_float(r[i + 1])), sl2_2, negm_2), x0, x1);
+            const float e0 = fast_exp2(x0), e1 = fast_exp2(x1);
+            sum2 = f2_add(sum2, f2_pack(e0, e1));
             p[i >> 1] = pack_bf16x2(e0, e1);
           }
           tmem_st16(tmem + lane_base + colS + 16 * c, p);
         }
       }
-      l = l * alpha + sum;
+      float sum_lo, sum_hi;
+      f2_unpack(sum2, sum_lo, sum_hi);
+      l = l * alpha + (sum_lo + sum_hi);
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(&p_full[wg]);
