@@ -355,16 +355,21 @@ __global__ void __launch_bounds__(192, 1)
 //   warp 0: TMA loads (Q0 and Q1 once; K_j and V_j through two-stage rings released
 //           separately: K after both S products, V after both P V products)
 //   warp 1: tcgen05.mma issue, in the order S0_0 S1_0 | PV0_j S0_{j+1} PV1_j S1_{j+1} ...
-//   warps 2-5 / 6-9: softmax of query tile 0 / 1, one row per thread
+//   warps 2-3: idle (they complete warpgroup 0, which gives registers away)
+//   warps 4-7 / 8-11: softmax of query tile 0 / 1, one row per thread
 // TMEM: S0 [0,128) S1 [128,256) O0 [256,384) O1 [384,512); P_i (bf16 pairs) overwrites
 // the first 64 columns of S_i once the row has been read. Because tcgen05.mma operations
 // of one thread complete in issue order, S_i(j) completing implies P_i(j-1) V_{j-1} has
 // completed, so the softmax may rescale O_i as soon as S_i(j) is ready.
-// The softmax makes two passes over S in TMEM (row maximum, then exponentials), which
-// keeps register use low enough for ten warps.
+// Warpgroup 0 (loads, MMA issue) shrinks to kRegsCtrl registers per thread and the two
+// softmax warpgroups grow to kRegsSoftmax, so each softmax thread holds its whole row of
+// S (128 scores) and reads it from TMEM in one round trip per tile.
 constexpr size_t kSmemPP = 1024 + 6 * kTileBytes + 256;
+constexpr int kThreadsPP = 384;
+constexpr int kRegsCtrl = 80, kRegsSoftmax = 208;
+constexpr int kRegsNeededPP = kRegsCtrl * 128 + kRegsSoftmax * 256;  // <= launch regs x 384
 
-__global__ void __launch_bounds__(320, 1)
+__global__ void __launch_bounds__(kThreadsPP, 1)
     attention_pp_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                         const __grid_constant__ CUtensorMap tmV, const AttnArgs args) {
   extern __shared__ unsigned char smem_raw[];
@@ -425,98 +430,103 @@ __global__ void __launch_bounds__(320, 1)
   pdl_trigger();
   const uint32_t tmem = *tmem_slot;
   const WaitGuard guard{abort_flag, args.limit_ns, args.status};
-
-  if (warp == 0) {
-    if (lane == 0) {
-      uint32_t issued_k = 0, issued_v = 0, par_k = 0, par_v = 0;
-      mbar_arrive_expect_tx(q_full, 2 * kTileBytes);
-      for (int i = 0; i < 2; ++i) {
-        tma_load_3d(sQ + i * kTileBytes, &tmQ, q_full, 0, (2 * qt2 + i) * kTile, bh);
-        tma_load_3d(sQ + i * kTileBytes + kBox, &tmQ, q_full, 64, (2 * qt2 + i) * kTile, bh);
-      }
-      for (int j = 0; j < n_kv; ++j) {
-        const int s = j & 1;
-        const uint32_t use_par = (j >> 1) & 1;
-        if (!mbar_wait(&k_empty[s], use_par ^ 1, guard)) break;
-        mbar_arrive_expect_tx(&k_full[s], kTileBytes);
-        tma_load_3d(sK + s * kTileBytes, &tmK, &k_full[s], 0, (j0 + j) * kTile, bh);
-        tma_load_3d(sK + s * kTileBytes + kBox, &tmK, &k_full[s], 64, (j0 + j) * kTile, bh);
-        issued_k |= 1u << s;
-        par_k = (par_k & ~(1u << s)) | (use_par << s);
-        if (!mbar_wait(&v_empty[s], use_par ^ 1, guard)) break;
-        mbar_arrive_expect_tx(&v_full[s], kTileBytes);
-        tma_load_3d(sV + s * kTileBytes, &tmV, &v_full[s], 0, (j0 + j) * kTile, bh);
-        tma_load_3d(sV + s * kTileBytes + kBox, &tmV, &v_full[s], 64, (j0 + j) * kTile, bh);
-        issued_v |= 1u << s;
-        par_v = (par_v & ~(1u << s)) | (use_par << s);
-      }
-      if (*abort_flag) {
-        drain_wait(q_full, 0, args.limit_ns);
-        for (int s = 0; s < 2; ++s) {
-          if (issued_k & (1u << s)) drain_wait(&k_full[s], (par_k >> s) & 1, args.limit_ns);
-          if (issued_v & (1u << s)) drain_wait(&v_full[s], (par_v >> s) & 1, args.limit_ns);
+  // Each role runs inside the branch that set its register limit, so the compiler
+  // allocates it against that limit.
+  if (warp < 4) {
+    setmaxnreg_dec<kRegsCtrl>();
+    if (warp == 0) {
+      if (lane == 0) {
+        uint32_t issued_k = 0, issued_v = 0, par_k = 0, par_v = 0;
+        mbar_arrive_expect_tx(q_full, 2 * kTileBytes);
+        for (int i = 0; i < 2; ++i) {
+          tma_load_3d(sQ + i * kTileBytes, &tmQ, q_full, 0, (2 * qt2 + i) * kTile, bh);
+          tma_load_3d(sQ + i * kTileBytes + kBox, &tmQ, q_full, 64, (2 * qt2 + i) * kTile, bh);
+        }
+        for (int j = 0; j < n_kv; ++j) {
+          const int s = j & 1;
+          const uint32_t use_par = (j >> 1) & 1;
+          if (!mbar_wait(&k_empty[s], use_par ^ 1, guard)) break;
+          mbar_arrive_expect_tx(&k_full[s], kTileBytes);
+          tma_load_3d(sK + s * kTileBytes, &tmK, &k_full[s], 0, (j0 + j) * kTile, bh);
+          tma_load_3d(sK + s * kTileBytes + kBox, &tmK, &k_full[s], 64, (j0 + j) * kTile, bh);
+          issued_k |= 1u << s;
+          par_k = (par_k & ~(1u << s)) | (use_par << s);
+          if (!mbar_wait(&v_empty[s], use_par ^ 1, guard)) break;
+          mbar_arrive_expect_tx(&v_full[s], kTileBytes);
+          tma_load_3d(sV + s * kTileBytes, &tmV, &v_full[s], 0, (j0 + j) * kTile, bh);
+          tma_load_3d(sV + s * kTileBytes + kBox, &tmV, &v_full[s], 64, (j0 + j) * kTile, bh);
+          issued_v |= 1u << s;
+          par_v = (par_v & ~(1u << s)) | (use_par << s);
+        }
+        if (*abort_flag) {
+          drain_wait(q_full, 0, args.limit_ns);
+          for (int s = 0; s < 2; ++s) {
+            if (issued_k & (1u << s)) drain_wait(&k_full[s], (par_k >> s) & 1, args.limit_ns);
+            if (issued_v & (1u << s)) drain_wait(&v_full[s], (par_v >> s) & 1, args.limit_ns);
+          }
         }
       }
-    }
-  } else if (warp == 1) {
-    if (lane == 0) {
-      constexpr uint32_t IDESC_S = idesc_bf16(128, 128, false, false);
-      constexpr uint32_t IDESC_O = idesc_bf16(128, 128, false, true);
-      bool any_mma = false;
-      auto issue_s = [&](int i, int j) -> bool {  // S_i = Q_i K_j^T
-        const int s = j & 1;
-        if (!mbar_wait(&k_full[s], (j >> 1) & 1, guard)) return false;
-        tc_fence_after();
-        const uint32_t q0 = smem_u32(sQ + i * kTileBytes), k0 = smem_u32(sK + s * kTileBytes);
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint32_t off = (kk >> 2) * kBox + (kk & 3) * 32;
-          umma_ss(tmem + 128 * i, sdesc_kmajor_sw128(q0 + off), sdesc_kmajor_sw128(k0 + off), IDESC_S, kk > 0);
+    } else if (warp == 1) {
+      if (lane == 0) {
+        constexpr uint32_t IDESC_S = idesc_bf16(128, 128, false, false);
+        constexpr uint32_t IDESC_O = idesc_bf16(128, 128, false, true);
+        bool any_mma = false;
+        auto issue_s = [&](int i, int j) -> bool {  // S_i = Q_i K_j^T
+          const int s = j & 1;
+          if (!mbar_wait(&k_full[s], (j >> 1) & 1, guard)) return false;
+          tc_fence_after();
+          const uint32_t q0 = smem_u32(sQ + i * kTileBytes), k0 = smem_u32(sK + s * kTileBytes);
+  #pragma unroll
+          for (int kk = 0; kk < 8; ++kk) {
+            const uint32_t off = (kk >> 2) * kBox + (kk & 3) * 32;
+            umma_ss(tmem + 128 * i, sdesc_kmajor_sw128(q0 + off), sdesc_kmajor_sw128(k0 + off), IDESC_S, kk > 0);
+          }
+          umma_commit(&s_full[i]);
+          if (i == 1) umma_commit(&k_empty[s]);  // both products with K_j issued
+          any_mma = true;
+          return true;
+        };
+        auto issue_pv = [&](int i, int j) -> bool {  // O_i += P_i V_j
+          const int s = j & 1;
+          if (!mbar_wait(&p_full[i], j & 1, guard)) return false;
+          if (!mbar_wait(&v_full[s], (j >> 1) & 1, guard)) return false;
+          tc_fence_after();
+          const uint32_t v0 = smem_u32(sV + s * kTileBytes);
+  #pragma unroll
+          for (int kk = 0; kk < 8; ++kk)
+            umma_ts(tmem + 256 + 128 * i, tmem + 128 * i + kk * 8, sdesc_mnmajor_sw128(v0 + kk * 2048, kBox), IDESC_O,
+                    (j > 0 || kk > 0));
+          if (i == 1) umma_commit(&v_empty[s]);
+          return true;
+        };
+        bool ok = mbar_wait(q_full, 0, guard) && issue_s(0, 0) && issue_s(1, 0);
+        for (int j = 0; ok && j < n_kv; ++j) {
+          ok = issue_pv(0, j);
+          if (!ok) break;
+          if (j + 1 < n_kv) {
+            ok = issue_s(0, j + 1);
+          } else {
+            umma_commit(&o_final[0]);
+          }
+          if (!ok) break;
+          ok = issue_pv(1, j);
+          if (!ok) break;
+          if (j + 1 < n_kv) {
+            ok = issue_s(1, j + 1);
+          } else {
+            umma_commit(&o_final[1]);
+          }
         }
-        umma_commit(&s_full[i]);
-        if (i == 1) umma_commit(&k_empty[s]);  // both products with K_j issued
-        any_mma = true;
-        return true;
-      };
-      auto issue_pv = [&](int i, int j) -> bool {  // O_i += P_i V_j
-        const int s = j & 1;
-        if (!mbar_wait(&p_full[i], j & 1, guard)) return false;
-        if (!mbar_wait(&v_full[s], (j >> 1) & 1, guard)) return false;
-        tc_fence_after();
-        const uint32_t v0 = smem_u32(sV + s * kTileBytes);
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          umma_ts(tmem + 256 + 128 * i, tmem + 128 * i + kk * 8, sdesc_mnmajor_sw128(v0 + kk * 2048, kBox), IDESC_O,
-                  (j > 0 || kk > 0));
-        if (i == 1) umma_commit(&v_empty[s]);
-        return true;
-      };
-      bool ok = mbar_wait(q_full, 0, guard) && issue_s(0, 0) && issue_s(1, 0);
-      for (int j = 0; ok && j < n_kv; ++j) {
-        ok = issue_pv(0, j);
-        if (!ok) break;
-        if (j + 1 < n_kv) {
-          ok = issue_s(0, j + 1);
-        } else {
-          umma_commit(&o_final[0]);
+        if (*abort_flag && any_mma) {
+          umma_commit(drain);
+          drain_wait(drain, 0, args.limit_ns);
         }
-        if (!ok) break;
-        ok = issue_pv(1, j);
-        if (!ok) break;
-        if (j + 1 < n_kv) {
-          ok = issue_s(1, j + 1);
-        } else {
-          umma_commit(&o_final[1]);
-        }
-      }
-      if (*abort_flag && any_mma) {
-        umma_commit(drain);
-        drain_wait(drain, 0, args.limit_ns);
       }
     }
   } else {
+    setmaxnreg_inc<kRegsSoftmax>();
     // ------------------------------------------------------------ softmax warpgroups
-    const int wg = (warp - 2) >> 2;  // query tile 0 or 1
+    const int wg = (warp - 4) >> 2;  // query tile 0 or 1
     const int quarter = warp & 3;
     const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
     const uint32_t colS = 128u * wg, colO = 256u + 128u * wg;
@@ -535,30 +545,20 @@ __global__ void __launch_bounds__(320, 1)
       int c_lo, c_hi;
       tile_cols(row_lo, row_hi, j0 + j, c_lo, c_hi);
       const bool masked = !__all_sync(0xffffffffu, c_lo == 0 && c_hi == kTile);
-      // pass 1: row maximum (tiles that need a mask take a compact separate loop, so the
-      // common unmasked body carries no mask code)
-      float mx = -INFINITY;
-      if (!masked) {
+      // the whole row of S in registers (one wait for four loads)
+      uint32_t r[4][32];
 #pragma unroll
-        for (int c = 0; c < 4; c += 2) {
-          uint32_t ra[32], rb[32];
-          tmem_ld32(tmem + lane_base + colS + 32 * c, ra);
-          tmem_ld32(tmem + lane_base + colS + 32 * c + 32, rb);
-          tmem_wait_ld();
+      for (int c = 0; c < 4; ++c) tmem_ld32(tmem + lane_base + colS + 32 * c, r[c]);
+      tmem_wait_ld();
+      if (masked) {
 #pragma unroll
-          for (int i = 0; i < 32; ++i) mx = max3f(mx, __uint_as_float(ra[i]), __uint_as_float(rb[i]));
-        }
-      } else {
-#pragma unroll 1
-        for (int c = 0; c < 4; ++c) {
-          uint32_t r[32];
-          tmem_ld32(tmem + lane_base + colS + 32 * c, r);
-          tmem_wait_ld();
-          mask_chunk(r, 32 * c, c_lo, c_hi);
-#pragma unroll
-          for (int i = 0; i < 32; ++i) mx = fmaxf(mx, __uint_as_float(r[i]));
-        }
+        for (int c = 0; c < 4; ++c) mask_chunk(r[c], 32 * c, c_lo, c_hi);
       }
+      float mx = -INFINITY;
+#pragma unroll
+      for (int c = 0; c < 4; ++c)
+#pragma unroll
+        for (int i = 0; i < 32; i += 2) mx = max3f(mx, __uint_as_float(r[c][i]), __uint_as_float(r[c][i + 1]));
       mx *= sl2;
       float alpha = 1.f;
       bool rescale = false;
@@ -569,7 +569,24 @@ __global__ void __launch_bounds__(320, 1)
         m_ref = mx;
         rescale = true;
       }
-      // O_i(j-1) is complete (it was issued before S_i(j)); rescale it if the max moved
+      // exponentials, row sum, bf16 P packed in place over the scores already consumed
+      const float m_use = m_ref == -INFINITY ? 0.f : m_ref;  // a row with no key seen yet
+      const uint64_t sl2_2 = f2_pack(sl2, sl2), negm_2 = f2_pack(-m_use, -m_use);
+      uint64_t sum2 = f2_pack(0.f, 0.f);
+#pragma unroll
+      for (int c = 0; c < 4; ++c)
+#pragma unroll
+        for (int i = 0; i < 32; i += 2) {
+          float x0, x1;
+          f2_unpack(f2_fma(f2_pack(__uint_as_float(r[c][i]), __uint_as_float(r[c][i + 1])), sl2_2, negm_2), x0, x1);
+          const float e0 = fast_exp2(x0), e1 = fast_exp2(x1);
+          sum2 = f2_add(sum2, f2_pack(e0, e1));
+          r[c >> 1][(c & 1) * 16 + (i >> 1)] = pack_bf16x2(e0, e1);
+        }
+      tmem_st32(tmem + lane_base + colS, r[0]);
+      tmem_st32(tmem + lane_base + colS + 32, r[1]);
+      // O_i(j-1) is complete (it was issued before S_i(j)); rescale it if the max moved.
+      // PV_i(j) is issued only after p_full below, so this precedes it.
       if (j > 0 && __any_sync(0xffffffffu, rescale)) {
 #pragma unroll 1
         for (int c = 0; c < 4; ++c) {
@@ -579,46 +596,6 @@ __global__ void __launch_bounds__(320, 1)
 #pragma unroll
           for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
           tmem_st32(tmem + lane_base + colO + 32 * c, o);
-        }
-      }
-      // pass 2: exponentials, row sum, bf16 P over the first 64 columns of S
-      const float m_use = m_ref == -INFINITY ? 0.f : m_ref;  // a row with no key seen yet
-      const uint64_t sl2_2 = f2_pack(sl2, sl2), negm_2 = f2_pack(-m_use, -m_use);
-      uint64_t sum2 = f2_pack(0.f, 0.f);
-      if (!masked) {
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          uint32_t r[32];
-          tmem_ld32(tmem + lane_base + colS + 32 * c, r);
-          tmem_wait_ld();
-          uint32_t p[16];
-#pragma unroll
-          for (int i = 0; i < 32; i += 2) {
-            float x0, x1;
-            f2_unpack(f2_fma(f2_pack(__uint_as_float(r[i]), __uint_as_float(r[i + 1])), sl2_2, negm_2), x0, x1);
-            const float e0 = fast_exp2(x0), e1 = fast_exp2(x1);
-            sum2 = f2_add(sum2, f2_pack(e0, e1));
-            p[i >> 1] = pack_bf16x2(e0, e1);
-          }
-          tmem_st16(tmem + lane_base + colS + 16 * c, p);
-        }
-      } else {
-#pragma unroll 1
-        for (int c = 0; c < 4; ++c) {
-          uint32_t r[32];
-          tmem_ld32(tmem + lane_base + colS + 32 * c, r);
-          tmem_wait_ld();
-          mask_chunk(r, 32 * c, c_lo, c_hi);
-          uint32_t p[16];
-#pragma unroll
-          for (int i = 0; i < 32; i += 2) {
-            float x0, x1;
-            f2_unpack(f2_fma(f2_pack(__uint_as_float(r[i]), __uint_as_float(r[i + 1])), sl2_2, negm_2), x0, x1);
-            const float e0 = fast_exp2(x0), e1 = fast_exp2(x1);
-            sum2 = f2_add(sum2, f2_pack(e0, e1));
-            p[i >> 1] = pack_bf16x2(e0, e1);
-          }
-          tmem_st16(tmem + lane_base + colS + 16 * c, p);
         }
       }
       float sum_lo, sum_hi;
@@ -666,7 +643,7 @@ __global__ void __launch_bounds__(320, 1)
 
 std::mutex g_mu;
 bool g_attr[64] = {};
-bool g_attr_pp[64] = {};
+bool g_pp_ok[64] = {};  // the two-tile kernel's launch registers cover its warpgroup split
 
 }  // namespace
 
@@ -683,6 +660,11 @@ sal_status attention_launch(const void* q, const void* k, const void* v, int bat
           cudaFuncSetAttribute(attention_pp_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                static_cast<int>(kSmemPP)) != cudaSuccess)
         return SAL_ECUDA;
+      // setmaxnreg.inc waits until the registers it asks for are free: run the kernel only
+      // if what warpgroup 0 gives back covers what the softmax warpgroups take
+      cudaFuncAttributes fa{};
+      if (cudaFuncGetAttributes(&fa, attention_pp_kernel) != cudaSuccess) return SAL_ECUDA;
+      g_pp_ok[dev] = fa.numRegs * kThreadsPP >= kRegsNeededPP && fa.numRegs <= 168;
       g_attr[dev] = true;
     }
   }
@@ -708,9 +690,14 @@ sal_status attention_launch(const void* q, const void* k, const void* v, int bat
   const uint64_t ctas_1 = static_cast<uint64_t>((T + kTile - 1) / kTile) * bh;
   const double waves_pp = static_cast<double>((ctas_pp + sms - 1) / sms) * 1.6;
   const double waves_1 = static_cast<double>((ctas_1 + sms - 1) / sms);
-  if (ctas_pp >= 120 && waves_pp < waves_1 && attention_pp_enabled()) {
+  bool pp_ok = false;
+  {
+    std::lock_guard<std::mutex> lk(g_mu);
+    pp_ok = dev >= 0 && dev < 64 && g_pp_ok[dev];
+  }
+  if (pp_ok && ctas_pp >= 120 && waves_pp < waves_1 && attention_pp_enabled()) {
     const dim3 grid(static_cast<unsigned>((T + 2 * kTile - 1) / (2 * kTile)), static_cast<unsigned>(bh));
-    return launch_kernel(attention_pp_kernel, grid, dim3(320), kSmemPP, s, tq, tk, tv, a) == cudaSuccess
+    return launch_kernel(attention_pp_kernel, grid, dim3(kThreadsPP), kSmemPP, s, tq, tk, tv, a) == cudaSuccess
                ? SAL_OK
                : SAL_ECUDA;
   }
