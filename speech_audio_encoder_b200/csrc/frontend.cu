@@ -12,8 +12,7 @@
 //   1. the 400 windowed samples, zero-padded to 512, are packed as 256 complex values
 //      z[m] = y[2m] + i y[2m+1];
 //   2. a 256-point complex FFT factored 16 x 16: lane n2 transforms z[16 n1 + n2] over n1
-//      in registers and applies the twiddle W256^(n2 k1) (powers of W256^n2 formed in
-//      registers); one transposing exchange in
+//      in registers and applies the twiddle W256^(n2 k1); one transposing exchange in
 //      shared memory; lane k1 transforms over n2, giving Z[k1 + 16 k2] in its registers;
 //   3. the split step for the pair (k, 256 - k): with E = Z[k] + conj Z[256-k] and
 //      O = (Z[k] - conj Z[256-k]) / i, 2 X[k] = E + W512^k O and 2 X[256-k] =
@@ -66,7 +65,7 @@ static_assert(mel_table_consistent(), "mel group offsets");
 constexpr int kMelPadded = mel_base(8);  // 640
 
 struct FrontTables {
-  double2 tw256[16];       // [n2] = e^{-2 pi i n2 / 256}
+  double2 tw256[15 * 16];  // [k1 - 1][n2] = e^{-2 pi i n2 k1 / 256}
   double2 tw512[8 * 16];   // [k2][k1] = e^{-2 pi i k / 512}, k = k1 + 16 k2 < 128
   double hann[kWin];
   float mel_w[kMelPadded];  // [group h][tap j][lane]: weights / 4 of filter 16 h + lane at bin mel_k0 + j
@@ -109,12 +108,26 @@ __device__ __forceinline__ void dft4(C2 a, C2 b, C2 c, C2 d, C2& y0, C2& y1, C2&
 
 // X[k] = sum_n x[n] e^{-2 pi i n k / 16}, in place: n = 4a + b, k = c + 4d; a 4-point
 // transform over a for each b, the twiddle e^{-2 pi i b c / 16}, a 4-point transform over b.
+// kTailZero: x[13] = x[14] = x[15] = 0 (the zero padding in pass 1, where the 400 samples
+// fill z[0..199] of the 256 packed values), so three of the first 4-point transforms have
+// a zero last input and skip two complex additions each.
+template <bool kTailZero>
 __device__ __forceinline__ void dft16(C2 (&v)[16]) {
   const double c1 = 0.92387953251128675613, s1 = 0.38268343236508977173;  // cos, sin of pi/8
   const double r = 0.70710678118654752440;
   C2 y[4][4];
 #pragma unroll
-  for (int b = 0; b < 4; ++b) dft4(v[b], v[4 + b], v[8 + b], v[12 + b], y[b][0], y[b][1], y[b][2], y[b][3]);
+  for (int b = 0; b < 4; ++b) {
+    if (kTailZero && b > 0) {  // dft4(a, b, c, 0)
+      const C2 s0 = cadd(v[b], v[8 + b]), d0 = csub(v[b], v[8 + b]), m = v[4 + b];
+      y[b][0] = cadd(s0, m);
+      y[b][2] = csub(s0, m);
+      y[b][1] = cadd(d0, mul_neg_i(m));
+      y[b][3] = cadd(d0, mul_pos_i(m));
+    } else {
+      dft4(v[b], v[4 + b], v[8 + b], v[12 + b], y[b][0], y[b][1], y[b][2], y[b][3]);
+    }
+  }
   // twiddles W16^(b c)
   y[1][1] = cmul(y[1][1], make_double2(c1, -s1));                        // W^1
   y[1][2] = {(y[1][2].x + y[1][2].y) * r, (y[1][2].y - y[1][2].x) * r};  // W^2
@@ -224,19 +237,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         v[n1] = {0.0, 0.0};
       }
     }
-    dft16(v);
-    {
-      // twiddles W256^(n2 k1) by a running product from W256^n2 (fp64: 14 products add
-      // a few 1e-16); the table is read once per frame instead of 15 times
-      scr[hl * 17] = make_double2(v[0].x, v[0].y);
-      const double2 w1 = tab.tw256[hl];
-      double2 w = w1;
+    dft16<true>(v);
 #pragma unroll
-      for (int k1 = 1; k1 < 16; ++k1) {
-        const C2 t = cmul(v[k1], w);
-        scr[hl * 17 + k1] = make_double2(t.x, t.y);
-        if (k1 < 15) w = make_double2(fma(w.x, w1.x, -w.y * w1.y), fma(w.x, w1.y, w.y * w1.x));
-      }
+    for (int k1 = 0; k1 < 16; ++k1) {
+      const C2 t = k1 ? cmul(v[k1], tab.tw256[(k1 - 1) * 16 + hl]) : v[0];
+      scr[hl * 17 + k1] = make_double2(t.x, t.y);
     }
     __syncwarp();
 
@@ -246,7 +251,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const double2 a = scr[n2 * 17 + hl];
       v[n2] = {a.x, a.y};
     }
-    dft16(v);
+    dft16<false>(v);
     __syncwarp();  // the scratch now takes the powers
 
     // ---- split and power. Lane k1 owns the pairs (k, 256 - k), k = k1 + 16 k2, k2 < 8;
@@ -319,7 +324,11 @@ double mel_to_hz_slaney(double m) {
 
 bool build_tables(FrontTables* t) {
   const double pi = 3.14159265358979323846;
-  for (int n2 = 0; n2 < 16; ++n2) t->tw256[n2] = make_double2(std::cos(2 * pi * n2 / 256.0), -std::sin(2 * pi * n2 / 256.0));
+  for (int k1 = 1; k1 < 16; ++k1)
+    for (int n2 = 0; n2 < 16; ++n2) {
+      const double a = 2 * pi * n2 * k1 / 256.0;
+      t->tw256[(k1 - 1) * 16 + n2] = make_double2(std::cos(a), -std::sin(a));
+    }
   for (int k = 0; k < 128; ++k) t->tw512[k] = make_double2(std::cos(2 * pi * k / 512.0), -std::sin(2 * pi * k / 512.0));
   for (int n = 0; n < kWin; ++n) t->hann[n] = 0.5 - 0.5 * std::cos(2 * pi * n / 400.0);
   // Slaney filters: 130 points equally spaced in mel over 0..8000 Hz.
