@@ -30,6 +30,11 @@ Audits", flozi.net):
 * [CHUNK] section "Local encoder windows, recording-wide language context": in training the
   encoder runs on independent 30-second post-feature chunks with no attention across
   their borders, and the chunk outputs are concatenated in order; pairs scale as T w.
+* [CTC]   section "Use alignment and audio questions as supporting evidence": a CTC
+  timestamp adapter of about 50M parameters takes the unfused ASR states (width 1,280),
+  upsamples their 80 ms grid to 40 ms with a stride-two transposed convolution, runs two
+  Transformer layers with 16 heads, and projects to a 23,862-token vocabulary plus the
+  CTC blank. Widths and kernel size are not given; readings 17-21 below.
 
 Readings where the pages are silent (each one is listed in the design notes):
 
@@ -56,6 +61,18 @@ Readings where the pages are silent (each one is listed in the design notes):
 15. the speaker kernel is the sinusoidal table K[s, 2i] = sin(s w_i), K[s, 2i+1] = cos(s w_i),
     w_i = 10000^(-2i/1280), s = 0..7; fused = H + 1 * LN(indicators) K.
 16. the connector is x W^T + b with W [2688, 1280].
+17. the adapter's transposed convolution has kernel size 2 (equal to its stride), so each
+    80 ms state gives two 40 ms states with no overlap: U[2t + j] = h[t] W_j^T + b,
+    j in {0, 1}, one bias per output channel.
+18. the adapter width is 1,024 (16 heads of 64): with the encoder's layer recipe and an
+    FFN of 4,096, it is the width that gives about 50M parameters (52.3M; 768 gives 35M,
+    1,280 gives 73M).
+19. the adapter layers follow the encoder's recipe (readings 8-12) at that width; RoPE
+    positions count 40 ms steps from the clip start.
+20. a final LayerNorm precedes the projection (as after the encoder); the projection has a
+    bias and 23,863 outputs, the blank last.
+21. the adapter's output is the frame log-probabilities, log_softmax over the 23,863
+    classes.
 """
 from __future__ import annotations
 
@@ -92,7 +109,8 @@ __all__ = [
     "encoder_layer_rows", "encoder_forward", "stack_project", "encode",
     "param_count", "rel_l2", "chunk_bounds", "encoder_layer_chunked",
     "encoder_layer_rows_chunked", "encoder_forward_chunked", "N_SLOTS", "LLM_WIDTH",
-    "speaker_kernel", "speaker_fuse", "connector",
+    "speaker_kernel", "speaker_fuse", "connector", "CtcDims", "CTC", "ctc_upsample",
+    "log_softmax", "ctc_logits", "ctc_adapter", "ctc_param_count",
 ]
 
 
@@ -387,6 +405,67 @@ def speaker_fuse(H, P, g, b, scale: float = 1.0):
 def connector(x, w, b):
     """The identity connector: one linear projection to the language width ([FUSE], 16)."""
     return linear(x, w, b)
+
+# ----------------------------------------------------------------------------- CTC timestamp adapter
+
+@dataclass(frozen=True)
+class CtcDims:
+    """Shape of the CTC timestamp adapter ([CTC], readings 17-21)."""
+    in_width: int = 1280   # the unfused ASR states [CTC]
+    width: int = 1024      # reading 18
+    heads: int = 16        # [CTC]
+    head_dim: int = 64
+    ffn: int = 4096        # expansion four, as in the encoder (reading 19)
+    layers: int = 2        # [CTC]
+    classes: int = 23863   # 23,862 tokens + the CTC blank [CTC]
+
+    @property
+    def layer_dims(self) -> EncoderDims:
+        return EncoderDims(width=self.width, heads=self.heads, head_dim=self.head_dim, ffn=self.ffn)
+
+
+CTC = CtcDims()
+
+
+def ctc_upsample(h, w_up, b_up):
+    """Stride-two transposed convolution with kernel 2 ([CTC], reading 17): the state of
+    position t gives the states 2t and 2t + 1, U[2t + j] = h[t] W_j^T + b, with
+    w_up [2, width, in_width] holding W_0 and W_1 and b_up [width]."""
+    h, w = _f64(h), _f64(w_up)
+    U = np.empty((2 * h.shape[0], w.shape[1]), dtype=np.float64)
+    for j in range(2):
+        U[j::2] = h @ w[j].T + _f64(b_up)
+    return U
+
+
+def log_softmax(z):
+    """log(softmax(z)) over the last axis, with the row maximum subtracted (reading 21)."""
+    z = _f64(z)
+    m = z.max(axis=-1, keepdims=True)
+    return z - m - np.log(np.exp(z - m).sum(axis=-1, keepdims=True))
+
+
+def ctc_logits(h, cw, dims: CtcDims = CTC):
+    """Class scores [2T, classes] of the adapter on one clip's unfused states h [T, in_width]:
+    upsampling, the Transformer layers, the final LayerNorm and the projection."""
+    x = ctc_upsample(h, cw["w_up"], cw["b_up"])
+    for lw in cw["layers"][:dims.layers]:
+        x = encoder_layer(x, lw, dims.layer_dims)
+    return linear(layer_norm(x, cw["lnf_g"], cw["lnf_b"]), cw["w_out"], cw["b_out"])
+
+
+def ctc_adapter(h, cw, dims: CtcDims = CTC):
+    """Frame log-probabilities [2T, classes] on the 40 ms grid ([CTC], reading 21)."""
+    return log_softmax(ctc_logits(h, cw, dims))
+
+
+def ctc_param_count(dims: CtcDims = CTC) -> int:
+    """Parameters of the adapter: transposed convolution, layers, final LN, projection."""
+    W = dims.width
+    up = 2 * W * dims.in_width + W
+    layers = param_count(dims.layers, dims.layer_dims) - (dims.layer_dims.stack_in * W + W + 2 * W)
+    return up + layers + 2 * W + dims.classes * W + dims.classes
+
 
 
 def stack_project(stacked, weights):

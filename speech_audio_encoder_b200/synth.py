@@ -220,3 +220,35 @@ def make_fusion_weights(seed: int = 5000, width: int = 1280, llm_width: int = 26
         b = bf16_bits(_draw(shape, kind, seed + i, std, gain_std))
         out[name] = (b, bf16_to_f32(b))
     return out
+
+
+# ----------------------------------------------------------------------------- CTC adapter weights
+
+def make_ctc_weights(seed: int = 7000, in_width: int = 1280, width: int = 1024, ffn: int = 4096,
+                     head_dim: int = 64, n_layers: int = 2, classes: int = 23863, std: float = 0.02,
+                     gain_std: float = 0.02) -> dict:
+    """Random-init weights of the CTC timestamp adapter, bf16-rounded, as {name: (bits, f32)}
+    with "layers" a list of per-layer dicts (the encoder's layer tensors at this width).
+    w_up [2, width, in_width] holds the two taps of the transposed convolution; w_out
+    [classes, width]. Tensor i of the flat order uses seed + i."""
+    out: dict = {"layers": []}
+    idx = 0
+
+    def put(d, name, shape, kind):
+        nonlocal idx
+        b = bf16_bits(_draw(shape, kind, seed + idx, std, gain_std))
+        d[name] = (b, bf16_to_f32(b))
+        idx += 1
+
+    put(out, "w_up", (2, width, in_width), "normal")
+    put(out, "b_up", (width,), "normal")
+    for _ in range(n_layers):
+        lw: dict = {}
+        for name, shp, kind in LAYER_TENSORS:
+            put(lw, name, shp(width, ffn, head_dim), kind)
+        out["layers"].append(lw)
+    put(out, "lnf_g", (width,), "gain")
+    put(out, "lnf_b", (width,), "normal")
+    put(out, "w_out", (classes, width), "normal")
+    put(out, "b_out", (classes,), "normal")
+    return out
