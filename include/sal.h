@@ -264,6 +264,62 @@ sal_status sal_connector(const void* x, int64_t rows, const void* W, const void*
 sal_status sal_qkv_rope_noalloc(const void* h, int batch, int64_t T, const sal_layer* layer,
                                 void* q, void* k, void* v, void* stream);
 
+/* ---------------------------------------------------------------------------------
+ * CTC timestamp adapter (page "Nemotron 3.5 Transcribe: From Recorded Speech to Dataset
+ * Audits", section "Use alignment and audio questions as supporting evidence"): about 50M
+ * parameters on the unfused ASR states (width 1,280); a stride-two transposed
+ * convolution from the 80 ms to a 40 ms grid, two Transformer layers with 16 heads, and a
+ * projection to a 23,862-token vocabulary plus the CTC blank. The page gives no widths.
+ * This library reads the adapter as:
+ *   - width 1,024 (16 heads of 64, FFN 4,096): the width that gives about 50M parameters
+ *     with the encoder's layer recipe (pre-norm LN, RMS QK-norm, RoPE over 40 ms steps,
+ *     exact-erf GELU);
+ *   - a transposed-convolution kernel of 2 (each 80 ms state gives two 40 ms states);
+ *   - a final LayerNorm before the projection;
+ *   - log-softmax over the 23,863 classes (blank last) as the output.
+ * --------------------------------------------------------------------------------- */
+
+#define SAL_CTC_WIDTH 1024
+#define SAL_CTC_HEADS 16
+#define SAL_CTC_HEAD_DIM 64
+#define SAL_CTC_FFN 4096
+#define SAL_CTC_LAYERS 2
+#define SAL_CTC_CLASSES 23863
+
+/* Device pointers, bf16, 16-byte aligned (the layer array itself is host memory). */
+typedef struct {
+  const void* w_up;         /* [2 * 1024, 1280]: row 1024 j + c is tap j of output channel c */
+  const void* b_up;         /* [1024], shared by both taps */
+  const sal_layer* layers;  /* n_layers layers at width 1024: ln* [1024], w_qkv [3072, 1024], b_qkv [3072],
+                               qn_g / kn_g [64], w_o [1024, 1024], w1 [4096, 1024], b1 [4096],
+                               w2 [1024, 4096], other biases [1024] */
+  int n_layers;             /* SAL_CTC_LAYERS */
+  const void *lnf_g, *lnf_b;  /* [1024] */
+  const void *w_out, *b_out;  /* [23863, 1024], [23863] */
+} sal_ctc_weights;
+
+/* Workspace bytes for sal_ctc_adapter over batch clips of T encoder positions (0 when
+ * either is <= 0). About 110 KB per 40 ms position, most of it the fp32 class scores. */
+size_t sal_ctc_workspace_bytes(int batch, int64_t T);
+
+/* Frame log-probabilities of the adapter. h: [batch * T, 1280] bf16, the unfused encoder
+ * states (sal_encoder_forward's output); logp: [batch * 2T, 23863] float32, row
+ * 2 T b + u holding 40 ms position u of clip b. workspace: >= sal_ctc_workspace_bytes,
+ * 256-byte aligned, owned by the caller. Errors: SAL_EINVAL (null or misaligned pointer,
+ * n_layers out of range), SAL_ESHAPE (T > 45,000 or batch > 4095), SAL_EWORKSPACE. */
+sal_status sal_ctc_adapter(const void* h, int batch, int64_t T, const sal_ctc_weights* w, float* logp,
+                           void* workspace, size_t ws_bytes, void* stream);
+
+/* Attention for heads of width 64 or 128 (the encoder: 10 x 128; the CTC adapter:
+ * 16 x 64): q, k, v [batch, heads, T, head_dim] bf16; o [batch, T, heads * head_dim] bf16.
+ * SAL_ESHAPE for another head width, T > 90,000 or batch * heads > 65535. */
+sal_status sal_attention_heads(const void* q, const void* k, const void* v, int batch, int64_t T, int heads,
+                               int head_dim, void* o, void* stream);
+
+/* Row log-softmax (the adapter's last step): out[r, i] = z[r, i] - log sum_j exp z[r, j]
+ * for i < n. z rows are ld floats apart (ld >= n), out rows n floats apart; float32. */
+sal_status sal_log_softmax(const float* z, int64_t rows, int n, int64_t ld, float* out, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

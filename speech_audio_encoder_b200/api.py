@@ -41,6 +41,13 @@ class sal_weights(ctypes.Structure):
                 ("lnf_g", ctypes.c_void_p), ("lnf_b", ctypes.c_void_p)]
 
 
+class sal_ctc_weights(ctypes.Structure):
+    _fields_ = [("w_up", ctypes.c_void_p), ("b_up", ctypes.c_void_p),
+                ("layers", ctypes.POINTER(sal_layer)), ("n_layers", ctypes.c_int),
+                ("lnf_g", ctypes.c_void_p), ("lnf_b", ctypes.c_void_p),
+                ("w_out", ctypes.c_void_p), ("b_out", ctypes.c_void_p)]
+
+
 class sal_trace(ctypes.Structure):
     _fields_ = [("kind", ctypes.c_int), ("events", ctypes.POINTER(ctypes.c_void_p)),
                 ("n_events", ctypes.c_int)]
@@ -94,6 +101,15 @@ EXPORTS = {
                                       ctypes.c_int64, ctypes.c_void_p, ctypes.c_void_p]),
     "sal_attention_chunked": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int,
                                               ctypes.c_int64, ctypes.c_int64, ctypes.c_void_p, ctypes.c_void_p]),
+    "sal_attention_heads": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int,
+                                            ctypes.c_int64, ctypes.c_int, ctypes.c_int, ctypes.c_void_p,
+                                            ctypes.c_void_p]),
+    "sal_log_softmax": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_int64,
+                                        ctypes.c_void_p, ctypes.c_void_p]),
+    "sal_ctc_workspace_bytes": (ctypes.c_size_t, [ctypes.c_int, ctypes.c_int64]),
+    "sal_ctc_adapter": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int, ctypes.c_int64,
+                                        ctypes.POINTER(sal_ctc_weights), ctypes.c_void_p, ctypes.c_void_p,
+                                        ctypes.c_size_t, ctypes.c_void_p]),
 }
 
 _lib = None
@@ -198,6 +214,45 @@ class DeviceWeights:
                           self.record.lnf_g, self.record.lnf_b)
         rec._keep = self  # keep the layer array alive
         return rec
+
+
+class DeviceCtcWeights:
+    """CTC adapter parameters in one device buffer, plus the sal_ctc_weights record.
+
+    ``w`` is the dict of (bf16 bits, float32) pairs from ``synth.make_ctc_weights``; w_up
+    [2, 1024, 1280] is laid out as the [2048, 1280] the library reads.
+    """
+
+    GLOBALS = ("w_up", "b_up", "lnf_g", "lnf_b", "w_out", "b_out")
+
+    def __init__(self, w: dict, device="cuda"):
+        names, arrays = [], []
+        for k in self.GLOBALS:
+            names.append((None, k))
+            arrays.append(w[k][0])
+        for i, lw in enumerate(w["layers"]):
+            for k in LAYER_FIELDS:
+                names.append((i, k))
+                arrays.append(lw[k][0])
+        offsets, off = [], 0
+        for a in arrays:
+            offsets.append(off)
+            off += (a.size + 127) // 128 * 128
+        host = np.zeros(off, dtype=np.uint16)
+        for a, o in zip(arrays, offsets):
+            host[o:o + a.size] = a.reshape(-1)
+        self.buffer = torch.from_numpy(host.view(np.int16)).to(device).view(torch.bfloat16)
+        base = self.buffer.data_ptr()
+        self.n_layers = len(w["layers"])
+        self._layers = (sal_layer * max(self.n_layers, 1))()
+        ptr = {}
+        for (i, k), o in zip(names, offsets):
+            ptr[(i, k)] = base + 2 * o
+            if i is not None:
+                setattr(self._layers[i], k, base + 2 * o)
+        g = {k: ptr[(None, k)] for k in self.GLOBALS}
+        self.record = sal_ctc_weights(g["w_up"], g["b_up"], self._layers, self.n_layers, g["lnf_g"], g["lnf_b"],
+                                      g["w_out"], g["b_out"])
 
 
 # ----------------------------------------------------------------------------- calls
@@ -364,3 +419,43 @@ def sal_last_device_status(stream=None) -> int:
 
 def sal_set_wait_limit_ns(ns: int) -> None:
     lib().sal_set_wait_limit_ns(int(ns))
+
+
+CTC_CLASSES = 23863
+
+
+def ctc_workspace(batch: int, T: int, device="cuda") -> torch.Tensor:
+    n = lib().sal_ctc_workspace_bytes(batch, T)
+    return torch.empty(max(n, 256), dtype=torch.uint8, device=device)
+
+
+def sal_ctc_adapter(h: torch.Tensor, batch: int, T: int, weights: DeviceCtcWeights,
+                    logp: torch.Tensor | None = None, workspace: torch.Tensor | None = None,
+                    stream=None) -> torch.Tensor:
+    """Unfused encoder states h [batch * T, 1280] bf16 -> log-probabilities
+    [batch * 2T, 23863] float32 on the 40 ms grid."""
+    if logp is None:
+        logp = torch.empty((batch * 2 * T, CTC_CLASSES), dtype=torch.float32, device=h.device)
+    if workspace is None:
+        workspace = ctc_workspace(batch, T, h.device)
+    _check("sal_ctc_adapter", lib().sal_ctc_adapter(_ptr(h), batch, T, ctypes.byref(weights.record), _ptr(logp),
+                                                    _ptr(workspace), workspace.numel(), _stream(stream)))
+    return logp
+
+
+def sal_attention_heads(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, stream=None) -> torch.Tensor:
+    """q, k, v [batch, heads, T, head_dim] bf16 (head_dim 64 or 128) -> o [batch, T, heads * head_dim]."""
+    B, H, T, hd = q.shape
+    o = torch.empty((B, T, H * hd), dtype=torch.bfloat16, device=q.device)
+    _check("sal_attention_heads", lib().sal_attention_heads(_ptr(q), _ptr(k), _ptr(v), B, T, H, hd, _ptr(o),
+                                                            _stream(stream)))
+    return o
+
+
+def sal_log_softmax(z: torch.Tensor, n: int | None = None, stream=None) -> torch.Tensor:
+    """Row log-softmax of the first n columns of z [rows, ld] float32 -> [rows, n]."""
+    rows, ld = z.shape
+    n = ld if n is None else n
+    out = torch.empty((rows, n), dtype=torch.float32, device=z.device)
+    _check("sal_log_softmax", lib().sal_log_softmax(_ptr(z), rows, n, ld, _ptr(out), _stream(stream)))
+    return out

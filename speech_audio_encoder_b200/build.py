@@ -19,7 +19,7 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libsal.so")
-SOURCES = ["sal_api.cu", "frontend.cu", "rowops.cu", "gemm.cu", "attention.cu", "noalloc.cu"]
+SOURCES = ["sal_api.cu", "frontend.cu", "rowops.cu", "gemm.cu", "attention.cu", "noalloc.cu", "ctc.cu"]
 HEADERS = ["sal_internal.h", "sal_ptx.cuh"]
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]

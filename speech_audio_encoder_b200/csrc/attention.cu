@@ -34,7 +34,8 @@ constexpr int kTileBytes = 2 * kBox;       // 32 KB
 constexpr uint32_t kColO = 256;
 __device__ __forceinline__ uint32_t col_s(int s) { return s ? 128u : 0u; }    // score buffers
 __device__ __forceinline__ uint32_t col_p(int s) { return s ? 448u : 384u; }  // bf16 P buffers
-constexpr size_t kSmem = 1024 + 5 * kTileBytes + 256;
+__host__ __device__ constexpr int tile_bytes(int hd) { return kTile * hd * 2; }  // a 128-row tile of Q, K or V
+__host__ __device__ constexpr size_t smem_one_tile(int hd) { return 1024 + 5 * tile_bytes(hd) + 256; }
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 
 // The two-tile kernel can be turned off with SAL_ATTN_PP=0 (to compare the two designs).
@@ -93,15 +94,17 @@ __device__ __forceinline__ void mask_chunk(uint32_t (&r)[32], int col0, int c_lo
     if (col0 + i < c_lo || col0 + i >= c_hi) r[i] = 0xff800000u;  // -inf
 }
 
+template <int HD>
 __global__ void __launch_bounds__(192, 1)
     attention_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                      const __grid_constant__ CUtensorMap tmV, const AttnArgs args) {
   extern __shared__ unsigned char smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  constexpr int TB = tile_bytes(HD);
   uint8_t* sQ = smem;
-  uint8_t* sK[2] = {smem + kTileBytes, smem + 2 * kTileBytes};
-  uint8_t* sV[2] = {smem + 3 * kTileBytes, smem + 4 * kTileBytes};
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + 5 * kTileBytes);
+  uint8_t* sK[2] = {smem + TB, smem + 2 * TB};
+  uint8_t* sV[2] = {smem + 3 * TB, smem + 4 * TB};
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + 5 * TB);
   uint64_t* q_full = bars + 0;
   uint64_t* k_full = bars + 1;    // [2]
   uint64_t* v_full = bars + 3;    // [2]
@@ -155,20 +158,20 @@ __global__ void __launch_bounds__(192, 1)
   if (warp == 0) {
     if (lane == 0) {
       uint32_t issued_q = 0, issued = 0, par_k = 0;
-      mbar_arrive_expect_tx(q_full, kTileBytes);
-      tma_load_3d(sQ, &tmQ, q_full, 0, qt * kTile, bh);
-      tma_load_3d(sQ + kBox, &tmQ, q_full, 64, qt * kTile, bh);
+      mbar_arrive_expect_tx(q_full, TB);
+#pragma unroll
+      for (int b = 0; b < HD / 64; ++b) tma_load_3d(sQ + b * kBox, &tmQ, q_full, 64 * b, qt * kTile, bh);
       issued_q = 1;
       for (int j = 0; j < n_kv; ++j) {
         const int s = j & 1;
         const uint32_t use_par = (j >> 1) & 1;
         if (!mbar_wait(&kv_empty[s], use_par ^ 1, guard)) break;
-        mbar_arrive_expect_tx(&k_full[s], kTileBytes);
-        tma_load_3d(sK[s], &tmK, &k_full[s], 0, (j0 + j) * kTile, bh);
-        tma_load_3d(sK[s] + kBox, &tmK, &k_full[s], 64, (j0 + j) * kTile, bh);
-        mbar_arrive_expect_tx(&v_full[s], kTileBytes);
-        tma_load_3d(sV[s], &tmV, &v_full[s], 0, (j0 + j) * kTile, bh);
-        tma_load_3d(sV[s] + kBox, &tmV, &v_full[s], 64, (j0 + j) * kTile, bh);
+        mbar_arrive_expect_tx(&k_full[s], TB);
+#pragma unroll
+        for (int b = 0; b < HD / 64; ++b) tma_load_3d(sK[s] + b * kBox, &tmK, &k_full[s], 64 * b, (j0 + j) * kTile, bh);
+        mbar_arrive_expect_tx(&v_full[s], TB);
+#pragma unroll
+        for (int b = 0; b < HD / 64; ++b) tma_load_3d(sV[s] + b * kBox, &tmV, &v_full[s], 64 * b, (j0 + j) * kTile, bh);
         issued |= 1u << s;
         par_k = (par_k & ~(1u << s)) | (use_par << s);
       }
@@ -184,7 +187,7 @@ __global__ void __launch_bounds__(192, 1)
   } else if (warp == 1) {
     if (lane == 0) {
       constexpr uint32_t IDESC_S = idesc_bf16(128, 128, false, false);
-      constexpr uint32_t IDESC_O = idesc_bf16(128, 128, false, true);
+      constexpr uint32_t IDESC_O = idesc_bf16(128, HD, false, true);
       bool ok = mbar_wait(q_full, 0, guard);
       bool any_mma = false;
       const uint32_t q0 = smem_u32(sQ);
@@ -194,7 +197,7 @@ __global__ void __launch_bounds__(192, 1)
         tc_fence_after();
         const uint32_t k0 = smem_u32(sK[s]);
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
+        for (int kk = 0; kk < HD / 16; ++kk) {
           const uint32_t off = (kk >> 2) * kBox + (kk & 3) * 32;
           umma_ss(tmem + col_s(s), sdesc_kmajor_sw128(q0 + off), sdesc_kmajor_sw128(k0 + off), IDESC_S,
                   kk > 0);
@@ -294,7 +297,7 @@ __global__ void __launch_bounds__(192, 1)
         tc_fence_after();
         if (__any_sync(0xffffffffu, rescale)) {
 #pragma unroll 1
-          for (int c = 0; c < 4; ++c) {
+          for (int c = 0; c < HD / 32; ++c) {
             uint32_t o[32];
             tmem_ld32(tmem + lane_base + kColO + 32 * c, o);
             tmem_wait_ld();
@@ -316,9 +319,9 @@ __global__ void __launch_bounds__(192, 1)
       const int64_t t = static_cast<int64_t>(qt) * kTile + row;
       const int b = bh / args.heads, h = bh % args.heads;
       const float inv_l = 1.0f / l;
-      __nv_bfloat16* dst = args.o + (static_cast<int64_t>(b) * T + t) * (args.heads * kHeadDim) + h * kHeadDim;
+      __nv_bfloat16* dst = args.o + (static_cast<int64_t>(b) * T + t) * (args.heads * HD) + h * HD;
 #pragma unroll 1
-      for (int c = 0; c < 4; ++c) {
+      for (int c = 0; c < HD / 32; ++c) {
         uint32_t o[32];
         tmem_ld32(tmem + lane_base + kColO + 32 * c, o);
         tmem_wait_ld();
@@ -647,16 +650,19 @@ bool g_pp_ok[64] = {};  // the two-tile kernel's launch registers cover its warp
 
 }  // namespace
 
-sal_status attention_launch(const void* q, const void* k, const void* v, int batch, int64_t T,
-                            int64_t chunk, void* o, cudaStream_t s) {
+sal_status attention_launch_heads(const void* q, const void* k, const void* v, int batch, int64_t T,
+                                  int64_t chunk, int heads, int head_dim, void* o, cudaStream_t s) {
   if (T == 0 || batch == 0) return SAL_OK;
+  if (head_dim != 64 && head_dim != 128) return SAL_ESHAPE;
   int dev = 0;
   cudaGetDevice(&dev);
   {
     std::lock_guard<std::mutex> lk(g_mu);
     if (dev >= 0 && dev < 64 && !g_attr[dev]) {
-      if (cudaFuncSetAttribute(attention_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               static_cast<int>(kSmem)) != cudaSuccess ||
+      if (cudaFuncSetAttribute(attention_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               static_cast<int>(smem_one_tile(128))) != cudaSuccess ||
+          cudaFuncSetAttribute(attention_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               static_cast<int>(smem_one_tile(64))) != cudaSuccess ||
           cudaFuncSetAttribute(attention_pp_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                static_cast<int>(kSmemPP)) != cudaSuccess)
         return SAL_ECUDA;
@@ -668,20 +674,26 @@ sal_status attention_launch(const void* q, const void* k, const void* v, int bat
       g_attr[dev] = true;
     }
   }
-  const uint64_t bh = static_cast<uint64_t>(batch) * kHeads;
+  const uint64_t bh = static_cast<uint64_t>(batch) * heads;
   CUtensorMap tq, tk, tv;
-  if (!make_tmap_3d_bf16(&tq, q, kHeadDim, T, bh, 64, kTile, 1)) return SAL_ECUDA;
-  if (!make_tmap_3d_bf16(&tk, k, kHeadDim, T, bh, 64, kTile, 1)) return SAL_ECUDA;
-  if (!make_tmap_3d_bf16(&tv, v, kHeadDim, T, bh, 64, kTile, 1)) return SAL_ECUDA;
+  if (!make_tmap_3d_bf16(&tq, q, head_dim, T, bh, 64, kTile, 1)) return SAL_ECUDA;
+  if (!make_tmap_3d_bf16(&tk, k, head_dim, T, bh, 64, kTile, 1)) return SAL_ECUDA;
+  if (!make_tmap_3d_bf16(&tv, v, head_dim, T, bh, 64, kTile, 1)) return SAL_ECUDA;
   AttnArgs a;
   a.T = T;
   a.chunk = chunk > 0 && chunk < T ? chunk : T;
-  a.heads = kHeads;
+  a.heads = heads;
   a.o = static_cast<__nv_bfloat16*>(o);
-  a.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(128.0));
+  a.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(head_dim)));
   a.limit_ns = wait_limit_ns();
   a.status = device_status_ptr();
   if (!a.status) return SAL_ECUDA;
+  const dim3 grid1(static_cast<unsigned>((T + kTile - 1) / kTile), static_cast<unsigned>(bh));
+  if (head_dim == 64)
+    return launch_kernel(attention_kernel<64>, grid1, dim3(192), smem_one_tile(64), s, tq, tk, tv, a) ==
+                   cudaSuccess
+               ? SAL_OK
+               : SAL_ECUDA;
   // Pick the kernel by waves of CTAs over the SMs: a two-tile CTA costs about 1.6 one-tile
   // CTAs (measured), so it wins unless its coarser grain leaves a mostly empty last wave.
   int sms = 148;
@@ -701,9 +713,15 @@ sal_status attention_launch(const void* q, const void* k, const void* v, int bat
                ? SAL_OK
                : SAL_ECUDA;
   }
-  const dim3 grid(static_cast<unsigned>((T + kTile - 1) / kTile), static_cast<unsigned>(bh));
-  return launch_kernel(attention_kernel, grid, dim3(192), kSmem, s, tq, tk, tv, a) == cudaSuccess ? SAL_OK
-                                                                                        : SAL_ECUDA;
+  return launch_kernel(attention_kernel<128>, grid1, dim3(192), smem_one_tile(128), s, tq, tk, tv, a) ==
+                 cudaSuccess
+             ? SAL_OK
+             : SAL_ECUDA;
+}
+
+sal_status attention_launch(const void* q, const void* k, const void* v, int batch, int64_t T,
+                            int64_t chunk, void* o, cudaStream_t s) {
+  return attention_launch_heads(q, k, v, batch, T, chunk, kHeads, kHeadDim, o, s);
 }
 
 }  // namespace sal

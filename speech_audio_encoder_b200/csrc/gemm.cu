@@ -34,6 +34,7 @@ namespace {
 struct GemmArgs {
   int64_t M;
   int N, K, splits;
+  int n_valid;  // rows of W and entries of the bias that exist (<= N; the rest read as 0)
   const __nv_bfloat16* bias;
   void* out;
   // QKV epilogue
@@ -385,7 +386,19 @@ __global__ void __launch_bounds__(192, 1)
             uint4 word;
             if constexpr (C::F32_OUT) {
               float v[4];
-              const uint2 bb = add_bias ? __ldg(reinterpret_cast<const uint2*>(bias8) + j) : make_uint2(0, 0);
+              uint2 bb = make_uint2(0, 0);
+              if (add_bias) {
+                const int cb = col0 + 4 * j;
+                if (cb + 4 <= args.n_valid) {
+                  bb = __ldg(reinterpret_cast<const uint2*>(bias8) + j);
+                } else {  // the last, partial bias chunk
+                  const uint16_t* bu = reinterpret_cast<const uint16_t*>(args.bias);
+                  uint32_t e[4];
+#pragma unroll
+                  for (int q = 0; q < 4; ++q) e[q] = cb + q < args.n_valid ? bu[cb + q] : 0u;
+                  bb = make_uint2(e[0] | (e[1] << 16), e[2] | (e[3] << 16));
+                }
+              }
               v[0] = __uint_as_float(r[4 * j + 0]) + bf16_lo(bb.x);
               v[1] = __uint_as_float(r[4 * j + 1]) + bf16_hi(bb.x);
               v[2] = __uint_as_float(r[4 * j + 2]) + bf16_lo(bb.y);
@@ -393,7 +406,17 @@ __global__ void __launch_bounds__(192, 1)
               word = make_uint4(__float_as_uint(v[0]), __float_as_uint(v[1]), __float_as_uint(v[2]),
                                 __float_as_uint(v[3]));
             } else {
-              const uint4 bb = __ldg(bias8 + j);
+              uint4 bb;
+              const int cb = col0 + 8 * j;
+              if (cb + 8 <= args.n_valid) {
+                bb = __ldg(bias8 + j);
+              } else {  // the last, partial bias chunk
+                const uint16_t* bu = reinterpret_cast<const uint16_t*>(args.bias);
+                uint32_t e[8];
+#pragma unroll
+                for (int q = 0; q < 8; ++q) e[q] = cb + q < args.n_valid ? bu[cb + q] : 0u;
+                bb = make_uint4(e[0] | (e[1] << 16), e[2] | (e[3] << 16), e[4] | (e[5] << 16), e[6] | (e[7] << 16));
+              }
               const uint32_t bw[4] = {bb.x, bb.y, bb.z, bb.w};
               uint32_t o[4];
 #pragma unroll
@@ -471,7 +494,7 @@ sal_status launch_bn(const GemmArgs& a, const void* A, const void* W, cudaStream
   }
   CUtensorMap ta, tb, tc;
   if (!make_tmap_2d_bf16(&ta, A, a.K, a.M, C::BK, C::BM)) return SAL_ECUDA;
-  if (!make_tmap_2d_bf16(&tb, W, a.K, a.N, C::BK, BN)) return SAL_ECUDA;
+  if (!make_tmap_2d_bf16(&tb, W, a.K, a.n_valid, C::BK, BN)) return SAL_ECUDA;  // rows >= n_valid: zeros
   if constexpr (C::QKV) {
     tc = ta;  // unused
   } else if constexpr (C::F32_OUT) {
@@ -514,9 +537,11 @@ int pick_bn(int64_t M, int N, bool qkv) {
 }  // namespace
 
 sal_status gemm_launch(int epilogue, const void* A, int64_t M, int K, const void* W, int N,
-                       const void* bias, void* out, const QkvOut* qkv, cudaStream_t s) {
+                       const void* bias, void* out, const QkvOut* qkv, cudaStream_t s, int n_valid) {
   if (M == 0) return SAL_OK;
   if (K <= 0 || K % 64 || N <= 0 || N % 64) return SAL_ESHAPE;
+  if (n_valid <= 0) n_valid = N;
+  if (n_valid > N || (epilogue == kEpiQkv && n_valid != N)) return SAL_EINVAL;
   if (M > (int64_t(1) << 31) - 1) return SAL_ESHAPE;
   const bool is_qkv = epilogue == kEpiQkv;
   if (is_qkv && (N != 3 * kWidth || !qkv)) return SAL_EINVAL;
@@ -525,6 +550,7 @@ sal_status gemm_launch(int epilogue, const void* A, int64_t M, int K, const void
   a.N = N;
   a.K = K;
   a.splits = 1;
+  a.n_valid = n_valid;
   a.bias = static_cast<const __nv_bfloat16*>(bias);
   a.out = out;
   a.limit_ns = wait_limit_ns();

@@ -1,8 +1,9 @@
 // Row kernels of the encoder: the pre-norm / final LayerNorm, and the RoPE table.
 //
-// LayerNorm (eps 1e-5, affine) normalises each 1280-wide fp32 row of the residual
-// stream and writes it as bf16, the operand of the next tensor-core GEMM. One warp per
-// row: 40 values per lane held in registers, two-pass mean and variance.
+// LayerNorm (eps 1e-5, affine) normalises each fp32 row of the residual stream (1280
+// wide in the encoder, 1024 in the CTC adapter) and writes it as bf16, the operand of the
+// next tensor-core GEMM. One warp per row: width / 32 values per lane held in registers,
+// two-pass mean and variance.
 //
 // RoPE table: cos and sin of t * 10000^(-2 i / 128), i < 64, t < T. The angle reaches
 // 4.5e4 rad at one hour, where fp32 would lose ~3 digits, so it is formed and reduced in
@@ -28,7 +29,6 @@ namespace sal {
 namespace {
 
 constexpr int kLnWarps = 8;
-constexpr int kVec = kWidth / 4 / 32;  // float4 per lane = 10
 
 __device__ __forceinline__ float warp_sum(float v) {
 #pragma unroll
@@ -36,16 +36,19 @@ __device__ __forceinline__ float warp_sum(float v) {
   return v;
 }
 
+// kVec float4 per lane: the row width is 128 kVec.
+template <int kVec>
 __global__ void __launch_bounds__(256) layernorm_kernel(const float* __restrict__ x, int64_t rows,
                                                         const __nv_bfloat16* __restrict__ g,
                                                         const __nv_bfloat16* __restrict__ b,
                                                         __nv_bfloat16* __restrict__ y) {
+  constexpr int kW = 128 * kVec;
   const int lane = threadIdx.x & 31;
   const int64_t row = static_cast<int64_t>(blockIdx.x) * kLnWarps + (threadIdx.x >> 5);
   pdl_wait();
   pdl_trigger();
   if (row >= rows) return;
-  const float4* xr = reinterpret_cast<const float4*>(x + row * kWidth);
+  const float4* xr = reinterpret_cast<const float4*>(x + row * kW);
   float4 v[kVec];
   float s = 0.f;
 #pragma unroll
@@ -53,17 +56,17 @@ __global__ void __launch_bounds__(256) layernorm_kernel(const float* __restrict_
     v[i] = xr[lane + 32 * i];
     s += (v[i].x + v[i].y) + (v[i].z + v[i].w);
   }
-  const float mean = warp_sum(s) * (1.0f / kWidth);
+  const float mean = warp_sum(s) * (1.0f / kW);
   float q = 0.f;
 #pragma unroll
   for (int i = 0; i < kVec; ++i) {
     const float a = v[i].x - mean, bb = v[i].y - mean, c = v[i].z - mean, d = v[i].w - mean;
     q += (a * a + bb * bb) + (c * c + d * d);
   }
-  const float rstd = 1.0f / sqrtf(warp_sum(q) * (1.0f / kWidth) + 1e-5f);
+  const float rstd = 1.0f / sqrtf(warp_sum(q) * (1.0f / kW) + 1e-5f);
   const uint2* g2 = reinterpret_cast<const uint2*>(g);
   const uint2* b2 = reinterpret_cast<const uint2*>(b);
-  uint2* yr = reinterpret_cast<uint2*>(y + row * kWidth);
+  uint2* yr = reinterpret_cast<uint2*>(y + row * kW);
 #pragma unroll
   for (int i = 0; i < kVec; ++i) {
     const int c4 = lane + 32 * i;
@@ -202,14 +205,20 @@ sal_status speaker_fuse_launch(const void* H, const float* P, int64_t rows, cons
 }
 
 sal_status layernorm_launch(const float* x, int64_t rows, const void* g, const void* b, void* y,
-                            cudaStream_t s) {
+                            cudaStream_t s, int width) {
   if (rows == 0) return SAL_OK;
   const unsigned grid = static_cast<unsigned>((rows + kLnWarps - 1) / kLnWarps);
-  return launch_kernel(layernorm_kernel, dim3(grid), dim3(32 * kLnWarps), 0, s, x, rows,
-                       static_cast<const __nv_bfloat16*>(g), static_cast<const __nv_bfloat16*>(b),
-                       static_cast<__nv_bfloat16*>(y)) == cudaSuccess
-             ? SAL_OK
-             : SAL_ECUDA;
+  const auto gg = static_cast<const __nv_bfloat16*>(g);
+  const auto bb = static_cast<const __nv_bfloat16*>(b);
+  const auto yy = static_cast<__nv_bfloat16*>(y);
+  cudaError_t e;
+  if (width == kWidth)
+    e = launch_kernel(layernorm_kernel<kWidth / 128>, dim3(grid), dim3(32 * kLnWarps), 0, s, x, rows, gg, bb, yy);
+  else if (width == 1024)
+    e = launch_kernel(layernorm_kernel<8>, dim3(grid), dim3(32 * kLnWarps), 0, s, x, rows, gg, bb, yy);
+  else
+    return SAL_ESHAPE;
+  return e == cudaSuccess ? SAL_OK : SAL_ECUDA;
 }
 
 sal_status rope_table_launch(float* cs, int64_t T, cudaStream_t s) {

@@ -91,6 +91,44 @@ EncoderWs encoder_ws_layout(void* base, int batch, int64_t T) {
   return w;
 }
 
+// CTC adapter workspace over M2 = batch * 2T positions of width 1024: the fp32 residual
+// stream x, the bf16 LN output h, q / k / v / o, one large region that holds in turn the
+// fp32 QKV rows, the bf16 FFN hidden rows and the fp32 class scores, the RoPE table of
+// the 2T positions, and the upsampling bias repeated for both taps.
+constexpr int kCtcClassesPad = (SAL_CTC_CLASSES + 255) / 256 * 256;  // 24,064: 256-wide column tiles
+
+struct CtcWs {
+  float* x;
+  void *h, *q, *k, *v, *o, *big, *bias2;
+  float* rope;
+  size_t bytes;
+};
+
+CtcWs ctc_ws_layout(void* base, int batch, int64_t T) {
+  const size_t M2 = static_cast<size_t>(batch) * static_cast<size_t>(2 * T);
+  const size_t W = SAL_CTC_WIDTH;
+  char* p = static_cast<char*>(base);
+  CtcWs w{};
+  size_t off = 0;
+  auto take = [&](size_t n) {
+    char* r = p + off;
+    off += align256(n);
+    return r;
+  };
+  w.x = reinterpret_cast<float*>(take(M2 * W * 4));
+  w.h = take(M2 * W * 2);
+  w.q = take(M2 * W * 2);
+  w.k = take(M2 * W * 2);
+  w.v = take(M2 * W * 2);
+  w.o = take(M2 * W * 2);
+  w.big = take(M2 * std::max(std::max(3 * W * 4, static_cast<size_t>(SAL_CTC_FFN) * 2),
+                             static_cast<size_t>(kCtcClassesPad) * 4));
+  w.rope = reinterpret_cast<float*>(take(static_cast<size_t>(2 * T) * 64 * 2 * sizeof(float)));
+  w.bias2 = take(2 * W * 2);
+  w.bytes = off;
+  return w;
+}
+
 bool layer_ok(const sal_layer& L) {
   const void* ps[] = {L.ln1_g, L.ln1_b, L.w_qkv, L.b_qkv, L.qn_g, L.kn_g, L.w_o,
                       L.b_o,   L.ln2_g, L.ln2_b, L.w1,    L.b1,    L.w2,   L.b2};
@@ -448,6 +486,81 @@ sal_status sal_attention_chunked(const void* q, const void* k, const void* v, in
     return SAL_EINVAL;
   SAL_TRY(check_device());
   return attention_launch(q, k, v, batch, T, chunk, o, static_cast<cudaStream_t>(stream));
+}
+
+sal_status sal_attention_heads(const void* q, const void* k, const void* v, int batch, int64_t T, int heads,
+                               int head_dim, void* o, void* stream) {
+  if (batch < 0 || T < 0 || heads < 0) return SAL_EINVAL;
+  if (head_dim != 64 && head_dim != 128) return SAL_ESHAPE;
+  if (T > 2 * SAL_MAX_POSITIONS) return SAL_ESHAPE;
+  if (batch == 0 || T == 0 || heads == 0) return SAL_OK;
+  if (static_cast<int64_t>(batch) * heads > 65535) return SAL_ESHAPE;  // grid.y
+  if (!q || !k || !v || !o || !aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o))
+    return SAL_EINVAL;
+  SAL_TRY(check_device());
+  return attention_launch_heads(q, k, v, batch, T, 0, heads, head_dim, o, static_cast<cudaStream_t>(stream));
+}
+
+sal_status sal_log_softmax(const float* z, int64_t rows, int n, int64_t ld, float* out, void* stream) {
+  if (rows < 0 || n < 0 || ld < n) return SAL_EINVAL;
+  if (rows == 0 || n == 0) return SAL_OK;
+  if (!z || !out) return SAL_EINVAL;
+  SAL_TRY(check_device());
+  return log_softmax_launch(z, rows, n, ld, out, static_cast<cudaStream_t>(stream));
+}
+
+size_t sal_ctc_workspace_bytes(int batch, int64_t T) {
+  if (batch <= 0 || T <= 0) return 0;
+  return ctc_ws_layout(nullptr, batch, T).bytes;
+}
+
+sal_status sal_ctc_adapter(const void* h, int batch, int64_t T, const sal_ctc_weights* w, float* logp,
+                           void* workspace, size_t ws_bytes, void* stream) {
+  if (batch < 0 || T < 0 || !w || w->n_layers < 0) return SAL_EINVAL;
+  if (T > SAL_MAX_POSITIONS || batch > 4095) return SAL_ESHAPE;  // attention grid.y = 16 * batch
+  if (batch == 0 || T == 0) return SAL_OK;
+  if (!h || !logp || !aligned16(h) || !aligned16(logp)) return SAL_EINVAL;
+  const void* ps[] = {w->w_up, w->b_up, w->lnf_g, w->lnf_b, w->w_out, w->b_out};
+  for (const void* p : ps)
+    if (!p || !aligned16(p)) return SAL_EINVAL;
+  if (w->n_layers > 0 && !w->layers) return SAL_EINVAL;
+  for (int i = 0; i < w->n_layers; ++i)
+    if (!layer_ok(w->layers[i])) return SAL_EINVAL;
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u)) return SAL_EINVAL;
+  const CtcWs ws = ctc_ws_layout(workspace, batch, T);
+  if (ws_bytes < ws.bytes) return SAL_EWORKSPACE;
+  SAL_TRY(check_device());
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  constexpr int W = SAL_CTC_WIDTH, F = SAL_CTC_FFN;
+  const int64_t T2 = 2 * T, M2 = static_cast<int64_t>(batch) * T2;
+  // the transposed convolution as one GEMM: [B T, 1280] x [2048, 1280]^T -> [B T, 2048],
+  // which read row-major is [B 2T, 1024] (tap j of input t lands on row 2t + j); the bias
+  // of an output channel is the same for both taps
+  if (cudaMemcpyAsync(ws.bias2, w->b_up, W * 2, cudaMemcpyDeviceToDevice, s) != cudaSuccess ||
+      cudaMemcpyAsync(static_cast<char*>(ws.bias2) + W * 2, w->b_up, W * 2, cudaMemcpyDeviceToDevice, s) !=
+          cudaSuccess)
+    return SAL_ECUDA;
+  SAL_TRY(gemm_launch(SAL_EPI_STORE_F32, h, static_cast<int64_t>(batch) * T, kWidth, w->w_up, 2 * W, ws.bias2,
+                      ws.x, nullptr, s));
+  if (w->n_layers > 0) SAL_TRY(rope_table_launch(ws.rope, T2, s));
+  for (int i = 0; i < w->n_layers; ++i) {
+    const sal_layer& L = w->layers[i];
+    SAL_TRY(layernorm_launch(ws.x, M2, L.ln1_g, L.ln1_b, ws.h, s, W));
+    SAL_TRY(gemm_launch(SAL_EPI_STORE_F32, ws.h, M2, W, L.w_qkv, 3 * W, L.b_qkv, ws.big, nullptr, s));
+    SAL_TRY(ctc_qk_norm_rope_launch(static_cast<const float*>(ws.big), M2, T2, L.qn_g, L.kn_g, ws.rope, ws.q, ws.k,
+                                    ws.v, s));
+    SAL_TRY(attention_launch_heads(ws.q, ws.k, ws.v, batch, T2, 0, SAL_CTC_HEADS, SAL_CTC_HEAD_DIM, ws.o, s));
+    SAL_TRY(gemm_launch(SAL_EPI_RESID_F32, ws.o, M2, W, L.w_o, W, L.b_o, ws.x, nullptr, s));
+    SAL_TRY(layernorm_launch(ws.x, M2, L.ln2_g, L.ln2_b, ws.h, s, W));
+    SAL_TRY(gemm_launch(SAL_EPI_GELU_BF16, ws.h, M2, W, L.w1, F, L.b1, ws.big, nullptr, s));
+    SAL_TRY(gemm_launch(SAL_EPI_RESID_F32, ws.big, M2, F, L.w2, W, L.b2, ws.x, nullptr, s));
+  }
+  SAL_TRY(layernorm_launch(ws.x, M2, w->lnf_g, w->lnf_b, ws.h, s, W));
+  // class scores over a width padded to a multiple of 256 (the rows of w_out past 23,863
+  // read as zero), then the log-softmax of the 23,863 real ones
+  SAL_TRY(gemm_launch(SAL_EPI_STORE_F32, ws.h, M2, W, w->w_out, kCtcClassesPad, w->b_out, ws.big, nullptr, s,
+                      SAL_CTC_CLASSES));
+  return log_softmax_launch(static_cast<const float*>(ws.big), M2, SAL_CTC_CLASSES, kCtcClassesPad, logp, s);
 }
 
 }  // extern "C"

@@ -33,7 +33,7 @@ sal_status frontend_launch(const float* wave, int64_t n_samples, int batch, int6
 
 // rowops.cu
 sal_status layernorm_launch(const float* x, int64_t rows, const void* g, const void* b, void* y,
-                            cudaStream_t s);
+                            cudaStream_t s, int width = kWidth);  // width 1280 or 1024
 sal_status rope_table_launch(float* cs, int64_t T, cudaStream_t s);
 sal_status speaker_fuse_launch(const void* H, const float* P, int64_t rows, const void* g, const void* b, void* out,
                                cudaStream_t s);
@@ -46,13 +46,25 @@ struct QkvOut {
   int64_t T;
   int64_t chunk;         // positions restart every `chunk` positions (<= 0: whole clip)
 };
+// n_valid (0: N) < N runs the column tiles over N but reads only n_valid rows of W and
+// entries of the bias; the columns past n_valid come out as 0 (for an N that is not a
+// multiple of 64, into an output N columns wide).
 sal_status gemm_launch(int epilogue, const void* A, int64_t M, int K, const void* W, int N,
-                       const void* bias, void* out, const QkvOut* qkv, cudaStream_t s);
+                       const void* bias, void* out, const QkvOut* qkv, cudaStream_t s, int n_valid = 0);
 constexpr int kEpiQkv = 100;  // internal epilogue id: QK-norm + RoPE scatter
 
 // attention.cu
 sal_status attention_launch(const void* q, const void* k, const void* v, int batch, int64_t T,
                             int64_t chunk, void* o, cudaStream_t s);
+// Any number of heads of width 64 or 128 (o is [batch, T, heads * head_dim]); head_dim 64
+// always runs the one-tile kernel.
+sal_status attention_launch_heads(const void* q, const void* k, const void* v, int batch, int64_t T,
+                                  int64_t chunk, int heads, int head_dim, void* o, cudaStream_t s);
+
+// ctc.cu
+sal_status ctc_qk_norm_rope_launch(const float* qkv, int64_t rows, int64_t T, const void* qn_g, const void* kn_g,
+                                   const float* cs, void* q, void* k, void* v, cudaStream_t s);
+sal_status log_softmax_launch(const float* z, int64_t rows, int n, int64_t ld, float* out, cudaStream_t s);
 
 // tensor maps (sal_api.cu)
 bool make_tmap_2d_bf16(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer,

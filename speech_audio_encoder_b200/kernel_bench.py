@@ -3,7 +3,7 @@
     python -m speech_audio_encoder_b200.kernel_bench KIND [--batch B] [--T T] [--reps R]
 
 KIND is one of frontend, stack_proj, layernorm, qkv, attention, out_proj, ffn_up, ffn_down,
-speaker_fuse, connector, linear (any --N, --K, --epi).
+speaker_fuse, connector, ctc (the whole CTC adapter), linear (any --N, --K, --epi).
 Each repetition is one launch (qkv also launches the small RoPE-table kernel). The
 repetitions are captured once as a CUDA graph and the replay is timed with CUDA events on
 the launching stream after warm-up (eager launches from Python would measure the host). Prints one JSON line with the
@@ -86,6 +86,18 @@ def main():
 
         def run():
             api.sal_connector(x, W, bias)
+    elif a.kind == "ctc":
+        # the whole CTC timestamp adapter on B clips of T encoder positions (2T at 40 ms)
+        dw = api.DeviceCtcWeights(synth.make_ctc_weights())
+        h = _bf16((M, 1280), 13, 1.0)
+        logp = torch.empty((2 * M, api.CTC_CLASSES), dtype=torch.float32, device="cuda")
+        ws = api.ctc_workspace(B, T)
+        M2, T2 = 2 * M, 2 * T
+        flops = (2.0 * M * 1280 * 2048 + 2 * (2.0 * M2 * 1024 * (3072 + 1024 + 2 * 4096) + 4.0 * T2 * T2 * 1024 * B)
+                 + 2.0 * M2 * 1024 * api.CTC_CLASSES)
+
+        def run():
+            api.sal_ctc_adapter(h, B, T, dw, logp=logp, workspace=ws)
     elif a.kind == "linear":
         K, N, epi = a.K, a.N, a.epi
         A = _bf16((M, K), 4, 1.0)

@@ -3,6 +3,7 @@
 Runs without a GPU: it only calls host-side functions (counts, workspace sizes, status
 strings) and argument checks that return before any CUDA call.
 """
+import ctypes
 import os
 import re
 
@@ -67,3 +68,23 @@ def test_argument_checks_before_any_cuda_call(api):
     assert lib.sal_linear(0, 0, 0, 64, 0, 64, 0, 0, 0) == 0     # M = 0
     assert lib.sal_attention(0, 0, 0, 1, 45001, 0, 0) == 2
     assert lib.sal_attention(0, 0, 0, 1, 0, 0, 0) == 0
+
+
+def test_ctc_adapter_host_checks(api):
+    lib = api.lib()
+    assert lib.sal_ctc_workspace_bytes(0, 10) == 0
+    w1 = lib.sal_ctc_workspace_bytes(1, 374)
+    # per 40 ms position at least: fp32 x, bf16 h/q/k/v/o, fp32 class scores over 23,872 columns
+    assert w1 >= 748 * (1024 * 4 + 5 * 1024 * 2 + 23872 * 4)
+    assert lib.sal_ctc_workspace_bytes(2, 374) > w1
+    rec = api.sal_ctc_weights()
+    assert lib.sal_ctc_adapter(0, -1, 10, ctypes.byref(rec), 0, 0, 0, 0) == 1      # negative batch
+    assert lib.sal_ctc_adapter(0, 1, 45001, ctypes.byref(rec), 0, 0, 0, 0) == 2    # more than one hour
+    assert lib.sal_ctc_adapter(0, 4096, 10, ctypes.byref(rec), 0, 0, 0, 0) == 2    # attention grid.y
+    assert lib.sal_ctc_adapter(0, 0, 10, ctypes.byref(rec), 0, 0, 0, 0) == 0       # nothing to do
+    assert lib.sal_ctc_adapter(0, 1, 10, ctypes.byref(rec), 0, 0, 0, 0) == 1       # null pointers
+    assert lib.sal_attention_heads(0, 0, 0, 1, 10, 16, 96, 0, 0) == 2              # head width 96
+    assert lib.sal_attention_heads(0, 0, 0, 1, 90001, 16, 64, 0, 0) == 2
+    assert lib.sal_attention_heads(0, 0, 0, 1, 10, 16, 64, 0, 0) == 1
+    assert lib.sal_log_softmax(0, 4, 10, 5, 0, 0) == 1                             # ld < n
+    assert lib.sal_log_softmax(0, 0, 10, 10, 0, 0) == 0
