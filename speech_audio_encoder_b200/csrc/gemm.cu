@@ -142,7 +142,9 @@ __global__ void __launch_bounds__(192, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  pdl_wait();
+  // Programmatic dependent launch: the roles that read or write what earlier kernels
+  // produce (the A loads, the epilogue) wait for them below; the weight loads of the
+  // first tile and the MMA warp (shared and tensor memory only) do not.
   pdl_trigger();
   const uint32_t tmem_base = *tmem_slot;
   const WaitGuard guard{abort_flag, args.limit_ns, args.status};
@@ -156,16 +158,34 @@ __global__ void __launch_bounds__(192, 1)
     if (lane == 0) {
       int stage = 0;
       uint32_t phase = 0, issued = 0, issued_par = 0;
+      // The weights do not depend on the previous kernel: the W tiles of the first stages
+      // of this CTA's first tile go out before the wait (the stages start empty), their
+      // A tiles after it, completing the same barriers.
+      const int tile0 = blockIdx.x;
+      int pre = 0;
+      if (tile0 < num_tiles) {
+        const int sp0 = tile0 % args.splits, n0 = (tile0 / args.splits) % num_n;
+        pre = kb_per < C::STAGES ? kb_per : C::STAGES;
+        for (int i = 0; i < pre; ++i) {
+          mbar_arrive_expect_tx(&full[i], C::STAGE_BYTES);
+          tma_load_2d(sB + i * C::B_BYTES, &tmB, &full[i], (sp0 * kb_per + i) * C::BK, n0 * BN);
+        }
+      }
+      pdl_wait();
       for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
         const int sp = tile % args.splits;
         const int rest = tile / args.splits;
         const int n = rest % num_n, m = rest / num_n;
         for (int i = 0; i < kb_per; ++i) {
           const int kb = sp * kb_per + i;
-          if (!mbar_wait(&empty[stage], phase ^ 1, guard)) goto producer_done;
-          mbar_arrive_expect_tx(&full[stage], C::STAGE_BYTES);
-          tma_load_2d(sA + stage * C::A_BYTES, &tmA, &full[stage], kb * C::BK, m * C::BM);
-          tma_load_2d(sB + stage * C::B_BYTES, &tmB, &full[stage], kb * C::BK, n * BN);
+          if (tile == tile0 && i < pre) {  // stage i already expects its bytes; W is in flight
+            tma_load_2d(sA + stage * C::A_BYTES, &tmA, &full[stage], kb * C::BK, m * C::BM);
+          } else {
+            if (!mbar_wait(&empty[stage], phase ^ 1, guard)) goto producer_done;
+            mbar_arrive_expect_tx(&full[stage], C::STAGE_BYTES);
+            tma_load_2d(sA + stage * C::A_BYTES, &tmA, &full[stage], kb * C::BK, m * C::BM);
+            tma_load_2d(sB + stage * C::B_BYTES, &tmB, &full[stage], kb * C::BK, n * BN);
+          }
           issued |= 1u << stage;
           issued_par = (issued_par & ~(1u << stage)) | (phase << stage);
           if (++stage == C::STAGES) {
@@ -223,6 +243,7 @@ __global__ void __launch_bounds__(192, 1)
   } else {
     // ------------------------------------------------------------ epilogue warps 2..5
     // Each warp owns TMEM lanes (= tile rows) 32 q .. 32 q + 31, one row per thread.
+    pdl_wait();  // outputs (and the RoPE table) are shared with earlier kernels
     const int quarter = warp & 3;
     uint32_t acc = 0, acc_phase = 0;
     if constexpr (C::QKV) {
