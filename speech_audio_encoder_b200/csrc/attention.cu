@@ -279,9 +279,16 @@ __global__ void __launch_bounds__(192, 1)
       for (int c = 0; c < 4; ++c)
 #pragma unroll
         for (int i = 0; i < 32; i += 2) {
-          float x0, x1;
+          float x0, x1, e0, e1;
           f2_unpack(f2_fma(f2_pack(__uint_as_float(r[c][i]), __uint_as_float(r[c][i + 1])), sl2_2, negm_2), x0, x1);
-          const float e0 = fast_exp2(x0), e1 = fast_exp2(x1);
+          if (HD == 64 && ((i >> 1) & 7) < 3) {
+            // head dim 64: the MMAs of a tile take half the SFU's exponential time, so 6 of
+            // every 16 pairs go to the FMA pipe
+            exp2_pair_poly(x0, x1, e0, e1);
+          } else {
+            e0 = fast_exp2(x0);
+            e1 = fast_exp2(x1);
+          }
           sum2 = f2_add(sum2, f2_pack(e0, e1));
           p[c >> 1][(c & 1) * 16 + (i >> 1)] = pack_bf16x2(e0, e1);
         }

@@ -352,4 +352,29 @@ __device__ __forceinline__ float fast_exp2(float x) {
   return y;
 }
 
+// 2^x for a pair of inputs on the FMA and integer pipes, leaving the SFU free: Cody-Waite
+// style reduction x = j + f with j = round(x) obtained by adding the shifter 1.5 * 2^23
+// (f in [-0.5, 0.5]), the degree-4 Taylor polynomial of 2^f = e^(f ln 2) (coefficients
+// (ln 2)^k / k!, relative error < 6e-5 on that interval), and 2^j applied by adding j to
+// the exponent field. Inputs are clamped at -125; the result there (< 2^-124) is
+// negligible next to a softmax row sum, which is at least 1.
+__device__ __forceinline__ void exp2_pair_poly(float x0, float x1, float& e0, float& e1) {
+  constexpr float kShift = 12582912.0f;  // 1.5 * 2^23: the sum's last mantissa bit has weight 1
+  const uint64_t x = f2_pack(fmaxf(x0, -125.f), fmaxf(x1, -125.f));
+  const uint64_t t = f2_add(x, f2_pack(kShift, kShift));
+  const uint64_t jf = f2_add(t, f2_pack(-kShift, -kShift));
+  const uint64_t f = f2_fma(jf, f2_pack(-1.f, -1.f), x);
+  uint64_t p = f2_fma(f, f2_pack(0.009618129107628477f, 0.009618129107628477f),
+                      f2_pack(0.055504108664821576f, 0.055504108664821576f));
+  p = f2_fma(p, f, f2_pack(0.2402265069591007f, 0.2402265069591007f));
+  p = f2_fma(p, f, f2_pack(0.6931471805599453f, 0.6931471805599453f));
+  p = f2_fma(p, f, f2_pack(1.f, 1.f));
+  float p0, p1, t0, t1;
+  f2_unpack(p, p0, p1);
+  f2_unpack(t, t0, t1);
+  const int j0 = __float_as_int(t0) - 0x4B400000, j1 = __float_as_int(t1) - 0x4B400000;
+  e0 = __int_as_float(__float_as_int(p0) + (j0 << 23));
+  e1 = __int_as_float(__float_as_int(p1) + (j1 << 23));
+}
+
 }  // namespace sal

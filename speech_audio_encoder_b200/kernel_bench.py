@@ -3,7 +3,8 @@
     python -m speech_audio_encoder_b200.kernel_bench KIND [--batch B] [--T T] [--reps R]
 
 KIND is one of frontend, stack_proj, layernorm, qkv, attention, out_proj, ffn_up, ffn_down,
-speaker_fuse, connector, ctc (the whole CTC adapter), linear (any --N, --K, --epi).
+speaker_fuse, connector, ctc (the whole CTC adapter), attention64 (its 16 heads of 64),
+linear (any --N, --K, --epi).
 Each repetition is one launch (qkv also launches the small RoPE-table kernel). The
 repetitions are captured once as a CUDA graph and the replay is timed with CUDA events on
 the launching stream after warm-up (eager launches from Python would measure the host). Prints one JSON line with the
@@ -70,6 +71,12 @@ def main():
 
         def run():
             api.sal_attention(q, k, v)
+    elif a.kind == "attention64":  # the CTC adapter's heads: 16 of width 64
+        q, k, v = (_bf16((B, 16, T, 64), 20 + i, 1.0) for i in range(3))
+        flops = 4.0 * T * T * 1024 * B
+
+        def run():
+            api.sal_attention_heads(q, k, v)
     elif a.kind == "speaker_fuse":
         H = _bf16((M, 1280), 7, 1.0)
         P = torch.from_numpy(synth.speaker_activity(M, 1)).cuda()
