@@ -38,13 +38,15 @@ __host__ __device__ constexpr int tile_bytes(int hd) { return kTile * hd * 2; } 
 __host__ __device__ constexpr size_t smem_one_tile(int hd) { return 1024 + 5 * tile_bytes(hd) + 256; }
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 
-// The two-tile kernel can be turned off with SAL_ATTN_PP=0 (to compare the two designs).
-bool attention_pp_enabled() {
-  static const bool on = [] {
+// The choice between the one-tile and two-tile kernels can be forced with SAL_ATTN_PP.
+// SAL_ATTN_PP: unset = choose by the wave model below, 0 = never the two-tile kernel,
+// 1 = always (where its grid has at least one query-tile pair); for measuring the choice.
+int attention_pp_mode() {
+  static const int mode = [] {
     const char* e = std::getenv("SAL_ATTN_PP");
-    return !(e && e[0] == '0');
+    return e && e[0] == '0' ? 0 : (e && e[0] == '1' ? 1 : -1);
   }();
-  return on;
+  return mode;
 }
 
 struct AttnArgs {
@@ -714,7 +716,8 @@ sal_status attention_launch_heads(const void* q, const void* k, const void* v, i
     std::lock_guard<std::mutex> lk(g_mu);
     pp_ok = dev >= 0 && dev < 64 && g_pp_ok[dev];
   }
-  if (pp_ok && ctas_pp >= 120 && waves_pp < waves_1 && attention_pp_enabled()) {
+  const int mode = attention_pp_mode();
+  if (pp_ok && mode != 0 && (mode == 1 || (ctas_pp >= 120 && waves_pp < waves_1))) {
     const dim3 grid(static_cast<unsigned>((T + 2 * kTile - 1) / (2 * kTile)), static_cast<unsigned>(bh));
     return launch_kernel(attention_pp_kernel, grid, dim3(kThreadsPP), kSmemPP, s, tq, tk, tv, a) == cudaSuccess
                ? SAL_OK
