@@ -57,7 +57,7 @@ struct Cfg {
   // other kinds stage 128-byte-wide output boxes for TMA, two per warp
   static constexpr int CW = F32_OUT ? 32 : 64;  // output columns per 128-byte box row
   static constexpr int SCR_BYTES = QKV ? 4 * 32 * 128 * 4 + 4 * 32 * 4 : 4 * 2 * 4096;
-  static constexpr int STAGES = QKV ? 4 : (BN == 256 ? 4 : (BN == 128 ? 6 : 8));
+  static constexpr int STAGES = QKV ? (BN == 256 ? 3 : 4) : (BN == 256 ? 4 : (BN == 128 ? 6 : 8));
   static constexpr int A_BYTES = BM * BK * 2;
   static constexpr int B_BYTES = BN * BK * 2;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
@@ -532,8 +532,8 @@ sal_status launch_bn(const GemmArgs& a, const void* A, const void* W, cudaStream
 
 template <int EPI>
 sal_status launch_epi(int BN, const GemmArgs& a, const void* A, const void* W, cudaStream_t s) {
-  if constexpr (EPI == kEpiQkv) {  // one head per tile
-    return BN == 128 ? launch_bn<128, EPI>(a, A, W, s) : SAL_ESHAPE;
+  if constexpr (EPI == kEpiQkv) {  // one or two heads per tile
+    return BN == 256 ? launch_bn<256, EPI>(a, A, W, s) : (BN == 128 ? launch_bn<128, EPI>(a, A, W, s) : SAL_ESHAPE);
   } else {
     switch (BN) {
       case 256: return launch_bn<256, EPI>(a, A, W, s);
@@ -548,8 +548,10 @@ sal_status launch_epi(int BN, const GemmArgs& a, const void* A, const void* W, c
 // re-reading A for every column tile and W for every row tile; measured at M = 374,
 // 128-wide tiles beat 64 (fewer A re-reads) and 256 (too few CTAs).
 int pick_bn(int64_t M, int N, bool qkv) {
-  if (qkv) return 128;
   const int64_t mt = (M + 127) / 128;
+  // QKV: two heads per tile once those tiles fill the SMs (a 256-wide tile never straddles
+  // the q / k / v sections: 1280 and 2560 are multiples of 256)
+  if (qkv) return mt * (N / 256) >= num_sms() ? 256 : 128;
   if (N % 256 == 0 && mt * (N / 256) >= num_sms()) return 256;
   if (N % 128 == 0) return 128;
   return 64;

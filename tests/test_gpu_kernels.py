@@ -103,7 +103,9 @@ def test_linear_rejects_bad_shapes():
 
 # ---------------------------------------------------------------- QKV + QK-norm + RoPE
 
-@pytest.mark.parametrize("batch,T", [(1, 1), (2, 7), (1, 129), (3, 300), (1, 3000)])
+# (2, 700) and (1, 3000) fill the SMs with two-head (256-wide) tiles; (2, 700) also puts
+# a clip boundary inside a tile.
+@pytest.mark.parametrize("batch,T", [(1, 1), (2, 7), (1, 129), (3, 300), (2, 700), (1, 3000)])
 def test_qkv_rope(batch, T):
     api = _api()
     w, wf, dw = weights(1)
