@@ -20,7 +20,11 @@
 #include <math.h>
 
 #include <cstdlib>
+#include <map>
 #include <mutex>
+#include <queue>
+#include <tuple>
+#include <vector>
 
 #include "sal_internal.h"
 #include "sal_ptx.cuh"
@@ -50,6 +54,8 @@ int attention_pp_mode() {
 }
 
 struct AttnArgs {
+  int qt0 = 0;    // one-tile kernel: first query tile of this launch
+  int tail = 0;   // one-tile kernel launched behind the two-tile kernel (see attention_launch_heads)
   int64_t T;
   int64_t chunk;  // attention stays inside chunks of this many positions (T: whole clip)
   int heads;
@@ -122,7 +128,7 @@ __global__ void __launch_bounds__(192, 1)
   const int lane = threadIdx.x & 31;
   const int64_t T = args.T;
   const int bh = blockIdx.y;
-  const int qt = blockIdx.x;
+  const int qt = blockIdx.x + args.qt0;
   int j0, n_kv;
   kv_tile_range(static_cast<int64_t>(qt) * kTile,
                 static_cast<int64_t>(qt) * kTile + kTile < T ? static_cast<int64_t>(qt) * kTile + kTile : T, T,
@@ -152,7 +158,10 @@ __global__ void __launch_bounds__(192, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  pdl_wait();
+  // A tail launch reads only what the two-tile kernel ahead of it had already waited for
+  // (its CTAs start after every two-tile CTA passed griddepcontrol.wait), so it starts at
+  // once and waits for that kernel at exit instead, before its own completion.
+  if (!args.tail) pdl_wait();
   pdl_trigger();
   const uint32_t tmem = *tmem_slot;
   const WaitGuard guard{abort_flag, args.limit_ns, args.status};
@@ -357,6 +366,7 @@ __global__ void __launch_bounds__(192, 1)
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
+  if (args.tail) pdl_wait();
 }
 
 // ---------------------------------------------------------------------------------
@@ -657,6 +667,63 @@ std::mutex g_mu;
 bool g_attr[64] = {};
 bool g_pp_ok[64] = {};  // the two-tile kernel's launch registers cover its warpgroup split
 
+// Makespan of n2 two-tile CTAs (cost kPairCost each, in units of one one-tile CTA over the
+// same keys) followed by n1 one-tile CTAs, placed in launch order on the first free SM.
+constexpr double kPairCost = 1.55;  // measured: 1.41 - 1.57 over 3,000 - 12,000 positions
+constexpr int kMinSplitTiles = 16;  // query tiles per clip below which no split is tried
+
+double makespan(uint64_t n2, uint64_t n1, int sms) {
+  std::priority_queue<double, std::vector<double>, std::greater<double>> free_at;
+  for (int i = 0; i < sms; ++i) free_at.push(0.0);
+  double end = 0.0;
+  auto place = [&](uint64_t n, double cost) {
+    for (uint64_t i = 0; i < n; ++i) {
+      const double t = free_at.top() + cost;
+      free_at.pop();
+      free_at.push(t);
+      end = t > end ? t : end;
+    }
+  };
+  place(n2, kPairCost);
+  place(n1, 1.0);
+  return end;
+}
+
+// Pairs per (clip, head) for the two-tile kernel: 0 (one-tile only), all of them, or the
+// largest count whose CTAs fill whole waves, whichever schedules shortest. Cached per shape.
+int choose_pairs(int n_qt, uint64_t bh, int sms) {
+  static std::mutex mu;
+  static std::map<std::tuple<int, uint64_t, int>, int> cache;
+  const auto key = std::make_tuple(n_qt, bh, sms);
+  {
+    std::lock_guard<std::mutex> lk(mu);
+    auto it = cache.find(key);
+    if (it != cache.end()) return it->second;
+  }
+  const int all = (n_qt + 1) / 2;
+  int best = 0;
+  double best_t = makespan(0, static_cast<uint64_t>(n_qt) * bh, sms);
+  std::vector<int> cands{all};
+  // Splitting only pays where every CTA walks many key tiles: the cost ratio was measured
+  // on 24 - 94 tiles, and at 6 tiles (16 clips of 60 s) a split ran 11 % slower than all
+  // pairs. Shorter clips choose between none and all.
+  if (n_qt >= kMinSplitTiles)
+    for (uint64_t w = 1; w * sms <= static_cast<uint64_t>(all) * bh; ++w)
+      cands.push_back(static_cast<int>(w * sms / bh));
+  for (int P : cands) {
+    if (P <= 0 || static_cast<uint64_t>(P) * bh < 120) continue;  // too few CTAs to pair tiles
+    const int rest = n_qt - 2 * P > 0 ? n_qt - 2 * P : 0;
+    const double t = makespan(static_cast<uint64_t>(P) * bh, static_cast<uint64_t>(rest) * bh, sms);
+    if (t < best_t - 1e-9) {
+      best_t = t;
+      best = P;
+    }
+  }
+  std::lock_guard<std::mutex> lk(mu);
+  cache[key] = best;
+  return best;
+}
+
 }  // namespace
 
 sal_status attention_launch_heads(const void* q, const void* k, const void* v, int batch, int64_t T,
@@ -703,27 +770,35 @@ sal_status attention_launch_heads(const void* q, const void* k, const void* v, i
                    cudaSuccess
                ? SAL_OK
                : SAL_ECUDA;
-  // Pick the kernel by waves of CTAs over the SMs: a two-tile CTA costs about 1.6 one-tile
-  // CTAs (measured), so it wins unless its coarser grain leaves a mostly empty last wave.
+  // Split the query tiles between the kernels: the two-tile kernel takes the first P pairs
+  // of every (clip, head), the one-tile kernel the rest, launched right behind it so its
+  // CTAs fill the SMs that two-tile CTAs leave. P is chosen by list scheduling (below).
   int sms = 148;
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  const uint64_t ctas_pp = static_cast<uint64_t>((T + 2 * kTile - 1) / (2 * kTile)) * bh;
-  const uint64_t ctas_1 = static_cast<uint64_t>((T + kTile - 1) / kTile) * bh;
-  const double waves_pp = static_cast<double>((ctas_pp + sms - 1) / sms) * 1.6;
-  const double waves_1 = static_cast<double>((ctas_1 + sms - 1) / sms);
+  const int n_qt = static_cast<int>((T + kTile - 1) / kTile);
   bool pp_ok = false;
   {
     std::lock_guard<std::mutex> lk(g_mu);
     pp_ok = dev >= 0 && dev < 64 && g_pp_ok[dev];
   }
   const int mode = attention_pp_mode();
-  if (pp_ok && mode != 0 && (mode == 1 || (ctas_pp >= 120 && waves_pp < waves_1))) {
-    const dim3 grid(static_cast<unsigned>((T + 2 * kTile - 1) / (2 * kTile)), static_cast<unsigned>(bh));
-    return launch_kernel(attention_pp_kernel, grid, dim3(kThreadsPP), kSmemPP, s, tq, tk, tv, a) == cudaSuccess
-               ? SAL_OK
-               : SAL_ECUDA;
+  int P = 0;  // query-tile pairs per (clip, head) for the two-tile kernel
+  if (pp_ok && mode == 1) {
+    P = (n_qt + 1) / 2;
+  } else if (pp_ok && mode != 0) {
+    P = choose_pairs(n_qt, bh, sms);
   }
-  return launch_kernel(attention_kernel<128>, grid1, dim3(192), smem_one_tile(128), s, tq, tk, tv, a) ==
+  const int pp_tiles = 2 * P < n_qt ? 2 * P : n_qt;
+  if (P > 0) {
+    const dim3 grid(static_cast<unsigned>(P), static_cast<unsigned>(bh));
+    if (launch_kernel(attention_pp_kernel, grid, dim3(kThreadsPP), kSmemPP, s, tq, tk, tv, a) != cudaSuccess)
+      return SAL_ECUDA;
+  }
+  if (pp_tiles == n_qt) return SAL_OK;
+  a.qt0 = pp_tiles;
+  a.tail = P > 0 ? 1 : 0;
+  const dim3 grid_rest(static_cast<unsigned>(n_qt - pp_tiles), static_cast<unsigned>(bh));
+  return launch_kernel(attention_kernel<128>, grid_rest, dim3(192), smem_one_tile(128), s, tq, tk, tv, a) ==
                  cudaSuccess
              ? SAL_OK
              : SAL_ECUDA;
