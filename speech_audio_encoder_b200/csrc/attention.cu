@@ -743,7 +743,8 @@ sal_status attention_launch_heads(const void* q, const void* k, const void* v, i
                                static_cast<int>(kSmemPP)) != cudaSuccess)
         return SAL_ECUDA;
       // setmaxnreg.inc waits until the registers it asks for are free: run the kernel only
-      // if what warpgroup 0 gives back covers what the softmax warpgroups take
+      // if what warpgroup 0 gives back covers what the softmax warpgroups take (and the
+      // launch count is one that 384 threads can get at all: at most 168)
       cudaFuncAttributes fa{};
       if (cudaFuncGetAttributes(&fa, attention_pp_kernel) != cudaSuccess) return SAL_ECUDA;
       g_pp_ok[dev] = fa.numRegs * kThreadsPP >= kRegsNeededPP && fa.numRegs <= 168;
