@@ -1,0 +1,39 @@
+"""The measurement arithmetic of bench.py against closed forms: algorithmic flops per
+position and layer (two-matrix FFN, width 1280), attention flops 4 T^2 d per layer and clip,
+the front end's algorithmic bytes, and the workload totals the baseline notes quote
+(0.494 TFLOP at 30 s, 388.5 TFLOP at one hour)."""
+import bench
+import oracle as O
+
+
+def test_per_unit_flops():
+    assert bench.GEMM_FLOPS_PER_POS_LAYER == 2 * (4 * 1280 ** 2 + 2 * 1280 * 5120) == 39_321_600
+    assert bench.ATTN_FLOPS_PER_T2_LAYER == 4 * 1280 == 5120
+    assert bench.STACK_PROJ_FLOPS_PER_POS == 2 * 1024 * 1280
+
+
+def test_kernel_flops_sum_to_the_layer():
+    B, T = 2, 700
+    gemm = sum(bench.kernel_flops(k, B, T) for k in ("qkv", "out_proj", "ffn_up", "ffn_down"))
+    assert gemm == bench.GEMM_FLOPS_PER_POS_LAYER * B * T
+    assert bench.kernel_flops("attention", B, T) == 4 * T * T * 1280 * B
+
+
+def test_chunked_attention_pairs():
+    assert bench.attention_pairs(1000, 0) == 1000 ** 2
+    assert bench.attention_pairs(1000, 375) == 2 * 375 ** 2 + 250 ** 2
+    assert bench.attention_pairs(1000, 5000) == 1000 ** 2
+
+
+def test_workload_totals():
+    t30 = O.position_count(480_000)
+    t1h = O.position_count(57_600_000)
+    assert abs(bench.workload_flops(1, t30, 32) / 1e12 - 0.494) < 0.001
+    assert abs(bench.workload_flops(1, t1h, 32) / 1e12 - 388.5) < 0.1
+
+
+def test_frontend_bytes():
+    # one hour: 57.6 M samples read, 359,998 fp32 log-mel rows, 44,999 bf16 stacked rows
+    assert bench.frontend_bytes(1, 57_600_000) == 4 * 57_600_000 + 512 * 359_998 + 2048 * 44_999
+    assert bench.frontend_bytes(3, 16_000) == 3 * (4 * 16_000 + 512 * 98 + 2048 * 12)
+    assert bench.frontend_bytes(1, 399) == 4 * 399
