@@ -354,7 +354,10 @@ def encoder_layer_rows(x, lw, rows, dims: EncoderDims = DIMS):
 
 
 def chunk_bounds(T: int, chunk: int):
-    """[(start, end)] of consecutive chunks of ``chunk`` positions; the last may be shorter."""
+    """[(start, end)] of consecutive chunks of ``chunk`` positions (``chunk`` <= 0: one chunk,
+    the whole clip); the last may be shorter; an empty clip has none."""
+    if T <= 0:
+        return []
     chunk = T if chunk <= 0 else chunk
     return [(s, min(s + chunk, T)) for s in range(0, T, chunk)]
 
