@@ -316,6 +316,15 @@ sal_status sal_ctc_adapter(const void* h, int batch, int64_t T, const sal_ctc_we
 sal_status sal_attention_heads(const void* q, const void* k, const void* v, int batch, int64_t T, int heads,
                                int head_dim, void* o, void* stream);
 
+/* The kernels sal_attention would launch for 128-wide heads on a GPU with `sms` SMs:
+ * *pairs query-tile pairs (of 128 rows) per (clip, head) go to the two-tile kernel and the
+ * remaining of the *query_tiles tiles to the one-tile kernel launched behind it. P is the
+ * count among none, all and the largest filling whole waves whose greedy schedule ends
+ * first (a two-tile CTA counted as 1.55 one-tile CTAs); splits are tried from 16 query
+ * tiles up. SAL_ATTN_PP=0/1 in the environment forces none/all. Host arithmetic only: no
+ * device is needed. *pairs is 0 for head_dim 64 (one-tile kernel only). */
+sal_status sal_attention_plan(int batch, int64_t T, int heads, int head_dim, int sms, int* pairs, int* query_tiles);
+
 /* Row log-softmax (the adapter's last step): out[r, i] = z[r, i] - log sum_j exp z[r, j]
  * for i < n. z rows are ld floats apart (ld >= n), out rows n floats apart; float32. */
 sal_status sal_log_softmax(const float* z, int64_t rows, int n, int64_t ld, float* out, void* stream);

@@ -106,6 +106,8 @@ EXPORTS = {
                                             ctypes.c_void_p]),
     "sal_log_softmax": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_int64,
                                         ctypes.c_void_p, ctypes.c_void_p]),
+    "sal_attention_plan": (ctypes.c_int, [ctypes.c_int, ctypes.c_int64, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                           ctypes.POINTER(ctypes.c_int), ctypes.POINTER(ctypes.c_int)]),
     "sal_ctc_workspace_bytes": (ctypes.c_size_t, [ctypes.c_int, ctypes.c_int64]),
     "sal_ctc_adapter": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int, ctypes.c_int64,
                                         ctypes.POINTER(sal_ctc_weights), ctypes.c_void_p, ctypes.c_void_p,
@@ -459,3 +461,11 @@ def sal_log_softmax(z: torch.Tensor, n: int | None = None, stream=None) -> torch
     out = torch.empty((rows, n), dtype=torch.float32, device=z.device)
     _check("sal_log_softmax", lib().sal_log_softmax(_ptr(z), rows, n, ld, _ptr(out), _stream(stream)))
     return out
+
+
+def attention_plan(batch: int, T: int, heads: int = 10, head_dim: int = 128, sms: int = 148) -> tuple[int, int]:
+    """(pairs for the two-tile kernel, query tiles per clip) that sal_attention would use."""
+    p, q = ctypes.c_int(), ctypes.c_int()
+    _check("sal_attention_plan", lib().sal_attention_plan(batch, T, heads, head_dim, sms, ctypes.byref(p),
+                                                          ctypes.byref(q)))
+    return p.value, q.value

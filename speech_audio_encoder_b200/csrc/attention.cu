@@ -811,3 +811,23 @@ sal_status attention_launch(const void* q, const void* k, const void* v, int bat
 }
 
 }  // namespace sal
+
+// The split attention_launch_heads makes for 128-wide heads when the two-tile kernel is
+// available (host arithmetic only; no device is touched).
+extern "C" sal_status sal_attention_plan(int batch, int64_t T, int heads, int head_dim, int sms, int* pairs,
+                                         int* query_tiles) {
+  using namespace sal;
+  if (batch < 0 || T < 0 || heads < 0 || sms <= 0 || !pairs || !query_tiles) return SAL_EINVAL;
+  const int n_qt = static_cast<int>((T + kTile - 1) / kTile);
+  *query_tiles = n_qt;
+  *pairs = 0;
+  if (head_dim != 128 || batch == 0 || T == 0 || heads == 0) return SAL_OK;
+  const uint64_t bh = static_cast<uint64_t>(batch) * heads;
+  const int mode = attention_pp_mode();
+  *pairs = mode == 0 ? 0 : (mode == 1 ? (n_qt + 1) / 2 : choose_pairs(n_qt, bh, sms));
+  return SAL_OK;
+}
+
+namespace sal {
+
+}  // namespace sal

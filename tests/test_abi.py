@@ -88,3 +88,16 @@ def test_ctc_adapter_host_checks(api):
     assert lib.sal_attention_heads(0, 0, 0, 1, 10, 16, 64, 0, 0) == 1
     assert lib.sal_log_softmax(0, 4, 10, 5, 0, 0) == 1                             # ld < n
     assert lib.sal_log_softmax(0, 0, 10, 10, 0, 0) == 0
+
+
+def test_attention_plan_matches_the_stated_schedule(api):
+    """The library's split of query tiles between the two attention kernels equals the
+    rule its header states (list scheduling, written out in the GPU tests), over clip
+    lengths and batch sizes on both sides of every threshold."""
+    from test_gpu_kernels import _pairs_for_two_tile_kernel
+    cases = [(b, T) for b in (1, 2, 8, 16, 30) for T in (1, 129, 749, 1000, 2000, 2047, 2048, 3000)]
+    cases += [(b, T) for b in (1, 2) for T in (5000, 7499, 12000, 20000, 44999)]
+    for batch, T in cases:
+        assert api.attention_plan(batch, T) == _pairs_for_two_tile_kernel(batch, T), (batch, T)
+    assert api.attention_plan(1, 20000, heads=16, head_dim=64) == (0, 157)  # 64-wide heads: one-tile
+    assert api.attention_plan(0, 100) == (0, 1)

@@ -168,8 +168,8 @@ def _pairs_for_two_tile_kernel(batch, T, sms=148, rho=1.55):
 def test_attention(batch, T, scale):
     api = _api()
     expect = {(30, 129): (1, 2), (1, 3000): (12, 24), (8, 1000): (4, 8), (16, 749): (3, 6), (1, 5000): (14, 40)}
-    P, n_qt = _pairs_for_two_tile_kernel(batch, T)
-    assert (P, n_qt) == expect.get((batch, T), (0, n_qt))
+    n_qt = -(-T // 128)
+    assert api.attention_plan(batch, T) == expect.get((batch, T), (0, n_qt))
     q, q64 = rand_bf16((batch, 10, T, 128), 50 + T, scale)
     k, k64 = rand_bf16((batch, 10, T, 128), 60 + T, 1.0)
     v, v64 = rand_bf16((batch, 10, T, 128), 70 + T, 1.0)
