@@ -206,7 +206,7 @@ typedef enum {
 } sal_epilogue;
 
 /* Linear layer on the tensor cores: A [M, K] bf16 (row-major), W [N, K] bf16, bias [N]
- * bf16. K must be a multiple of 64 and N of 64 (N of 128 when M > 512). */
+ * bf16. K and N must be multiples of 64 (SAL_ESHAPE otherwise). */
 sal_status sal_linear(int epilogue, const void* A, int64_t M, int K, const void* W, int N,
                       const void* bias, void* out, void* stream);
 
