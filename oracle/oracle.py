@@ -3,9 +3,12 @@
 TEST INFRASTRUCTURE. Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline
 legs of ``bench.py`` may call this module. The product path never routes through it.
 
-Every function is the plain definition of one step, written in numpy float64. Library
-primitives (matrix product, ``erf``) are used as single steps; there is no blocking or
-reordering beyond chunking over independent frames or query rows to bound memory.
+The arithmetic is the plain C++ of ``sal_oracle.cpp`` (``liboracle.so``, textbook loops in
+double precision: an explicit DFT sum, explicit Slaney mel rows, triple-loop matrix
+products, two-pass LayerNorm, max-subtracted softmax, ``std::erf`` GELU and fp64 RoPE).
+This module marshals numpy arrays to it and composes its steps in the page's order;
+integer bookkeeping (frame counts, chunk and window bounds, parameter counts) is written
+here directly.
 
 Sources (all on the page "Nemotron 3.5 Transcribe: From Recorded Speech to Dataset
 Audits", flozi.net):
@@ -30,6 +33,11 @@ Audits", flozi.net):
 * [CHUNK] section "Local encoder windows, recording-wide language context": in training the
   encoder runs on independent 30-second post-feature chunks with no attention across
   their borders, and the chunk outputs are concatenated in order; pairs scale as T w.
+* [WINDOW] section "Local encoder windows, recording-wide language context", the
+  paragraph on the serving path: the encoder runs on context-extended windows, the outputs
+  at overlap (context) positions are discarded and the core outputs concatenated; the
+  defaults are 500 encoded core positions with 50 context positions on each side (80 ms
+  per position). Edge handling is not given; reading 22 below.
 * [CTC]   section "Use alignment and audio questions as supporting evidence": a CTC
   timestamp adapter of about 50M parameters takes the unfused ASR states (width 1,280),
   upsamples their 80 ms grid to 40 ms with a stride-two transposed convolution, runs two
@@ -73,14 +81,23 @@ Readings where the pages are silent (each one is listed in the design notes):
     bias and 23,863 outputs, the blank last.
 21. the adapter's output is the frame log-probabilities, log_softmax over the 23,863
     classes.
+22. serving windows: the cores are consecutive runs of ``core`` positions from the clip
+    start (the last may be shorter); a window is its core extended by ``context``
+    positions on each side, clipped to the clip, so the first window has no left context
+    and the last no right context beyond the clip end. Each window is encoded as an
+    independent sequence (all layers and the final LayerNorm, attention inside the window,
+    RoPE positions from 0 at the window start); its core outputs are kept in order.
 """
 from __future__ import annotations
 
+import ctypes
 import math
+import os
+import subprocess
+import threading
 from dataclasses import dataclass
 
 import numpy as np
-from scipy.special import erf as _erf
 
 SAMPLE_RATE = 16000  # [ARCH]
 WIN = 400            # 25 ms at 16 kHz [ARCH]
@@ -89,13 +106,13 @@ NFFT = 512           # [ARCH]
 NBINS = NFFT // 2 + 1
 NMEL = 128           # [ARCH]
 STACK = 8            # [ARCH]
-MEL_FMIN = 0.0       # reading 4
-MEL_FMAX = 8000.0    # reading 4
 LOG_FLOOR = 1e-10    # reading 5
 LN_EPS = 1e-5        # reading 8
 QK_EPS = 1e-6        # reading 9
 ROPE_BASE = 10000.0  # reading 10
 MAX_POSITIONS = 45000  # one hour at 12.5 positions/s [POS]
+WINDOW_CORE = 500      # serving window core positions [WINDOW]
+WINDOW_CONTEXT = 50    # serving window context positions on each side [WINDOW]
 N_SLOTS = 8            # speaker slots [FUSE]
 LLM_WIDTH = 2688       # language width [FUSE]
 
@@ -108,11 +125,95 @@ __all__ = [
     "rope", "attention_probs", "attention", "gelu", "encoder_layer",
     "encoder_layer_rows", "encoder_forward", "stack_project", "encode",
     "param_count", "rel_l2", "chunk_bounds", "encoder_layer_chunked",
-    "encoder_layer_rows_chunked", "encoder_forward_chunked", "N_SLOTS", "LLM_WIDTH",
+    "encoder_layer_rows_chunked", "encoder_forward_chunked", "window_bounds",
+    "encoder_forward_windowed", "WINDOW_CORE", "WINDOW_CONTEXT", "N_SLOTS", "LLM_WIDTH",
     "speaker_kernel", "speaker_fuse", "connector", "CtcDims", "CTC", "ctc_upsample",
-    "log_softmax", "ctc_logits", "ctc_adapter", "ctc_param_count",
+    "log_softmax", "ctc_logits", "ctc_adapter", "ctc_param_count", "threads", "LIB_PATH",
 ]
 
+# ----------------------------------------------------------------------------- the C++ library
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+SOURCE = os.path.join(_HERE, "sal_oracle.cpp")
+LIB_PATH = os.path.join(_HERE, "liboracle.so")
+# x86-64-v3 (AVX2, FMA): a target every current server CPU runs, here and on other hosts
+CXX_FLAGS = ["-O3", "-march=x86-64-v3", "-fopenmp", "-fPIC", "-shared", "-std=c++17"]
+
+_lib = None
+_lock = threading.Lock()
+
+
+def build(force: bool = False) -> str:
+    """Compile liboracle.so next to its source with g++ (when missing or older)."""
+    if not force and os.path.exists(LIB_PATH) and os.path.getmtime(LIB_PATH) >= os.path.getmtime(SOURCE):
+        return LIB_PATH
+    tmp = LIB_PATH + f".{os.getpid()}.tmp"
+    r = subprocess.run(["g++", *CXX_FLAGS, SOURCE, "-o", tmp], capture_output=True, text=True)
+    if r.returncode != 0:
+        raise RuntimeError(f"building the oracle failed:\n{r.stdout}\n{r.stderr}")
+    os.replace(tmp, LIB_PATH)
+    return LIB_PATH
+
+
+_D = ctypes.POINTER(ctypes.c_double)
+_I64 = ctypes.c_int64
+
+
+class _Layer(ctypes.Structure):
+    _fields_ = [(n, _D) for n in ("ln1_g", "ln1_b", "w_qkv", "b_qkv", "qn_g", "kn_g", "w_o", "b_o",
+                                  "ln2_g", "ln2_b", "w1", "b1", "w2", "b2")]
+
+
+_SIGS = {
+    "oc_threads": (ctypes.c_int, []),
+    "oc_frame_count": (_I64, [_I64]),
+    "oc_hann": (None, [_D]),
+    "oc_hz_to_mel": (ctypes.c_double, [ctypes.c_double]),
+    "oc_mel_to_hz": (ctypes.c_double, [ctypes.c_double]),
+    "oc_mel_filterbank": (None, [_D]),
+    "oc_linear": (None, [_D, _I64, _I64, _D, _I64, _D, _D]),
+    "oc_power_spectrum": (None, [_D, _I64, _I64, _D]),
+    "oc_log_mel": (None, [ctypes.POINTER(ctypes.c_float), _I64, _I64, _I64, _D]),
+    "oc_layer_norm": (None, [_D, _I64, _I64, _D, _D, ctypes.c_double, _D]),
+    "oc_rms_norm": (None, [_D, _I64, _I64, _D, ctypes.c_double, _D]),
+    "oc_rope": (None, [_D, _I64, _I64, _D, _D]),
+    "oc_attention_probs": (None, [_D, _I64, _D, _I64, _I64, _D]),
+    "oc_attention": (None, [_D, _I64, _I64, _D, _D, _I64, _I64, _D]),
+    "oc_gelu": (None, [_D, _I64, _D]),
+    "oc_encoder_layer_rows": (None, [_D, _I64, _I64, _I64, _I64, _I64, ctypes.POINTER(_Layer),
+                                     ctypes.POINTER(_I64), _I64, _D]),
+    "oc_speaker_kernel": (None, [_I64, _I64, _D]),
+    "oc_log_softmax": (None, [_D, _I64, _I64, _D]),
+}
+
+
+def _load():
+    global _lib
+    with _lock:
+        if _lib is None:
+            l = ctypes.CDLL(build())
+            for name, (res, args) in _SIGS.items():
+                f = getattr(l, name)
+                f.restype = res
+                f.argtypes = args
+            _lib = l
+    return _lib
+
+
+def threads() -> int:
+    """Threads the C++ oracle runs on (OpenMP)."""
+    return _load().oc_threads()
+
+
+def _f64(a) -> np.ndarray:
+    return np.ascontiguousarray(a, dtype=np.float64)
+
+
+def _p(a: np.ndarray):
+    return a.ctypes.data_as(_D)
+
+
+# ----------------------------------------------------------------------------- counts
 
 @dataclass(frozen=True)
 class EncoderDims:
@@ -126,8 +227,6 @@ class EncoderDims:
 
 DIMS = EncoderDims()
 
-
-# ----------------------------------------------------------------------------- counts
 
 def frame_count(n_samples: int) -> int:
     """Number of 400-sample frames at a 160-sample hop (reading 1, [ARCH])."""
@@ -144,8 +243,9 @@ def position_count(n_samples: int) -> int:
 
 def hann_window() -> np.ndarray:
     """Periodic Hann window of length 400 (reading 2)."""
-    n = np.arange(WIN, dtype=np.float64)
-    return 0.5 - 0.5 * np.cos(2.0 * math.pi * n / WIN)
+    w = np.empty(WIN)
+    _load().oc_hann(_p(w))
+    return w
 
 
 def frame_signal(wave: np.ndarray, first: int = 0, count: int | None = None) -> np.ndarray:
@@ -159,46 +259,32 @@ def frame_signal(wave: np.ndarray, first: int = 0, count: int | None = None) -> 
 
 
 def power_spectrum(y: np.ndarray) -> np.ndarray:
-    """|X_k|^2 for k = 0..256 of frames zero-padded to 512 samples (reading 3).
-
-    The DFT is the explicit sum X_k = sum_n y[n] exp(-2 pi i k n / 512); the zero padding
-    contributes nothing, so the sum runs over the frame's own samples.
-    """
-    y = np.asarray(y, dtype=np.float64)
-    n = np.arange(y.shape[-1], dtype=np.float64)[:, None]
-    k = np.arange(NBINS, dtype=np.float64)[None, :]
-    ang = 2.0 * math.pi * ((k * n) % NFFT) / NFFT
-    re = y @ np.cos(ang)
-    im = -(y @ np.sin(ang))
-    return re * re + im * im
+    """|X_k|^2 for k = 0..256 of frames zero-padded to 512 samples (reading 3), by the
+    explicit DFT sum over the frame's own samples."""
+    y = _f64(y)
+    shape = y.shape[:-1]
+    y2 = y.reshape(-1, y.shape[-1])
+    P = np.empty((y2.shape[0], NBINS))
+    _load().oc_power_spectrum(_p(y2), y2.shape[0], y2.shape[1], _p(P))
+    return P.reshape(shape + (NBINS,))
 
 
 def hz_to_mel(f):
     """Slaney mel scale: linear 3 f / 200 below 1 kHz, logarithmic above (reading 4)."""
-    f = np.asarray(f, dtype=np.float64)
-    lin = f * 3.0 / 200.0
-    logstep = math.log(6.4) / 27.0
-    with np.errstate(divide="ignore"):
-        lg = 15.0 + np.log(np.maximum(f, 1e-300) / 1000.0) / logstep
-    return np.where(f >= 1000.0, lg, lin)
+    l = _load()
+    return np.vectorize(l.oc_hz_to_mel, otypes=[np.float64])(np.asarray(f, dtype=np.float64))
 
 
 def mel_to_hz(m):
     """Inverse of :func:`hz_to_mel`."""
-    m = np.asarray(m, dtype=np.float64)
-    logstep = math.log(6.4) / 27.0
-    return np.where(m >= 15.0, 1000.0 * np.exp(logstep * (m - 15.0)), m * 200.0 / 3.0)
+    l = _load()
+    return np.vectorize(l.oc_mel_to_hz, otypes=[np.float64])(np.asarray(m, dtype=np.float64))
 
 
 def mel_filterbank() -> np.ndarray:
     """128 x 257 Slaney-normalised triangular filters over 0..8 kHz (reading 4)."""
-    pts = mel_to_hz(np.linspace(hz_to_mel(MEL_FMIN), hz_to_mel(MEL_FMAX), NMEL + 2))
-    fk = np.arange(NBINS, dtype=np.float64) * SAMPLE_RATE / NFFT
-    W = np.zeros((NMEL, NBINS), dtype=np.float64)
-    for m in range(NMEL):
-        rise = (fk - pts[m]) / (pts[m + 1] - pts[m])
-        fall = (pts[m + 2] - fk) / (pts[m + 2] - pts[m + 1])
-        W[m] = np.maximum(0.0, np.minimum(rise, fall)) * (2.0 / (pts[m + 2] - pts[m]))
+    W = np.empty((NMEL, NBINS))
+    _load().oc_mel_filterbank(_p(W))
     return W
 
 
@@ -207,18 +293,18 @@ def log_mel(wave: np.ndarray, chunk: int = 8192, first: int = 0,
     """[F, 128] natural-log mel energies of one clip ([ARCH], readings 1-5).
 
     ``first``/``count`` select a range of frames; frames are independent, so the range
-    is only a way to sample long clips.
+    is only a way to sample long clips. (``chunk`` is kept for callers; the C++ side
+    takes frames 8,192 at a time.)
     """
-    x = np.asarray(wave, dtype=np.float32)
+    x = np.ascontiguousarray(wave, dtype=np.float32)
     F = frame_count(x.shape[0])
     if count is None:
         count = F - first
-    W = mel_filterbank()
-    out = np.empty((count, NMEL), dtype=np.float64)
-    for s in range(0, count, chunk):
-        c = min(chunk, count - s)
-        P = power_spectrum(frame_signal(x, first + s, c))
-        out[s:s + c] = np.log(np.maximum(P @ W.T, LOG_FLOOR))
+    if first < 0 or count < 0 or first + count > F:
+        raise ValueError("frame range outside the clip")
+    out = np.empty((count, NMEL))
+    if count:
+        _load().oc_log_mel(x.ctypes.data_as(ctypes.POINTER(ctypes.c_float)), x.shape[0], first, count, _p(out))
     return out
 
 
@@ -234,28 +320,34 @@ def stack_frames(logmel: np.ndarray) -> np.ndarray:
 
 # ----------------------------------------------------------------------------- encoder pieces
 
-def _f64(a):
-    return np.asarray(a, dtype=np.float64)
-
-
 def linear(x, w, b):
     """x W^T + b with W stored [out, in] (reading 7)."""
-    return _f64(x) @ _f64(w).T + _f64(b)
+    x, w = _f64(x), _f64(w)
+    lead = x.shape[:-1]
+    x2 = x.reshape(-1, x.shape[-1])
+    out = np.empty((x2.shape[0], w.shape[0]))
+    bb = None if b is None else _f64(b)
+    _load().oc_linear(_p(x2), x2.shape[0], x2.shape[1], _p(w), w.shape[0], None if bb is None else _p(bb), _p(out))
+    return out.reshape(lead + (w.shape[0],))
 
 
 def layer_norm(x, g, b, eps: float = LN_EPS):
     """Per-row LayerNorm with two-pass mean and variance (reading 8)."""
     x = _f64(x)
-    mu = x.mean(axis=-1, keepdims=True)
-    d = x - mu
-    var = (d * d).mean(axis=-1, keepdims=True)
-    return d / np.sqrt(var + eps) * _f64(g) + _f64(b)
+    x2 = x.reshape(-1, x.shape[-1])
+    y = np.empty_like(x2)
+    _load().oc_layer_norm(_p(x2), x2.shape[0], x2.shape[1], _p(_f64(np.broadcast_to(g, x.shape[-1:]))),
+                          _p(_f64(np.broadcast_to(b, x.shape[-1:]))), eps, _p(y))
+    return y.reshape(x.shape)
 
 
 def rms_norm(x, g, eps: float = QK_EPS):
     """x / sqrt(mean(x^2) + eps) * g over the last axis (reading 9)."""
     x = _f64(x)
-    return x / np.sqrt((x * x).mean(axis=-1, keepdims=True) + eps) * _f64(g)
+    x2 = x.reshape(-1, x.shape[-1])
+    y = np.empty_like(x2)
+    _load().oc_rms_norm(_p(x2), x2.shape[0], x2.shape[1], _p(_f64(np.broadcast_to(g, x.shape[-1:]))), eps, _p(y))
+    return y.reshape(x.shape)
 
 
 def rope_angles(positions, head_dim: int):
@@ -268,89 +360,67 @@ def rope_angles(positions, head_dim: int):
 def rope(x, positions):
     """Rotate the pairs (i, i + hd/2) of x [..., T, hd] by the angles of ``positions``."""
     x = _f64(x)
-    hd = x.shape[-1]
-    half = hd // 2
-    ang = rope_angles(positions, hd)
-    c, s = np.cos(ang), np.sin(ang)
-    a, b = x[..., :half], x[..., half:]
-    return np.concatenate([a * c - b * s, b * c + a * s], axis=-1)
+    T, hd = x.shape[-2], x.shape[-1]
+    pos = _f64(positions)
+    x3 = x.reshape(-1, T, hd)
+    y = np.empty_like(x3)
+    for i in range(x3.shape[0]):
+        _load().oc_rope(_p(np.ascontiguousarray(x3[i])), T, hd, _p(pos), _p(y[i]))
+    return y.reshape(x.shape)
 
 
 def attention_probs(q, k):
     """softmax(q k^T / sqrt(hd)) over keys, with the row maximum subtracted (reading 11)."""
     q, k = _f64(q), _f64(k)
-    s = q @ k.T / math.sqrt(q.shape[-1])
-    s = s - s.max(axis=-1, keepdims=True)
-    e = np.exp(s)
-    return e / e.sum(axis=-1, keepdims=True)
+    P = np.empty((q.shape[0], k.shape[0]))
+    _load().oc_attention_probs(_p(q), q.shape[0], _p(k), k.shape[0], q.shape[1], _p(P))
+    return P
 
 
 def attention(q, k, v, chunk: int = 2048):
     """Per head: softmax(q k^T / sqrt(hd)) v. q [H, Tq, hd], k and v [H, Tk, hd].
-
-    Query rows are independent, so they are taken ``chunk`` at a time to bound memory.
-    """
+    (``chunk`` is kept for callers; the C++ side walks query rows one at a time.)"""
     q, k, v = _f64(q), _f64(k), _f64(v)
-    out = np.empty(q.shape[:-1] + (v.shape[-1],), dtype=np.float64)
-    for h in range(q.shape[0]):
-        for s in range(0, q.shape[1], chunk):
-            out[h, s:s + chunk] = attention_probs(q[h, s:s + chunk], k[h]) @ v[h]
+    out = np.empty(q.shape[:-1] + (v.shape[-1],))
+    _load().oc_attention(_p(q), q.shape[0], q.shape[1], _p(k), _p(v), k.shape[1], q.shape[2], _p(out))
     return out
 
 
 def gelu(x):
     """Exact GELU 0.5 x (1 + erf(x / sqrt 2)) (reading 12)."""
     x = _f64(x)
-    return 0.5 * x * (1.0 + _erf(x / math.sqrt(2.0)))
+    y = np.empty_like(x)
+    _load().oc_gelu(_p(x), x.size, _p(y))
+    return y
 
 
-def _split_heads(y, dims: EncoderDims):
-    # y [T, width] -> [heads, T, head_dim]
-    return y.reshape(y.shape[0], dims.heads, dims.head_dim).transpose(1, 0, 2)
-
-
-def _qkv(h, lw, dims: EncoderDims, positions):
-    """Q, K, V [heads, T, hd] after QK normalisation and RoPE (readings 9, 10)."""
-    qkv = linear(h, lw["w_qkv"], lw["b_qkv"])
-    W = dims.width
-    q = _split_heads(qkv[:, :W], dims)
-    k = _split_heads(qkv[:, W:2 * W], dims)
-    v = _split_heads(qkv[:, 2 * W:], dims)
-    q = rope(rms_norm(q, lw["qn_g"]), positions)
-    k = rope(rms_norm(k, lw["kn_g"]), positions)
-    return q, k, v
-
-
-def encoder_layer(x, lw, dims: EncoderDims = DIMS):
-    """One pre-norm bidirectional Transformer layer on one clip x [T, width] ([ARCH]).
-
-    x + Attn(LN1(x)), then + FFN(LN2(.)), with the attention over all T positions.
-    """
-    x = _f64(x)
-    T = x.shape[0]
-    q, k, v = _qkv(layer_norm(x, lw["ln1_g"], lw["ln1_b"]), lw, dims, np.arange(T))
-    o = attention(q, k, v).transpose(1, 0, 2).reshape(T, dims.width)
-    x = x + linear(o, lw["w_o"], lw["b_o"])
-    u = gelu(linear(layer_norm(x, lw["ln2_g"], lw["ln2_b"]), lw["w1"], lw["b1"]))
-    return x + linear(u, lw["w2"], lw["b2"])
+_LAYER_KEYS = ("ln1_g", "ln1_b", "w_qkv", "b_qkv", "qn_g", "kn_g", "w_o", "b_o",
+               "ln2_g", "ln2_b", "w1", "b1", "w2", "b2")
 
 
 def encoder_layer_rows(x, lw, rows, dims: EncoderDims = DIMS):
-    """:func:`encoder_layer` evaluated only at the positions ``rows`` of one clip.
-
-    Keys and values still come from every position; everything after attention is
-    per position, so the selected rows equal the same rows of the full layer.
-    """
+    """One pre-norm bidirectional Transformer layer on one clip x [T, width] ([ARCH]),
+    evaluated only at the positions ``rows``: x + Attn(LN1(x)), then + FFN(LN2(.)), with
+    keys and values from every position (so the rows equal the same rows of the full
+    layer)."""
     x = _f64(x)
-    rows = np.asarray(rows)
+    rows = np.ascontiguousarray(rows, dtype=np.int64)
     T = x.shape[0]
-    h = layer_norm(x, lw["ln1_g"], lw["ln1_b"])
-    _, k, v = _qkv(h, lw, dims, np.arange(T))
-    q, _, _ = _qkv(h[rows], lw, dims, rows)
-    o = attention(q, k, v).transpose(1, 0, 2).reshape(len(rows), dims.width)
-    xr = x[rows] + linear(o, lw["w_o"], lw["b_o"])
-    u = gelu(linear(layer_norm(xr, lw["ln2_g"], lw["ln2_b"]), lw["w1"], lw["b1"]))
-    return xr + linear(u, lw["w2"], lw["b2"])
+    if rows.size and (rows.min() < 0 or rows.max() >= T):
+        raise IndexError("row outside the clip")
+    keep = {k: _f64(lw[k]) for k in _LAYER_KEYS}
+    L = _Layer(*[_p(keep[k]) for k in _LAYER_KEYS])
+    out = np.empty((len(rows), dims.width))
+    if len(rows):
+        _load().oc_encoder_layer_rows(_p(x), T, dims.width, dims.heads, dims.head_dim, dims.ffn, ctypes.byref(L),
+                                      rows.ctypes.data_as(ctypes.POINTER(_I64)), len(rows), _p(out))
+    return out
+
+
+def encoder_layer(x, lw, dims: EncoderDims = DIMS):
+    """One pre-norm bidirectional Transformer layer on one clip x [T, width] ([ARCH]),
+    with the attention over all T positions."""
+    return encoder_layer_rows(x, lw, np.arange(_f64(x).shape[0]), dims)
 
 
 def chunk_bounds(T: int, chunk: int):
@@ -389,25 +459,47 @@ def encoder_forward_chunked(x0, weights, n_layers: int, chunk: int, dims: Encode
     return layer_norm(x, weights["lnf_g"], weights["lnf_b"])
 
 
+def window_bounds(T: int, core: int = WINDOW_CORE, context: int = WINDOW_CONTEXT):
+    """[(lo, c0, c1, hi)] per serving window ([WINDOW], reading 22): the core [c0, c1) of
+    ``core`` positions (the last may be shorter) and the window [lo, hi) that extends it by
+    ``context`` positions on each side, clipped to [0, T). An empty clip has none."""
+    out = []
+    for c0 in range(0, max(T, 0), core):
+        c1 = min(c0 + core, T)
+        out.append((max(0, c0 - context), c0, c1, min(T, c1 + context)))
+    return out
+
+
+def encoder_forward_windowed(x0, weights, n_layers: int, core: int = WINDOW_CORE,
+                             context: int = WINDOW_CONTEXT, dims: EncoderDims = DIMS):
+    """Serving-window encoder ([WINDOW], reading 22): every window runs ``n_layers`` layers
+    and the final LayerNorm on its own positions as an independent sequence; the outputs
+    at its context positions are discarded and the core outputs concatenated in order."""
+    x = _f64(x0)
+    parts = [encoder_forward(x[lo:hi], weights, n_layers, dims)[c0 - lo:c1 - lo]
+             for lo, c0, c1, hi in window_bounds(len(x), core, context)]
+    return np.concatenate(parts) if parts else np.empty((0, x.shape[1]))
+
+
 def speaker_kernel(n_slots: int = N_SLOTS, width: int = 1280) -> np.ndarray:
     """Fixed sinusoidal speaker kernel K [n_slots, width] (reading 15)."""
-    s = np.arange(n_slots, dtype=np.float64)[:, None]
-    w = ROPE_BASE ** (-2.0 * np.arange(width // 2, dtype=np.float64) / width)[None, :]
-    K = np.empty((n_slots, width), dtype=np.float64)
-    K[:, 0::2] = np.sin(s * w)
-    K[:, 1::2] = np.cos(s * w)
+    K = np.empty((n_slots, width))
+    _load().oc_speaker_kernel(n_slots, width, _p(K))
     return K
 
 
 def speaker_fuse(H, P, g, b, scale: float = 1.0):
     """H + scale * LN_slots(P > 0.5) K ([FUSE], readings 13-15). H [T, 1280], P [T, 8]."""
     A = (np.asarray(P, dtype=np.float64) > 0.5).astype(np.float64)
-    return _f64(H) + scale * layer_norm(A, g, b) @ speaker_kernel(A.shape[1], H.shape[1])
+    H = _f64(H)
+    K = speaker_kernel(A.shape[1], H.shape[1])
+    return H + scale * linear(layer_norm(A, g, b), np.ascontiguousarray(K.T), None)
 
 
 def connector(x, w, b):
     """The identity connector: one linear projection to the language width ([FUSE], 16)."""
     return linear(x, w, b)
+
 
 # ----------------------------------------------------------------------------- CTC timestamp adapter
 
@@ -437,15 +529,17 @@ def ctc_upsample(h, w_up, b_up):
     h, w = _f64(h), _f64(w_up)
     U = np.empty((2 * h.shape[0], w.shape[1]), dtype=np.float64)
     for j in range(2):
-        U[j::2] = h @ w[j].T + _f64(b_up)
+        U[j::2] = linear(h, w[j], b_up)
     return U
 
 
 def log_softmax(z):
     """log(softmax(z)) over the last axis, with the row maximum subtracted (reading 21)."""
     z = _f64(z)
-    m = z.max(axis=-1, keepdims=True)
-    return z - m - np.log(np.exp(z - m).sum(axis=-1, keepdims=True))
+    z2 = z.reshape(-1, z.shape[-1])
+    y = np.empty_like(z2)
+    _load().oc_log_softmax(_p(z2), z2.shape[0], z2.shape[1], _p(y))
+    return y.reshape(z.shape)
 
 
 def ctc_logits(h, cw, dims: CtcDims = CTC):
@@ -468,7 +562,6 @@ def ctc_param_count(dims: CtcDims = CTC) -> int:
     up = 2 * W * dims.in_width + W
     layers = param_count(dims.layers, dims.layer_dims) - (dims.layer_dims.stack_in * W + W + 2 * W)
     return up + layers + 2 * W + dims.classes * W + dims.classes
-
 
 
 def stack_project(stacked, weights):
