@@ -34,7 +34,7 @@ from speech_audio_encoder_b200 import synth  # noqa: E402
 
 METRIC = "audio-sec encoded/sec (frontend+32-layer encoder, bf16) on 1 B200; % TC peak"
 UNIT = "audio-s/s"
-DEFAULT_WORKLOAD = "clip_30s"
+DEFAULT_WORKLOAD = "rec_1h"  # the largest single-GPU configuration
 FLUSH_BYTES = 256 << 20
 
 GEMM_FLOPS_PER_POS_LAYER = 2 * (4 * 1280 * 1280 + 2 * 1280 * 5120)  # 39,321,600
@@ -60,15 +60,32 @@ def attention_pairs(T: int, chunk: int = 0) -> int:
     return full * chunk * chunk + rest * rest
 
 
-def kernel_flops(kind: str, B: int, T: int, chunk: int = 0) -> float:
+def window_lengths(T: int, core: int, context: int) -> list[int]:
+    """Positions of each serving window of a clip of T positions: its core of ``core``
+    positions (the last may be shorter) and up to ``context`` more on each side."""
+    return [min(T, c0 + core + context) - max(0, c0 - context) for c0 in range(0, T, core)]
+
+
+def layer_work(T: int, chunk: int = 0, window: tuple[int, int] | None = None) -> tuple[int, int]:
+    """(positions a layer processes, query-key pairs of its attention) per clip: T and T^2
+    (or the sum of squared chunk lengths); with serving windows every window's own
+    positions and pairs, context positions included (they are encoded once per window)."""
+    if window:
+        lens = window_lengths(T, *window)
+        return sum(lens), sum(n * n for n in lens)
+    return T, attention_pairs(T, chunk)
+
+
+def kernel_flops(kind: str, B: int, T: int, chunk: int = 0, window=None) -> float:
     """Algorithmic flops of ONE launch of a kernel kind (all clips of the batch)."""
-    M = B * T
+    rows, pairs = layer_work(T, chunk, window)
+    M = B * rows
     return {
         "qkv": 2.0 * M * 1280 * 3840,
         "out_proj": 2.0 * M * 1280 * 1280,
         "ffn_up": 2.0 * M * 1280 * 5120,
         "ffn_down": 2.0 * M * 5120 * 1280,
-        "attention": float(ATTN_FLOPS_PER_T2_LAYER) * attention_pairs(T, chunk) * B,
+        "attention": float(ATTN_FLOPS_PER_T2_LAYER) * pairs * B,
     }.get(kind, 0.0)
 
 
@@ -89,8 +106,9 @@ def frontend_bytes(B: int, N: int) -> float:
     return float(B) * (4 * N + 512 * F + 2048 * T)
 
 
-def workload_flops(B: int, T: int, L: int, chunk: int = 0) -> float:
-    return (GEMM_FLOPS_PER_POS_LAYER * B * T * L + ATTN_FLOPS_PER_T2_LAYER * attention_pairs(T, chunk) * B * L
+def workload_flops(B: int, T: int, L: int, chunk: int = 0, window=None) -> float:
+    rows, pairs = layer_work(T, chunk, window)
+    return (GEMM_FLOPS_PER_POS_LAYER * B * rows * L + ATTN_FLOPS_PER_T2_LAYER * pairs * B * L
             + STACK_PROJ_FLOPS_PER_POS * B * T)
 
 
@@ -194,9 +212,8 @@ def oracle_step_estimate(wl: synth.Workload, budget_s: float, audio: np.ndarray,
     (estimated seconds per step, description, seconds actually spent, threads used).
     """
     import oracle as O
-    from threadpoolctl import threadpool_info
 
-    threads = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+    threads = O.threads()
     t_start = time.perf_counter()
     F, T, B, L = frames(wl.n_samples), positions(wl.n_samples), wl.batch, wl.n_layers
     fe_frames = max(1, min(F, int(4000 * budget_s)))
@@ -260,6 +277,7 @@ def run_reference(args, wl: synth.Workload) -> dict | None:
                    "positions": positions(wl.n_samples), "layers": wl.n_layers,
                    "parallelism": "host cores, rank 0 only"},
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
+                         "cpu_model": _cpu_model(), "nproc": os.cpu_count(),
                          "sample": desc + f"; {args.steps} samples, {spent_total:.1f} s of CPU work"},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
@@ -292,14 +310,16 @@ def run_sal(args, wl: synth.Workload) -> dict | None:
     stacked = torch.empty((B, T, 1024), dtype=torch.bfloat16, device=dev)
     x = torch.empty((B * T, 1280), dtype=torch.float32, device=dev)
     emb = torch.empty((B * T, 1280), dtype=torch.bfloat16, device=dev)
-    ws = api.encoder_workspace(B, T, dev)
+    window = (api.WINDOW_CORE, api.WINDOW_CONTEXT) if args.window else None
+    wcore, wctx = window if window else (0, 0)
+    ws = api.encoder_workspace_ex(B, T, args.chunk, wcore, wctx, dev)
     flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
     lib = api.lib()
     import ctypes
     rec = ctypes.byref(dw.record)
     sp = s.cuda_stream
 
-    opts = api.sal_forward_options(args.chunk, None)
+    opts = api.sal_forward_options(args.chunk, None, wcore, wctx)
 
     def step(stream_ptr=sp):
         api._check("sal_frontend", lib.sal_frontend(wave_d.data_ptr(), N, B, logmel.data_ptr(),
@@ -350,11 +370,12 @@ def run_sal(args, wl: synth.Workload) -> dict | None:
     if api.sal_last_device_status(s) != 0:
         raise RuntimeError("device wait timed out during the timed region")
     value = job_throughput(my_wl.audio_seconds * args.steps, world, total_s)
-    flops_step = workload_flops(B, T, L, args.chunk)
+    flops_step = workload_flops(B, T, L, args.chunk, window)
 
     # ---- per-kind launch durations (events around each launch, traced graph replays)
     kinds = {}
-    k_steps = max(3, min(args.steps, 20))
+    # traced replays per kind: up to 20, fewer for long steps (about 3 s of replays per kind)
+    k_steps = max(3, min(args.steps, 20, int(3000.0 / max(total_s * 1e3 / args.steps, 1e-3))))
     for kind_id, kind in enumerate(api.KIND_NAMES):
         per_step = {"rope_table": 1, "layernorm": 2 * L + 1}.get(kind, L)
         evs = [torch.cuda.Event(enable_timing=True) for _ in range(2 * per_step)]
@@ -369,7 +390,7 @@ def run_sal(args, wl: synth.Workload) -> dict | None:
             api._check("sal_stack_project", lib.sal_stack_project(stacked.data_ptr(), B, T, rec,
                                                                   x.data_ptr(), cs))
             api.sal_encoder_forward_ex(x, B, T, dw, L, workspace=ws, emb=emb, chunk=args.chunk, kind=kind_id,
-                                       events=evs, stream=cs)
+                                       events=evs, stream=cs, window_core=wcore, window_context=wctx)
         durs = []
         with torch.cuda.stream(s):
             for _ in range(k_steps):
@@ -386,12 +407,17 @@ def run_sal(args, wl: synth.Workload) -> dict | None:
     tensor_kinds = ["qkv", "attention", "out_proj", "ffn_up", "ffn_down"]
     dom = max(tensor_kinds, key=lambda k: kinds[k]["ms_per_step"])
     peaks = _peaks()
-    achieved = kernel_flops(dom, B, T, args.chunk) / (kinds[dom]["avg_ms"] / 1e3) / 1e12
+    achieved = kernel_flops(dom, B, T, args.chunk, window) / (kinds[dom]["avg_ms"] / 1e3) / 1e12
     roofline = {"kernel": dom, "bound": "tensor", "achieved": achieved, "peak": peaks["tflops"],
                 "unit": "TFLOP/s", "frac": achieved / peaks["tflops"],
-                "traffic": _traffic(dom, wl.name) if args.chunk == 0 else None,
+                "traffic": _traffic(dom, wl.name) if args.chunk == 0 and not window else None,
                 "peak_source": peaks["tflops_source"],
-                "per_launch_flops": kernel_flops(dom, B, T, args.chunk), "avg_launch_ms": kinds[dom]["avg_ms"]}
+                # the same rate against the pool's sustained (power-capped) GEMM figure, and
+                # the median SM clock of the timed region it ran at
+                "peak_sustained": peaks["tflops_sustained"], "frac_sustained": achieved / peaks["tflops_sustained"],
+                "sm_mhz_timed": clk.get("sm_mhz"),
+                "per_launch_flops": kernel_flops(dom, B, T, args.chunk, window),
+                "avg_launch_ms": kinds[dom]["avg_ms"]}
 
     # ---- the front end against HBM: algorithmic bytes (samples read once, fp32 log-mel and
     #      the bf16 stack written once) over its event-timed launch
@@ -424,7 +450,7 @@ def run_sal(args, wl: synth.Workload) -> dict | None:
 
     # ---- end to end through sal_encode with pinned host buffers
     e2e = None
-    if not args.no_e2e and args.chunk == 0:
+    if not args.no_e2e and args.chunk == 0 and not window:
         wave_h = torch.from_numpy(audio).pin_memory()
         emb_h = torch.empty((B, T, 1280), dtype=torch.bfloat16).pin_memory()
         ews = api.encode_workspace(B, N, dev)
@@ -453,6 +479,7 @@ def run_sal(args, wl: synth.Workload) -> dict | None:
     if world == 1 and not args.no_cpu_baseline:
         est, desc, spent, threads = oracle_step_estimate(wl, 15.0, audio[0])
         cpu = {"value": wl.audio_seconds / est, "unit": UNIT, "cores": threads, "kind": "oracle",
+               "cpu_model": _cpu_model(), "nproc": os.cpu_count(),
                "sample": desc + f"; {spent:.1f} s of CPU work"}
 
     if world > 1:
@@ -465,13 +492,18 @@ def run_sal(args, wl: synth.Workload) -> dict | None:
         "warmup": args.warmup, "ms_per_step": step_ms_mean, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": {"workload": wl.name, "batch": B, "n_samples": N, "positions": T, "layers": L,
-                   "attention": f"chunks of {args.chunk} positions" if 0 < args.chunk < T else "whole clip",
+                   "attention": (f"serving windows of {wcore} core + 2 x {wctx} context positions" if window
+                                 else f"chunks of {args.chunk} positions" if 0 < args.chunk < T else "whole clip"),
                    "parallelism": f"dp{world} (independent clips per GPU)" if world > 1 else "single GPU",
                    "l2": "256 MiB buffer rewritten between timed steps", "graph": "one CUDA graph per step"},
         "tc_frac_step": flops_step / (step_ms_mean / 1e3) / 1e12 / peaks["tflops"],
+        "tc_frac_step_sustained": flops_step / (step_ms_mean / 1e3) / 1e12 / peaks["tflops_sustained"],
         "roofline": roofline,
         "frontend_roofline": frontend_roofline,
         "kernels": kinds,
+        "kernels_note": ("per-launch durations from event pairs around every launch of one kind in a traced "
+                         "replay of the step; the event records break the programmatic-dependent-launch "
+                         "overlap, so each is an upper bound and the shares need not sum to 1"),
         "cpu_baseline": cpu,
         "e2e": e2e,
         "gpu_launches": int(launches_per_step * args.steps),
@@ -503,30 +535,49 @@ def _nvsmi_id(local: int) -> str:
 
 
 def _peaks() -> dict:
+    """Roofline denominators: the machine's measured HBM copy bandwidth and cuBLAS bf16 GEMM
+    rate, burst (a kernel timed on its own) and sustained (a seconds-long loop under the
+    power cap); else the fallback figures of an earlier measurement on the same pool."""
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
         p = json.load(open(path))
-        return {"tflops": float(p["bf16_tflops_sustained"]), "tflops_source": "measured (sustained bf16)",
+        return {"tflops": float(p["bf16_tflops"]), "tflops_source": "measured (burst bf16)",
+                "tflops_sustained": float(p["bf16_tflops_sustained"]),
                 "gbs": float(p["hbm_gbs"]), "gbs_source": "measured"}
-    except (OSError, KeyError, ValueError):
-        return {"tflops": 1400.0, "tflops_source": "fallback (sustained bf16)", "gbs": 6650.0,
-                "gbs_source": "fallback"}
+    except (OSError, KeyError, ValueError, TypeError):
+        return {"tflops": 1590.0, "tflops_source": "fallback (burst bf16)", "tflops_sustained": 1400.0,
+                "gbs": 6650.0, "gbs_source": "fallback"}
+
+
+def _cpu_model() -> str:
+    try:
+        for line in open("/proc/cpuinfo"):
+            if line.startswith("model name"):
+                return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    import platform
+    return platform.processor() or "unknown"
 
 
 def main():
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=300)
-    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=synth.WORKLOAD_ORDER)
     ap.add_argument("--impl", default="sal", choices=["sal", "reference"])
     ap.add_argument("--chunk", type=int, default=0,
                     help="attention within chunks of this many positions (0: whole clip)")
+    ap.add_argument("--window", action="store_true",
+                    help="serving windows: 500 core positions with 50 context positions on each side")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
+    if args.window and args.chunk:
+        ap.error("--window and --chunk are exclusive")
     wl = synth.WORKLOADS[args.workload]
     out = run_reference(args, wl) if args.impl == "reference" else run_sal(args, wl)
     if out is not None:

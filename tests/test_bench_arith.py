@@ -37,3 +37,17 @@ def test_frontend_bytes():
     assert bench.frontend_bytes(1, 57_600_000) == 4 * 57_600_000 + 512 * 359_998 + 2048 * 44_999
     assert bench.frontend_bytes(3, 16_000) == 3 * (4 * 16_000 + 512 * 98 + 2048 * 12)
     assert bench.frontend_bytes(1, 399) == 4 * 399
+
+
+def test_serving_window_work():
+    """Serving windows: every window's own positions and pairs, context included; the
+    lengths agree with the oracle's window bounds."""
+    T = O.position_count(57_600_000)
+    lens = bench.window_lengths(T, 500, 50)
+    assert lens == [hi - lo for lo, _, _, hi in O.window_bounds(T, 500, 50)]
+    assert len(lens) == 90 and lens[0] == 550 and lens[1] == 600 and lens[-1] == 549
+    rows, pairs = bench.layer_work(T, window=(500, 50))
+    assert rows == sum(lens) == T + 2 * 50 * 89
+    assert pairs == sum(n * n for n in lens)
+    assert bench.layer_work(T) == (T, T * T)
+    assert bench.kernel_flops("attention", 1, T, window=(500, 50)) == 5120 * pairs
