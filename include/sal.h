@@ -166,11 +166,33 @@ typedef struct {
  *          Speech to Dataset Audits", section "Local encoder windows, recording-wide
  *          language context" (independent 30-second post-feature chunks = 375 positions).
  *          chunk <= 0 or chunk >= T: attention over the whole clip (sal_encoder_forward).
- *   trace: optional event trace (may be NULL). */
+ *   trace: optional event trace (may be NULL).
+ *   window_core, window_context: serving windows (the serving-path paragraph of the same
+ *          section: context-extended windows, overlap outputs discarded, core outputs
+ *          concatenated; its defaults are SAL_WINDOW_CORE = 500 core positions and
+ *          SAL_WINDOW_CONTEXT = 50 context positions on each side). With window_core > 0
+ *          each clip is cut into cores of window_core consecutive positions from 0 (the
+ *          last may be shorter); window w is its core extended by up to window_context
+ *          positions on each side inside the clip. Every window runs the n_layers layers
+ *          and the final LayerNorm as an independent sequence (attention inside the
+ *          window, positions from 0 at its start), and emb receives each position's
+ *          output from the window whose core holds it; x receives, at each position, the
+ *          residual stream of that same window. window_core <= 0: no windows. Windows
+ *          and chunk > 0 together are SAL_EINVAL; window_context must be >= 0. The
+ *          workspace must hold sal_encoder_workspace_bytes_ex(batch, T, opts). */
 typedef struct {
     int64_t chunk;
     const sal_trace* trace;
+    int64_t window_core;
+    int64_t window_context;
 } sal_forward_options;
+
+#define SAL_WINDOW_CORE 500
+#define SAL_WINDOW_CONTEXT 50
+
+/* Workspace bytes of sal_encoder_forward_ex with these options (opts may be NULL; 0 when
+ * batch or T is <= 0). Equal to sal_encoder_workspace_bytes without serving windows. */
+size_t sal_encoder_workspace_bytes_ex(int batch, int64_t T, const sal_forward_options* opts);
 
 /* sal_encoder_forward with options (opts may be NULL: whole-clip attention, no trace). */
 sal_status sal_encoder_forward_ex(float* x, int batch, int64_t T, const sal_weights* w,
@@ -185,8 +207,10 @@ uint64_t sal_launch_count(void);
  * waits set when they give up: SAL_OK or SAL_ETIMEOUT. */
 sal_status sal_last_device_status(void* stream);
 
-/* Upper bound in nanoseconds of every mbarrier wait inside the kernels (default 4e9).
- * A wait that exceeds it sets the device status word and the kernel returns early. */
+/* Upper bound in nanoseconds of every mbarrier wait inside the kernels (default 4e9; 0 is
+ * taken as 1). A wait that exceeds it sets the device status word and the kernel winds
+ * down: each CTA waits for its own TMA loads and MMAs still in flight, with a fixed bound
+ * of 4 s that this limit does not shorten, then frees its tensor memory and returns. */
 void sal_set_wait_limit_ns(uint64_t ns);
 
 /* ---------------------------------------------------------------------------------
@@ -324,6 +348,19 @@ sal_status sal_attention_heads(const void* q, const void* k, const void* v, int 
  * tiles up. SAL_ATTN_PP=0/1 in the environment forces none/all. Host arithmetic only: no
  * device is needed. *pairs is 0 for head_dim 64 (one-tile kernel only). */
 sal_status sal_attention_plan(int batch, int64_t T, int heads, int head_dim, int sms, int* pairs, int* query_tiles);
+/* (sal_attention_plan returns SAL_ESHAPE for T > 90,000, as sal_attention_heads does.) */
+
+/* Test hook for the bounded waits (no counterpart on the pages). One launch of the
+ * attention kernel `kernel` (1: one query tile per CTA; 2: two query tiles per CTA) over
+ * 10 heads of width 128, as sal_attention, except that every CTA's producer never issues
+ * the loads of its key/value tile number `tile` (counted from the CTA's first key tile).
+ * The wait for that tile gives up after the limit of sal_set_wait_limit_ns, the kernel
+ * winds down, and sal_last_device_status then reports SAL_ETIMEOUT; o is unspecified.
+ * A CTA with `tile` or fewer key tiles is unaffected. Errors: SAL_EINVAL (kernel not 1 or
+ * 2, tile < 0, null or misaligned pointer), SAL_ESHAPE as sal_attention, SAL_EDEVICE
+ * (not an sm_100 GPU, or kernel 2 unavailable on it). */
+sal_status sal_attention_withhold(const void* q, const void* k, const void* v, int batch, int64_t T, int kernel,
+                                  int tile, void* o, void* stream);
 
 /* Row log-softmax (the adapter's last step): out[r, i] = z[r, i] - log sum_j exp z[r, j]
  * for i < n. z rows are ld floats apart (ld >= n), out rows n floats apart; float32. */

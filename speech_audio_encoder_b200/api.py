@@ -54,7 +54,11 @@ class sal_trace(ctypes.Structure):
 
 
 class sal_forward_options(ctypes.Structure):
-    _fields_ = [("chunk", ctypes.c_int64), ("trace", ctypes.POINTER(sal_trace))]
+    _fields_ = [("chunk", ctypes.c_int64), ("trace", ctypes.POINTER(sal_trace)),
+                ("window_core", ctypes.c_int64), ("window_context", ctypes.c_int64)]
+
+
+WINDOW_CORE, WINDOW_CONTEXT = 500, 50  # the serving-window defaults (sal.h)
 
 
 KIND_NAMES = ["rope_table", "layernorm", "qkv", "attention", "out_proj", "ffn_up", "ffn_down"]
@@ -69,6 +73,8 @@ EXPORTS = {
     "sal_stack_project": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int, ctypes.c_int64,
                                           ctypes.POINTER(sal_weights), ctypes.c_void_p, ctypes.c_void_p]),
     "sal_encoder_workspace_bytes": (ctypes.c_size_t, [ctypes.c_int, ctypes.c_int64]),
+    "sal_encoder_workspace_bytes_ex": (ctypes.c_size_t, [ctypes.c_int, ctypes.c_int64,
+                                                         ctypes.POINTER(sal_forward_options)]),
     "sal_encoder_forward": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int, ctypes.c_int64,
                                             ctypes.POINTER(sal_weights), ctypes.c_int, ctypes.c_void_p,
                                             ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]),
@@ -108,6 +114,9 @@ EXPORTS = {
                                         ctypes.c_void_p, ctypes.c_void_p]),
     "sal_attention_plan": (ctypes.c_int, [ctypes.c_int, ctypes.c_int64, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                            ctypes.POINTER(ctypes.c_int), ctypes.POINTER(ctypes.c_int)]),
+    "sal_attention_withhold": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int,
+                                               ctypes.c_int64, ctypes.c_int, ctypes.c_int, ctypes.c_void_p,
+                                               ctypes.c_void_p]),
     "sal_ctc_workspace_bytes": (ctypes.c_size_t, [ctypes.c_int, ctypes.c_int64]),
     "sal_ctc_adapter": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int, ctypes.c_int64,
                                         ctypes.POINTER(sal_ctc_weights), ctypes.c_void_p, ctypes.c_void_p,
@@ -298,14 +307,24 @@ def sal_encoder_forward(x: torch.Tensor, batch: int, T: int, weights, n_layers: 
     return emb
 
 
+def encoder_workspace_ex(batch: int, T: int, chunk: int = 0, window_core: int = 0, window_context: int = 0,
+                         device="cuda") -> torch.Tensor:
+    opts = sal_forward_options(chunk, None, window_core, window_context)
+    n = lib().sal_encoder_workspace_bytes_ex(batch, T, ctypes.byref(opts))
+    return torch.empty(max(n, 256), dtype=torch.uint8, device=device)
+
+
 def sal_encoder_forward_ex(x: torch.Tensor, batch: int, T: int, weights, n_layers: int,
                            workspace: torch.Tensor | None = None, emb: torch.Tensor | None = None,
-                           chunk: int = 0, kind: int | None = None, events=None, stream=None) -> torch.Tensor:
+                           chunk: int = 0, kind: int | None = None, events=None, stream=None,
+                           window_core: int = 0, window_context: int = 0) -> torch.Tensor:
     """sal_encoder_forward with chunked attention (``chunk`` positions per chunk, 0 = whole
-    clip) and, optionally, torch.cuda.Event pairs recorded around each launch of ``kind``."""
+    clip) or serving windows (``window_core`` core positions with ``window_context`` context
+    positions on each side, 0 = none) and, optionally, torch.cuda.Event pairs recorded
+    around each launch of ``kind``."""
     rec = weights.record if isinstance(weights, DeviceWeights) else weights
     if workspace is None:
-        workspace = encoder_workspace(batch, T, x.device)
+        workspace = encoder_workspace_ex(batch, T, chunk, window_core, window_context, x.device)
     if emb is None:
         emb = torch.empty((batch * T, WIDTH), dtype=torch.bfloat16, device=x.device)
     trace_p = None
@@ -315,7 +334,7 @@ def sal_encoder_forward_ex(x: torch.Tensor, batch: int, T: int, weights, n_layer
         handles = (ctypes.c_void_p * len(events))(*[e.cuda_event for e in events])
         tr = sal_trace(kind, ctypes.cast(handles, ctypes.POINTER(ctypes.c_void_p)), len(events))
         trace_p = ctypes.pointer(tr)
-    opts = sal_forward_options(chunk, trace_p)
+    opts = sal_forward_options(chunk, trace_p, window_core, window_context)
     _check("sal_encoder_forward_ex", lib().sal_encoder_forward_ex(
         _ptr(x), batch, T, ctypes.byref(rec), n_layers, _ptr(emb), _ptr(workspace), workspace.numel(),
         _stream(stream), ctypes.byref(opts)))
@@ -386,6 +405,17 @@ def sal_attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, stream=None
     batch, H, T, hd = q.shape
     o = torch.empty((batch * T, H * hd), dtype=torch.bfloat16, device=q.device)
     _check("sal_attention", lib().sal_attention(_ptr(q), _ptr(k), _ptr(v), batch, T, _ptr(o), _stream(stream)))
+    return o
+
+
+def sal_attention_withhold(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, kernel: int, tile: int,
+                           stream=None) -> torch.Tensor:
+    """Test hook: sal_attention with key/value tile ``tile`` of every CTA never loaded, so a
+    bounded wait gives up (read the outcome with sal_last_device_status)."""
+    batch, H, T, hd = q.shape
+    o = torch.empty((batch * T, H * hd), dtype=torch.bfloat16, device=q.device)
+    _check("sal_attention_withhold", lib().sal_attention_withhold(_ptr(q), _ptr(k), _ptr(v), batch, T, kernel, tile,
+                                                                  _ptr(o), _stream(stream)))
     return o
 
 

@@ -63,12 +63,33 @@ struct AttnArgs {
   float scale_log2;
   uint64_t limit_ns;
   unsigned int* status;
+  // Test hook (sal_attention_withhold): the key/value tile at this index (relative to the
+  // CTA's first key tile) is never loaded, so the wait for it gives up at limit_ns. -1: off.
+  int withhold = -1;
+  // Serving windows (win_count > 0): clip c of the batch is window c % win_count of a
+  // recording of win_total positions, left-aligned in its T slots; only its first
+  // window_len(c) positions are keys (see valid_len).
+  int win_count = 0, win_core = 0, win_ctx = 0;
+  int64_t win_total = 0;
 };
 
+// Positions of clip `clip` that are keys: T, or for serving windows the window's own
+// length (its core extended by up to win_ctx positions on each side inside the recording).
+__device__ __forceinline__ int64_t valid_len(const AttnArgs& a, int clip) {
+  if (a.win_count <= 0) return a.T;
+  const int64_t w = clip % a.win_count;
+  const int64_t lo = w * a.win_core - a.win_ctx, hi = (w + 1) * a.win_core + a.win_ctx;
+  return (hi < a.win_total ? hi : a.win_total) - (lo > 0 ? lo : 0);
+}
+
 // Key tiles [j0, j0 + n) that the query rows [q_lo, q_hi) can see: the union of their
-// chunks [floor(t / chunk) chunk, next chunk start) clipped to T.
+// chunks [floor(t / chunk) chunk, next chunk start) clipped to the T key positions. Rows
+// at or past T (padding slots of a serving window) see the chunk of row T - 1.
 __device__ __forceinline__ void kv_tile_range(int64_t q_lo, int64_t q_hi, int64_t T, int64_t chunk, int& j0,
                                               int& n) {
+  if (q_hi > T) q_hi = T;
+  if (q_lo > T - 1) q_lo = T - 1;
+  if (q_hi <= q_lo) q_hi = q_lo + 1;
   const int64_t kv_lo = (q_lo / chunk) * chunk;
   int64_t kv_hi = ((q_hi - 1) / chunk + 1) * chunk;
   if (kv_hi > T) kv_hi = T;
@@ -76,15 +97,17 @@ __device__ __forceinline__ void kv_tile_range(int64_t q_lo, int64_t q_hi, int64_
   n = static_cast<int>((kv_hi + 127) / 128) - j0;
 }
 
-// Keys [lo, hi) that row t may attend to: its own chunk (empty for rows t >= T). Positions
-// fit in 32 bits (T <= 45000).
-__device__ __forceinline__ void row_range(int t, int T, int chunk, int& lo, int& hi) {
+// Keys [lo, hi) that row t may attend to: its own chunk among the Tk key positions; empty
+// for rows t >= T (past the tensor), the chunk of row Tk - 1 for rows Tk <= t < T (padding
+// slots of a serving window, computed but never used). Positions fit in 32 bits.
+__device__ __forceinline__ void row_range(int t, int T, int Tk, int chunk, int& lo, int& hi) {
   if (t >= T) {
     lo = hi = 0;
     return;
   }
+  if (t >= Tk) t = Tk - 1;
   lo = (t / chunk) * chunk;
-  hi = lo + chunk < T ? lo + chunk : T;
+  hi = lo + chunk < Tk ? lo + chunk : Tk;
 }
 
 // Columns [c_lo, c_hi) of key tile jt inside [lo, hi).
@@ -92,6 +115,21 @@ __device__ __forceinline__ void tile_cols(int lo, int hi, int jt, int& c_lo, int
   const int base = jt * 128;
   c_lo = min(max(lo - base, 0), 128);
   c_hi = min(max(hi - base, 0), 128);
+}
+
+// Maximum of a row of 128 scores held as raw fp32 bits: eight independent chains of
+// three-input max over 16 scores each, then merged, so the longest dependent chain is 10
+// instructions instead of 64.
+__device__ __forceinline__ float row_max128(const uint32_t (&r)[4][32]) {
+  float m[8];
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    const uint32_t* v = &r[k >> 1][(k & 1) * 16];
+    m[k] = fmaxf(__uint_as_float(v[0]), __uint_as_float(v[1]));
+#pragma unroll
+    for (int i = 2; i < 16; i += 2) m[k] = max3f(m[k], __uint_as_float(v[i]), __uint_as_float(v[i + 1]));
+  }
+  return max3f(max3f(m[0], m[1], m[2]), max3f(m[3], m[4], m[5]), fmaxf(m[6], m[7]));
 }
 
 // Scores outside [c_lo, c_hi) of this 32-column chunk become -inf, so the unmasked softmax
@@ -129,10 +167,10 @@ __global__ void __launch_bounds__(192, 1)
   const int64_t T = args.T;
   const int bh = blockIdx.y;
   const int qt = blockIdx.x + args.qt0;
+  const int64_t Tk = valid_len(args, bh / args.heads);  // key positions of this clip
   int j0, n_kv;
-  kv_tile_range(static_cast<int64_t>(qt) * kTile,
-                static_cast<int64_t>(qt) * kTile + kTile < T ? static_cast<int64_t>(qt) * kTile + kTile : T, T,
-                args.chunk, j0, n_kv);
+  kv_tile_range(static_cast<int64_t>(qt) * kTile, static_cast<int64_t>(qt) * kTile + kTile, Tk, args.chunk, j0,
+                n_kv);
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
@@ -165,10 +203,11 @@ __global__ void __launch_bounds__(192, 1)
   pdl_trigger();
   const uint32_t tmem = *tmem_slot;
   const WaitGuard guard{abort_flag, args.limit_ns, args.status};
+  // the producer's record of the stages it loaded and their phases (for the wind-down)
+  uint32_t issued_q = 0, issued = 0, par_k = 0;
 
   if (warp == 0) {
     if (lane == 0) {
-      uint32_t issued_q = 0, issued = 0, par_k = 0;
       mbar_arrive_expect_tx(q_full, TB);
 #pragma unroll
       for (int b = 0; b < HD / 64; ++b) tma_load_3d(sQ + b * kBox, &tmQ, q_full, 64 * b, qt * kTile, bh);
@@ -177,6 +216,7 @@ __global__ void __launch_bounds__(192, 1)
         const int s = j & 1;
         const uint32_t use_par = (j >> 1) & 1;
         if (!mbar_wait(&kv_empty[s], use_par ^ 1, guard)) break;
+        if (j == args.withhold) continue;  // nothing issued: stage s keeps its last tracked load
         mbar_arrive_expect_tx(&k_full[s], TB);
 #pragma unroll
         for (int b = 0; b < HD / 64; ++b) tma_load_3d(sK[s] + b * kBox, &tmK, &k_full[s], 64 * b, (j0 + j) * kTile, bh);
@@ -185,14 +225,6 @@ __global__ void __launch_bounds__(192, 1)
         for (int b = 0; b < HD / 64; ++b) tma_load_3d(sV[s] + b * kBox, &tmV, &v_full[s], 64 * b, (j0 + j) * kTile, bh);
         issued |= 1u << s;
         par_k = (par_k & ~(1u << s)) | (use_par << s);
-      }
-      if (*abort_flag) {
-        if (issued_q) drain_wait(q_full, 0, args.limit_ns);
-        for (int s = 0; s < 2; ++s)
-          if (issued & (1u << s)) {
-            drain_wait(&k_full[s], (par_k >> s) & 1, args.limit_ns);
-            drain_wait(&v_full[s], (par_k >> s) & 1, args.limit_ns);
-          }
       }
     }
   } else if (warp == 1) {
@@ -235,7 +267,7 @@ __global__ void __launch_bounds__(192, 1)
       if (*abort_flag && any_mma) {
         // every MMA issued so far is covered by one more commit
         umma_commit(drain);
-        drain_wait(drain, 0, args.limit_ns);
+        drain_wait(drain, 0);
       }
     }
   } else {
@@ -247,7 +279,8 @@ __global__ void __launch_bounds__(192, 1)
     float m_ref = -INFINITY, l = 0.f;
     bool ok = true;
     int row_lo, row_hi;
-    row_range(qt * kTile + row, static_cast<int>(T), static_cast<int>(args.chunk), row_lo, row_hi);
+    row_range(qt * kTile + row, static_cast<int>(T), static_cast<int>(Tk), static_cast<int>(args.chunk), row_lo,
+              row_hi);
     for (int j = 0; j < n_kv; ++j) {
       const int s = j & 1;
       if (!mbar_wait_warp(&s_full[s], (j >> 1) & 1, guard)) {
@@ -265,12 +298,7 @@ __global__ void __launch_bounds__(192, 1)
 #pragma unroll
         for (int c = 0; c < 4; ++c) mask_chunk(r[c], 32 * c, c_lo, c_hi);
       }
-      float mx = -INFINITY;
-#pragma unroll
-      for (int c = 0; c < 4; ++c)
-#pragma unroll
-        for (int i = 0; i < 32; i += 2) mx = max3f(mx, __uint_as_float(r[c][i]), __uint_as_float(r[c][i + 1]));
-      mx *= sl2;
+      float mx = row_max128(r) * sl2;
       float alpha = 1.f;
       bool rescale = false;
       if (j == 0) {
@@ -284,7 +312,7 @@ __global__ void __launch_bounds__(192, 1)
       const float m_use = m_ref == -INFINITY ? 0.f : m_ref;
       // two scores per instruction: x = s * scale - m (packed fma), the row sum (packed add)
       const uint64_t sl2_2 = f2_pack(sl2, sl2), negm_2 = f2_pack(-m_use, -m_use);
-      uint64_t sum2 = f2_pack(0.f, 0.f);
+      uint64_t sum2[4];  // one running pair sum per 32-column chunk: four short chains
       uint32_t p[2][32];
 #pragma unroll
       for (int c = 0; c < 4; ++c)
@@ -300,11 +328,11 @@ __global__ void __launch_bounds__(192, 1)
             e0 = fast_exp2(x0);
             e1 = fast_exp2(x1);
           }
-          sum2 = f2_add(sum2, f2_pack(e0, e1));
+          sum2[c] = i == 0 ? f2_pack(e0, e1) : f2_add(sum2[c], f2_pack(e0, e1));
           p[c >> 1][(c & 1) * 16 + (i >> 1)] = pack_bf16x2(e0, e1);
         }
       float sum_lo, sum_hi;
-      f2_unpack(sum2, sum_lo, sum_hi);
+      f2_unpack(f2_add(f2_add(sum2[0], sum2[1]), f2_add(sum2[2], sum2[3])), sum_lo, sum_hi);
       const float sum = sum_lo + sum_hi;
       if (j > 0) {
         // PV_{j-1} must be complete before O is rescaled or P buffer s is overwritten
@@ -366,6 +394,17 @@ __global__ void __launch_bounds__(192, 1)
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
+  // Every role has finished, so the abort flag is final. After an abort some loads may
+  // have been issued that no consumer waited for: let each land before the CTA, and its
+  // shared memory, goes away.
+  if (warp == 0 && lane == 0 && *abort_flag) {
+    if (issued_q) drain_wait(q_full, 0);
+    for (int s = 0; s < 2; ++s)
+      if (issued & (1u << s)) {
+        drain_wait(&k_full[s], (par_k >> s) & 1);
+        drain_wait(&v_full[s], (par_k >> s) & 1);
+      }
+  }
   if (args.tail) pdl_wait();
 }
 
@@ -387,6 +426,18 @@ __global__ void __launch_bounds__(192, 1)
 // softmax warpgroups grow to kRegsSoftmax, so each softmax thread holds its whole row of
 // S (128 scores) and reads it from TMEM in one round trip per tile.
 constexpr size_t kSmemPP = 1024 + 6 * kTileBytes + 256;
+// Of every 16 score pairs of a row chunk, this many take their exponentials on the FMA
+// pipe (exp2_pair_poly) instead of the SFU.
+#ifndef SAL_PP_POLY_PAIRS
+#define SAL_PP_POLY_PAIRS 0
+#endif
+constexpr int kPolyPairsPP = SAL_PP_POLY_PAIRS;
+// Each softmax warpgroup hands P to the tensor core in two halves of 64 keys, so the first
+// half of P V runs while the second half's exponentials are computed.
+#ifndef SAL_PP_SPLIT_P
+#define SAL_PP_SPLIT_P 0
+#endif
+constexpr bool kSplitP = SAL_PP_SPLIT_P != 0;
 constexpr int kThreadsPP = 384;
 constexpr int kRegsCtrl = 80, kRegsSoftmax = 208;
 constexpr int kRegsNeededPP = kRegsCtrl * 128 + kRegsSoftmax * 256;  // <= launch regs x 384
@@ -411,17 +462,17 @@ __global__ void __launch_bounds__(kThreadsPP, 1)
   uint64_t* drain = bars + 15;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 16);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  uint64_t* p_half1 = bars + 18;  // [2] second half of P (kSplitP; p_full then means the first)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int64_t T = args.T;
   const int bh = blockIdx.y;
   const int qt2 = blockIdx.x;  // 256-row query block
+  const int64_t Tk = valid_len(args, bh / args.heads);  // key positions of this clip
   int j0, n_kv;
-  kv_tile_range(static_cast<int64_t>(qt2) * 2 * kTile,
-                static_cast<int64_t>(qt2) * 2 * kTile + 2 * kTile < T ? static_cast<int64_t>(qt2) * 2 * kTile + 2 * kTile
-                                                                      : T,
-                T, args.chunk, j0, n_kv);
+  kv_tile_range(static_cast<int64_t>(qt2) * 2 * kTile, static_cast<int64_t>(qt2) * 2 * kTile + 2 * kTile, Tk,
+                args.chunk, j0, n_kv);
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
@@ -432,6 +483,7 @@ __global__ void __launch_bounds__(kThreadsPP, 1)
       mbar_init(&v_empty[s], 1);
       mbar_init(&s_full[s], 1);
       mbar_init(&p_full[s], 128);
+      mbar_init(&p_half1[s], 128);
       mbar_init(&o_final[s], 1);
     }
     mbar_init(drain, 1);
@@ -452,13 +504,14 @@ __global__ void __launch_bounds__(kThreadsPP, 1)
   pdl_trigger();
   const uint32_t tmem = *tmem_slot;
   const WaitGuard guard{abort_flag, args.limit_ns, args.status};
+  // the producer's record of the stages it loaded and their phases (for the wind-down)
+  uint32_t issued_k = 0, issued_v = 0, par_k = 0, par_v = 0;
   // Each role runs inside the branch that set its register limit, so the compiler
   // allocates it against that limit.
   if (warp < 4) {
     setmaxnreg_dec<kRegsCtrl>();
     if (warp == 0) {
       if (lane == 0) {
-        uint32_t issued_k = 0, issued_v = 0, par_k = 0, par_v = 0;
         mbar_arrive_expect_tx(q_full, 2 * kTileBytes);
         for (int i = 0; i < 2; ++i) {
           tma_load_3d(sQ + i * kTileBytes, &tmQ, q_full, 0, (2 * qt2 + i) * kTile, bh);
@@ -468,6 +521,7 @@ __global__ void __launch_bounds__(kThreadsPP, 1)
           const int s = j & 1;
           const uint32_t use_par = (j >> 1) & 1;
           if (!mbar_wait(&k_empty[s], use_par ^ 1, guard)) break;
+          if (j == args.withhold) continue;  // nothing issued: stage s keeps its last tracked loads
           mbar_arrive_expect_tx(&k_full[s], kTileBytes);
           tma_load_3d(sK + s * kTileBytes, &tmK, &k_full[s], 0, (j0 + j) * kTile, bh);
           tma_load_3d(sK + s * kTileBytes + kBox, &tmK, &k_full[s], 64, (j0 + j) * kTile, bh);
@@ -479,13 +533,6 @@ __global__ void __launch_bounds__(kThreadsPP, 1)
           tma_load_3d(sV + s * kTileBytes + kBox, &tmV, &v_full[s], 64, (j0 + j) * kTile, bh);
           issued_v |= 1u << s;
           par_v = (par_v & ~(1u << s)) | (use_par << s);
-        }
-        if (*abort_flag) {
-          drain_wait(q_full, 0, args.limit_ns);
-          for (int s = 0; s < 2; ++s) {
-            if (issued_k & (1u << s)) drain_wait(&k_full[s], (par_k >> s) & 1, args.limit_ns);
-            if (issued_v & (1u << s)) drain_wait(&v_full[s], (par_v >> s) & 1, args.limit_ns);
-          }
         }
       }
     } else if (warp == 1) {
@@ -515,9 +562,14 @@ __global__ void __launch_bounds__(kThreadsPP, 1)
           tc_fence_after();
           const uint32_t v0 = smem_u32(sV + s * kTileBytes);
   #pragma unroll
-          for (int kk = 0; kk < 8; ++kk)
+          for (int kk = 0; kk < 8; ++kk) {
+            if (kSplitP && kk == 4) {  // keys 64-127: their P is the second half
+              if (!mbar_wait(&p_half1[i], j & 1, guard)) return false;
+              tc_fence_after();
+            }
             umma_ts(tmem + 256 + 128 * i, tmem + 128 * i + kk * 8, sdesc_mnmajor_sw128(v0 + kk * 2048, kBox), IDESC_O,
                     (j > 0 || kk > 0));
+          }
           if (i == 1) umma_commit(&v_empty[s]);
           return true;
         };
@@ -541,7 +593,7 @@ __global__ void __launch_bounds__(kThreadsPP, 1)
         }
         if (*abort_flag && any_mma) {
           umma_commit(drain);
-          drain_wait(drain, 0, args.limit_ns);
+          drain_wait(drain, 0);
         }
       }
     }
@@ -557,7 +609,8 @@ __global__ void __launch_bounds__(kThreadsPP, 1)
     float m_ref = -INFINITY, l = 0.f;
     bool ok = true;
     int row_lo, row_hi;
-    row_range((2 * qt2 + wg) * kTile + row, static_cast<int>(T), static_cast<int>(args.chunk), row_lo, row_hi);
+    row_range((2 * qt2 + wg) * kTile + row, static_cast<int>(T), static_cast<int>(Tk), static_cast<int>(args.chunk),
+              row_lo, row_hi);
     for (int j = 0; j < n_kv; ++j) {
       if (!mbar_wait_warp(&s_full[wg], j & 1, guard)) {
         ok = false;
@@ -576,12 +629,7 @@ __global__ void __launch_bounds__(kThreadsPP, 1)
 #pragma unroll
         for (int c = 0; c < 4; ++c) mask_chunk(r[c], 32 * c, c_lo, c_hi);
       }
-      float mx = -INFINITY;
-#pragma unroll
-      for (int c = 0; c < 4; ++c)
-#pragma unroll
-        for (int i = 0; i < 32; i += 2) mx = max3f(mx, __uint_as_float(r[c][i]), __uint_as_float(r[c][i + 1]));
-      mx *= sl2;
+      float mx = row_max128(r) * sl2;
       float alpha = 1.f;
       bool rescale = false;
       if (j == 0) {
@@ -591,25 +639,51 @@ __global__ void __launch_bounds__(kThreadsPP, 1)
         m_ref = mx;
         rescale = true;
       }
+      // O_i(j-1) is complete (it was issued before S_i(j)); rescale it if the max moved.
+      // PV_i(j) is issued only after P arrives below, so this precedes it.
+      if (kSplitP && j > 0 && __any_sync(0xffffffffu, rescale)) {
+#pragma unroll 1
+        for (int c = 0; c < 4; ++c) {
+          uint32_t o[32];
+          tmem_ld32(tmem + lane_base + colO + 32 * c, o);
+          tmem_wait_ld();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+          tmem_st32(tmem + lane_base + colO + 32 * c, o);
+        }
+      }
       // exponentials, row sum, bf16 P packed in place over the scores already consumed
       const float m_use = m_ref == -INFINITY ? 0.f : m_ref;  // a row with no key seen yet
       const uint64_t sl2_2 = f2_pack(sl2, sl2), negm_2 = f2_pack(-m_use, -m_use);
-      uint64_t sum2 = f2_pack(0.f, 0.f);
+      uint64_t sum2[4];  // one running pair sum per 32-column chunk: four short chains
 #pragma unroll
-      for (int c = 0; c < 4; ++c)
+      for (int c = 0; c < 4; ++c) {
+        if (kSplitP && c == 2) {  // the first 64 keys' P is complete: hand it over
+          tmem_st32(tmem + lane_base + colS, r[0]);
+          tmem_wait_st();
+          tc_fence_before();
+          mbar_arrive(&p_full[wg]);
+        }
 #pragma unroll
         for (int i = 0; i < 32; i += 2) {
           float x0, x1;
           f2_unpack(f2_fma(f2_pack(__uint_as_float(r[c][i]), __uint_as_float(r[c][i + 1])), sl2_2, negm_2), x0, x1);
-          const float e0 = fast_exp2(x0), e1 = fast_exp2(x1);
-          sum2 = f2_add(sum2, f2_pack(e0, e1));
+          float e0, e1;
+          if (kPolyPairsPP > 0 && ((i >> 1) & 15) < kPolyPairsPP) {
+            exp2_pair_poly(x0, x1, e0, e1);  // on the FMA pipe, leaving the SFU to the others
+          } else {
+            e0 = fast_exp2(x0);
+            e1 = fast_exp2(x1);
+          }
+          sum2[c] = i == 0 ? f2_pack(e0, e1) : f2_add(sum2[c], f2_pack(e0, e1));
           r[c >> 1][(c & 1) * 16 + (i >> 1)] = pack_bf16x2(e0, e1);
         }
-      tmem_st32(tmem + lane_base + colS, r[0]);
+      }
+      if (!kSplitP) tmem_st32(tmem + lane_base + colS, r[0]);
       tmem_st32(tmem + lane_base + colS + 32, r[1]);
       // O_i(j-1) is complete (it was issued before S_i(j)); rescale it if the max moved.
       // PV_i(j) is issued only after p_full below, so this precedes it.
-      if (j > 0 && __any_sync(0xffffffffu, rescale)) {
+      if (!kSplitP && j > 0 && __any_sync(0xffffffffu, rescale)) {
 #pragma unroll 1
         for (int c = 0; c < 4; ++c) {
           uint32_t o[32];
@@ -621,11 +695,11 @@ __global__ void __launch_bounds__(kThreadsPP, 1)
         }
       }
       float sum_lo, sum_hi;
-      f2_unpack(sum2, sum_lo, sum_hi);
+      f2_unpack(f2_add(f2_add(sum2[0], sum2[1]), f2_add(sum2[2], sum2[3])), sum_lo, sum_hi);
       l = l * alpha + (sum_lo + sum_hi);
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(&p_full[wg]);
+      mbar_arrive(kSplitP ? &p_half1[wg] : &p_full[wg]);
     }
     if (ok && mbar_wait_warp(&o_final[wg], 0, guard)) {
       tc_fence_after();
@@ -660,6 +734,15 @@ __global__ void __launch_bounds__(kThreadsPP, 1)
     __syncwarp();
     tc_fence_after();
     tmem_dealloc(tmem, 512);
+  }
+  // Every role has finished, so the abort flag is final: let every load this CTA issued
+  // land before the CTA, and its shared memory, goes away.
+  if (warp == 0 && lane == 0 && *abort_flag) {
+    drain_wait(q_full, 0);
+    for (int s = 0; s < 2; ++s) {
+      if (issued_k & (1u << s)) drain_wait(&k_full[s], (par_k >> s) & 1);
+      if (issued_v & (1u << s)) drain_wait(&v_full[s], (par_v >> s) & 1);
+    }
   }
 }
 
@@ -727,7 +810,8 @@ int choose_pairs(int n_qt, uint64_t bh, int sms) {
 }  // namespace
 
 sal_status attention_launch_heads(const void* q, const void* k, const void* v, int batch, int64_t T,
-                                  int64_t chunk, int heads, int head_dim, void* o, cudaStream_t s) {
+                                  int64_t chunk, int heads, int head_dim, void* o, cudaStream_t s,
+                                  const AttnWithhold* hold, const Windows* win) {
   if (T == 0 || batch == 0) return SAL_OK;
   if (head_dim != 64 && head_dim != 128) return SAL_ESHAPE;
   int dev = 0;
@@ -765,6 +849,13 @@ sal_status attention_launch_heads(const void* q, const void* k, const void* v, i
   a.limit_ns = wait_limit_ns();
   a.status = device_status_ptr();
   if (!a.status) return SAL_ECUDA;
+  if (hold) a.withhold = hold->tile;
+  if (win && win->count > 0) {
+    a.win_count = win->count;
+    a.win_core = win->core;
+    a.win_ctx = win->ctx;
+    a.win_total = win->total;
+  }
   const dim3 grid1(static_cast<unsigned>((T + kTile - 1) / kTile), static_cast<unsigned>(bh));
   if (head_dim == 64)
     return launch_kernel(attention_kernel<64>, grid1, dim3(192), smem_one_tile(64), s, tq, tk, tv, a) ==
@@ -784,7 +875,10 @@ sal_status attention_launch_heads(const void* q, const void* k, const void* v, i
   }
   const int mode = attention_pp_mode();
   int P = 0;  // query-tile pairs per (clip, head) for the two-tile kernel
-  if (pp_ok && mode == 1) {
+  if (hold) {
+    if (hold->kernel == 2 && !pp_ok) return SAL_EDEVICE;
+    P = hold->kernel == 2 ? (n_qt + 1) / 2 : 0;
+  } else if (pp_ok && mode == 1) {
     P = (n_qt + 1) / 2;
   } else if (pp_ok && mode != 0) {
     P = choose_pairs(n_qt, bh, sms);
@@ -806,11 +900,32 @@ sal_status attention_launch_heads(const void* q, const void* k, const void* v, i
 }
 
 sal_status attention_launch(const void* q, const void* k, const void* v, int batch, int64_t T,
-                            int64_t chunk, void* o, cudaStream_t s) {
-  return attention_launch_heads(q, k, v, batch, T, chunk, kHeads, kHeadDim, o, s);
+                            int64_t chunk, void* o, cudaStream_t s, const Windows* win) {
+  return attention_launch_heads(q, k, v, batch, T, chunk, kHeads, kHeadDim, o, s, nullptr, win);
 }
 
 }  // namespace sal
+
+// Test hook: one attention launch in which every CTA's producer withholds one key/value
+// tile, so that a bounded wait gives up (see sal.h).
+extern "C" sal_status sal_attention_withhold(const void* q, const void* k, const void* v, int batch, int64_t T,
+                                             int kernel, int tile, void* o, void* stream) {
+  using namespace sal;
+  if (batch < 0 || T < 0 || tile < 0 || (kernel != 1 && kernel != 2)) return SAL_EINVAL;
+  if (T > SAL_MAX_POSITIONS) return SAL_ESHAPE;
+  if (batch == 0 || T == 0) return SAL_OK;
+  if (batch > 6553) return SAL_ESHAPE;
+  if (!q || !k || !v || !o || !aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o))
+    return SAL_EINVAL;
+  int major = 0, dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess)
+    return SAL_ECUDA;
+  if (major != 10) return SAL_EDEVICE;
+  const AttnWithhold hold{kernel, tile};
+  return attention_launch_heads(q, k, v, batch, T, 0, kHeads, kHeadDim, o, static_cast<cudaStream_t>(stream),
+                                &hold);
+}
 
 // The split attention_launch_heads makes for 128-wide heads when the two-tile kernel is
 // available (host arithmetic only; no device is touched).
@@ -818,6 +933,7 @@ extern "C" sal_status sal_attention_plan(int batch, int64_t T, int heads, int he
                                          int* query_tiles) {
   using namespace sal;
   if (batch < 0 || T < 0 || heads < 0 || sms <= 0 || !pairs || !query_tiles) return SAL_EINVAL;
+  if (T > 2 * SAL_MAX_POSITIONS) return SAL_ESHAPE;  // the longest sequence sal_attention_heads takes
   const int n_qt = static_cast<int>((T + kTile - 1) / kTile);
   *query_tiles = n_qt;
   *pairs = 0;
@@ -827,7 +943,3 @@ extern "C" sal_status sal_attention_plan(int batch, int64_t T, int heads, int he
   *pairs = mode == 0 ? 0 : (mode == 1 ? (n_qt + 1) / 2 : choose_pairs(n_qt, bh, sms));
   return SAL_OK;
 }
-
-namespace sal {
-
-}  // namespace sal

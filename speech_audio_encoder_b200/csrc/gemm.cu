@@ -23,6 +23,7 @@
 #include <cuda_bf16.h>
 #include <math.h>
 
+#include <cstdlib>
 #include <mutex>
 
 #include "sal_internal.h"
@@ -48,7 +49,11 @@ struct GemmArgs {
   unsigned int* status;
 };
 
-template <int BN, int EPI>
+// PAIR: a cluster of two CTAs computes a 256 x BN tile with tcgen05.mma.cta_group::2. Each
+// CTA loads its own 128 rows of A and its own BN / 2 rows of W (no multicast), holds its 128
+// rows of the accumulator in its TMEM and runs the epilogue on them; the even CTA issues
+// the MMAs. Per SM this reads half of the W tile of the one-CTA form for the same MMA work.
+template <int BN, int EPI, bool PAIR = false>
 struct Cfg {
   static constexpr int BM = 128, BK = 64;
   static constexpr bool QKV = EPI == kEpiQkv;
@@ -57,13 +62,16 @@ struct Cfg {
   // other kinds stage 128-byte-wide output boxes for TMA, two per warp
   static constexpr int CW = F32_OUT ? 32 : 64;  // output columns per 128-byte box row
   static constexpr int SCR_BYTES = QKV ? 4 * 32 * 128 * 4 + 4 * 32 * 4 : 4 * 2 * 4096;
-  static constexpr int STAGES = QKV ? (BN == 256 ? 3 : 4) : (BN == 256 ? 4 : (BN == 128 ? 6 : 8));
+  static constexpr int BNL = PAIR ? BN / 2 : BN;  // rows of W this CTA loads per tile
+  static constexpr int STAGES = PAIR ? (QKV ? 5 : 6)
+                                     : (QKV ? (BN == 256 ? 3 : 4) : (BN == 256 ? 4 : (BN == 128 ? 6 : 8)));
   static constexpr int A_BYTES = BM * BK * 2;
-  static constexpr int B_BYTES = BN * BK * 2;
+  static constexpr int B_BYTES = BNL * BK * 2;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
   static constexpr int TMEM_COLS = 2 * BN;
   static constexpr size_t SMEM = 1024 + static_cast<size_t>(STAGES) * STAGE_BYTES + SCR_BYTES + 256;
   static_assert(SMEM <= 232448, "shared memory budget");
+  static_assert(!PAIR || BN == 256, "CTA pairs use 256-wide tiles");
 };
 
 __device__ __forceinline__ float gelu_erf(float x) {
@@ -97,11 +105,11 @@ __device__ __forceinline__ float warp_sum(float v) {
   return v;
 }
 
-template <int BN, int EPI>
+template <int BN, int EPI, bool PAIR>
 __global__ void __launch_bounds__(192, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                 const __grid_constant__ CUtensorMap tmC, const GemmArgs args) {
-  using C = Cfg<BN, EPI>;
+  using C = Cfg<BN, EPI, PAIR>;
   extern __shared__ unsigned char smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem;
@@ -113,11 +121,15 @@ __global__ void __launch_bounds__(192, 1)
   uint64_t* tfull = bars + 2 * C::STAGES;
   uint64_t* tempty = tfull + 2;
   uint64_t* drain = tempty + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  uint64_t* bye = drain + 1;  // pairs: the peer has finished every access to this CTA
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bye + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  // pairs: this CTA's rank; the even CTA (rank 0) issues the MMAs and owns the barriers
+  // that both CTAs' loads and epilogues report to
+  const uint32_t rank = PAIR ? cluster_ctarank() : 0u;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::STAGES; ++s) {
@@ -126,9 +138,10 @@ __global__ void __launch_bounds__(192, 1)
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&tfull[a], 1);
-      mbar_init(&tempty[a], 128);
+      mbar_init(&tempty[a], PAIR ? 8 : 128);  // pairs: one arrival per epilogue warp of both CTAs
     }
     mbar_init(drain, 1);
+    mbar_init(bye, 1);
     *abort_flag = 0;
     fence_mbar_init();
     tma_prefetch_desc(&tmA);
@@ -136,11 +149,20 @@ __global__ void __launch_bounds__(192, 1)
     if constexpr (!C::QKV) tma_prefetch_desc(&tmC);
   }
   if (warp == 1) {
-    tmem_alloc(tmem_slot, C::TMEM_COLS);
-    tmem_relinquish();
+    if constexpr (PAIR) {
+      tmem_alloc_pair(tmem_slot, C::TMEM_COLS);
+      tmem_relinquish_pair();
+    } else {
+      tmem_alloc(tmem_slot, C::TMEM_COLS);
+      tmem_relinquish();
+    }
   }
   tc_fence_before();
   __syncthreads();
+  if constexpr (PAIR) {
+    // both CTAs' barriers are initialised before either CTA touches the other's
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+  }
   tc_fence_after();
   // Programmatic dependent launch: the roles that read or write what earlier kernels
   // produce (the A loads, the epilogue) wait for them below; the weight loads of the
@@ -149,42 +171,69 @@ __global__ void __launch_bounds__(192, 1)
   const uint32_t tmem_base = *tmem_slot;
   const WaitGuard guard{abort_flag, args.limit_ns, args.status};
 
-  const int num_m = static_cast<int>((args.M + C::BM - 1) / C::BM);
+  // a work unit is one (row block, column tile, K split); a row block is 128 rows, or
+  // 256 for a CTA pair (this CTA's rows are the half given by its rank)
+  const int ROWS = PAIR ? 2 * C::BM : C::BM;
+  const int num_m = static_cast<int>((args.M + ROWS - 1) / ROWS);
   const int num_n = args.N / BN;
   const int kb_per = (args.K / C::BK) / args.splits;
   const int num_tiles = num_m * num_n * args.splits;
+  const int first_tile = PAIR ? static_cast<int>(blockIdx.x >> 1) : static_cast<int>(blockIdx.x);
+  const int tile_step = PAIR ? static_cast<int>(gridDim.x >> 1) : static_cast<int>(gridDim.x);
+  // the producer's record of the stages it loaded and their phases (for the wind-down)
+  uint32_t issued = 0, issued_par = 0;
 
   if (warp == 0) {
     if (lane == 0) {
       int stage = 0;
-      uint32_t phase = 0, issued = 0, issued_par = 0;
+      uint32_t phase = 0;
+      // A stage's barrier expects the bytes of every load into it: this CTA's, or for a
+      // pair both CTAs' (only the even CTA's barrier is armed; the odd CTA's loads report
+      // to it).
+      auto expect = [&](int st) {
+        if (!PAIR || rank == 0) mbar_arrive_expect_tx(&full[st], PAIR ? 2 * C::STAGE_BYTES : C::STAGE_BYTES);
+      };
+      auto load_a = [&](int st, int kb, int mrow) {
+        if constexpr (PAIR)
+          tma_load_2d_pair(sA + st * C::A_BYTES, &tmA, mapa_shared(smem_u32(&full[st]), 0), kb * C::BK, mrow);
+        else
+          tma_load_2d(sA + st * C::A_BYTES, &tmA, &full[st], kb * C::BK, mrow);
+      };
+      auto load_b = [&](int st, int kb, int n) {
+        if constexpr (PAIR)
+          tma_load_2d_pair(sB + st * C::B_BYTES, &tmB, mapa_shared(smem_u32(&full[st]), 0), kb * C::BK,
+                           n * BN + static_cast<int>(rank) * C::BNL);
+        else
+          tma_load_2d(sB + st * C::B_BYTES, &tmB, &full[st], kb * C::BK, n * BN);
+      };
       // The weights do not depend on the previous kernel: the W tiles of the first stages
       // of this CTA's first tile go out before the wait (the stages start empty), their
       // A tiles after it, completing the same barriers.
-      const int tile0 = blockIdx.x;
+      const int tile0 = first_tile;
       int pre = 0;
       if (tile0 < num_tiles) {
         const int sp0 = tile0 % args.splits, n0 = (tile0 / args.splits) % num_n;
         pre = kb_per < C::STAGES ? kb_per : C::STAGES;
         for (int i = 0; i < pre; ++i) {
-          mbar_arrive_expect_tx(&full[i], C::STAGE_BYTES);
-          tma_load_2d(sB + i * C::B_BYTES, &tmB, &full[i], (sp0 * kb_per + i) * C::BK, n0 * BN);
+          expect(i);
+          load_b(i, sp0 * kb_per + i, n0);
         }
       }
       pdl_wait();
-      for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
+      for (int tile = first_tile; tile < num_tiles; tile += tile_step) {
         const int sp = tile % args.splits;
         const int rest = tile / args.splits;
         const int n = rest % num_n, m = rest / num_n;
+        const int mrow = PAIR ? (2 * m + static_cast<int>(rank)) * C::BM : m * C::BM;
         for (int i = 0; i < kb_per; ++i) {
           const int kb = sp * kb_per + i;
           if (tile == tile0 && i < pre) {  // stage i already expects its bytes; W is in flight
-            tma_load_2d(sA + stage * C::A_BYTES, &tmA, &full[stage], kb * C::BK, m * C::BM);
+            load_a(stage, kb, mrow);
           } else {
             if (!mbar_wait(&empty[stage], phase ^ 1, guard)) goto producer_done;
-            mbar_arrive_expect_tx(&full[stage], C::STAGE_BYTES);
-            tma_load_2d(sA + stage * C::A_BYTES, &tmA, &full[stage], kb * C::BK, m * C::BM);
-            tma_load_2d(sB + stage * C::B_BYTES, &tmB, &full[stage], kb * C::BK, n * BN);
+            expect(stage);
+            load_a(stage, kb, mrow);
+            load_b(stage, kb, n);
           }
           issued |= 1u << stage;
           issued_par = (issued_par & ~(1u << stage)) | (phase << stage);
@@ -194,20 +243,16 @@ __global__ void __launch_bounds__(192, 1)
           }
         }
       }
-    producer_done:
-      if (*abort_flag) {  // let every load this CTA issued land before the CTA exits
-        for (int s = 0; s < C::STAGES; ++s)
-          if (issued & (1u << s)) drain_wait(&full[s], (issued_par >> s) & 1, args.limit_ns);
-      }
+    producer_done:;
     }
   } else if (warp == 1) {
-    if (lane == 0) {
-      constexpr uint32_t IDESC = idesc_bf16(128, BN, false, false);
+    if (lane == 0 && rank == 0) {  // pairs: the even CTA issues for both
+      constexpr uint32_t IDESC = idesc_bf16(PAIR ? 256 : 128, BN, false, false);
       int stage = 0;
       uint32_t phase = 0, acc = 0, acc_phase = 0;
       bool any_mma = false;
-      for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
-        if (!mbar_wait(&tempty[acc], acc_phase ^ 1, guard)) break;
+      for (int tile = first_tile; tile < num_tiles; tile += tile_step) {
+        if (!mbar_wait<PAIR>(&tempty[acc], acc_phase ^ 1, guard)) break;
         tc_fence_after();
         const uint32_t d = tmem_base + acc * BN;
         bool ok = true;
@@ -220,10 +265,18 @@ __global__ void __launch_bounds__(192, 1)
           const uint32_t a0 = smem_u32(sA + stage * C::A_BYTES);
           const uint32_t b0 = smem_u32(sB + stage * C::B_BYTES);
 #pragma unroll
-          for (int kk = 0; kk < C::BK / 16; ++kk)
-            umma_ss(d, sdesc_kmajor_sw128(a0 + kk * 32), sdesc_kmajor_sw128(b0 + kk * 32), IDESC,
-                    (i | kk) != 0);
-          umma_commit(&empty[stage]);
+          for (int kk = 0; kk < C::BK / 16; ++kk) {
+            if constexpr (PAIR)
+              umma_ss_pair(d, sdesc_kmajor_sw128(a0 + kk * 32), sdesc_kmajor_sw128(b0 + kk * 32), IDESC,
+                           (i | kk) != 0);
+            else
+              umma_ss(d, sdesc_kmajor_sw128(a0 + kk * 32), sdesc_kmajor_sw128(b0 + kk * 32), IDESC,
+                      (i | kk) != 0);
+          }
+          if constexpr (PAIR)
+            umma_commit_pair(&empty[stage]);  // frees the stage in both CTAs
+          else
+            umma_commit(&empty[stage]);
           any_mma = true;
           if (++stage == C::STAGES) {
             stage = 0;
@@ -231,13 +284,19 @@ __global__ void __launch_bounds__(192, 1)
           }
         }
         if (!ok) break;
-        umma_commit(&tfull[acc]);
+        if constexpr (PAIR)
+          umma_commit_pair(&tfull[acc]);  // both CTAs' epilogues
+        else
+          umma_commit(&tfull[acc]);
         acc ^= 1;
         if (acc == 0) acc_phase ^= 1;
       }
       if (*abort_flag && any_mma) {  // one more commit covers every MMA issued so far
-        umma_commit(drain);
-        drain_wait(drain, 0, args.limit_ns);
+        if constexpr (PAIR)
+          umma_commit_pair(drain);
+        else
+          umma_commit(drain);
+        drain_wait(drain, 0);
       }
     }
   } else {
@@ -246,6 +305,17 @@ __global__ void __launch_bounds__(192, 1)
     pdl_wait();  // outputs (and the RoPE table) are shared with earlier kernels
     const int quarter = warp & 3;
     uint32_t acc = 0, acc_phase = 0;
+    // This warp has read its lanes of accumulator a: every thread arrives (one CTA), or
+    // for a pair one lane per warp arrives on the even CTA's barrier.
+    auto release_acc = [&](uint32_t a) {
+      tc_fence_before();
+      if constexpr (PAIR) {
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&tempty[a]), 0));
+      } else {
+        mbar_arrive(&tempty[a]);
+      }
+    };
     if constexpr (C::QKV) {
       // Per head: stage the 32 x 128 accumulator block in shared memory, then walk its
       // rows with the lanes across the columns (lane l holds columns 4l .. 4l + 3): the
@@ -261,9 +331,9 @@ __global__ void __launch_bounds__(192, 1)
         c1 = __ldg(reinterpret_cast<const float4*>(args.rope_cs + 64) + q4);
         s1 = __ldg(reinterpret_cast<const float4*>(args.rope_cs + (args.rope_rows + 1) * 64) + q4);
       }
-      for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
+      for (int tile = first_tile; tile < num_tiles; tile += tile_step) {
         const int rest = tile / args.splits;
-        const int n = rest % num_n, m = rest / num_n;
+        const int n = rest % num_n, m = PAIR ? 2 * (rest / num_n) + static_cast<int>(rank) : rest / num_n;
         if (!mbar_wait_warp(&tfull[acc], acc_phase, guard)) break;
         tc_fence_after();
         const int64_t row0 = static_cast<int64_t>(m) * C::BM + quarter * 32;
@@ -297,10 +367,7 @@ __global__ void __launch_bounds__(192, 1)
             }
             stage_chunk<128>(scr, lane, cc, r);
           }
-          if (hb == BN / 128 - 1) {  // accumulator no longer needed
-            tc_fence_before();
-            mbar_arrive(&tempty[acc]);
-          }
+          if (hb == BN / 128 - 1) release_acc(acc);  // accumulator no longer needed
           inv_row[lane] = 1.0f / sqrtf(ss * (1.0f / kHeadDim) + 1e-6f);
           __syncwarp();
           __nv_bfloat16* base = sec == 0 ? args.q : (sec == 1 ? args.k : args.v);
@@ -376,10 +443,10 @@ __global__ void __launch_bounds__(192, 1)
       // fp32 residual stream, while the warp moves on to the next chunk.
       uint8_t* stg = reinterpret_cast<uint8_t*>(scratch) + (warp - 2) * 8192;
       uint32_t kbuf = 0;
-      for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
+      for (int tile = first_tile; tile < num_tiles; tile += tile_step) {
         const int sp = tile % args.splits;
         const int rest = tile / args.splits;
-        const int n = rest % num_n, m = rest / num_n;
+        const int n = rest % num_n, m = PAIR ? 2 * (rest / num_n) + static_cast<int>(rank) : rest / num_n;
         if (!mbar_wait_warp(&tfull[acc], acc_phase, guard)) break;
         tc_fence_after();
         const int y = m * C::BM + quarter * 32;
@@ -395,10 +462,7 @@ __global__ void __launch_bounds__(192, 1)
           tmem_ld32(taddr + c, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
           if constexpr (C::CW == 64) tmem_ld32(taddr + c + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
           tmem_wait_ld();
-          if (c + C::CW == BN) {  // accumulator no longer needed
-            tc_fence_before();
-            mbar_arrive(&tempty[acc]);
-          }
+          if (c + C::CW == BN) release_acc(acc);  // accumulator no longer needed
           const int col0 = n * BN + c;
           const bool add_bias = !(EPI == SAL_EPI_RESID_F32 && sp != 0);
           const uint4* bias8 = reinterpret_cast<const uint4*>(args.bias + col0);
@@ -475,10 +539,41 @@ __global__ void __launch_bounds__(192, 1)
 
   tc_fence_before();
   __syncthreads();
+  // Every role has finished, so the abort flag is final. After an abort some loads may
+  // have been issued that no consumer waited for: let each land before the CTA, and its
+  // shared memory, goes away. Thread 0 is the producer thread.
+  if constexpr (PAIR) {
+    // Neither CTA of a pair frees its TMEM or leaves while the other may still reach it.
+    // The odd CTA's loads and epilogue arrivals report to the even CTA; the even CTA's MMAs
+    // read the odd CTA's shared memory and write its TMEM (drained by the MMA thread before
+    // the barrier above). So: the odd CTA says it is done, the even CTA waits for that,
+    // drains the loads it armed (both CTAs' bytes), says goodbye, and only then does the
+    // odd CTA free its TMEM and leave. Every wait is bounded; the odd CTA's outlasts the
+    // even CTA's drains.
+    if (threadIdx.x == 0) {
+      if (rank == 1) {
+        mbar_arrive_cluster(mapa_shared(smem_u32(bye), 0));
+        drain_wait(bye, 0, (C::STAGES + 2) * kDrainLimitNs);
+      } else {
+        drain_wait(bye, 0);
+        if (*abort_flag)
+          for (int s = 0; s < C::STAGES; ++s)
+            if (issued & (1u << s)) drain_wait(&full[s], (issued_par >> s) & 1);
+        mbar_arrive_cluster(mapa_shared(smem_u32(bye), 1));
+      }
+    }
+    __syncthreads();
+  } else if (threadIdx.x == 0 && *abort_flag) {
+    for (int s = 0; s < C::STAGES; ++s)
+      if (issued & (1u << s)) drain_wait(&full[s], (issued_par >> s) & 1);
+  }
   if (warp == 1) {
     __syncwarp();
     tc_fence_after();
-    tmem_dealloc(tmem_base, C::TMEM_COLS);
+    if constexpr (PAIR)
+      tmem_dealloc_pair(tmem_base, C::TMEM_COLS);
+    else
+      tmem_dealloc(tmem_base, C::TMEM_COLS);
   }
 }
 
@@ -498,16 +593,16 @@ int num_sms() {
   return g_num_sms[dev];
 }
 
-template <int BN, int EPI>
+template <int BN, int EPI, bool PAIR = false>
 sal_status launch_bn(const GemmArgs& a, const void* A, const void* W, cudaStream_t s) {
-  using C = Cfg<BN, EPI>;
+  using C = Cfg<BN, EPI, PAIR>;
   static bool attr_done[64] = {};
   int dev = 0;
   cudaGetDevice(&dev);
   {
     std::lock_guard<std::mutex> lk(g_mu);
     if (dev >= 0 && dev < 64 && !attr_done[dev]) {
-      if (cudaFuncSetAttribute(gemm_kernel<BN, EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+      if (cudaFuncSetAttribute(gemm_kernel<BN, EPI, PAIR>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                static_cast<int>(C::SMEM)) != cudaSuccess)
         return SAL_ECUDA;
       attr_done[dev] = true;
@@ -515,7 +610,8 @@ sal_status launch_bn(const GemmArgs& a, const void* A, const void* W, cudaStream
   }
   CUtensorMap ta, tb, tc;
   if (!make_tmap_2d_bf16(&ta, A, a.K, a.M, C::BK, C::BM)) return SAL_ECUDA;
-  if (!make_tmap_2d_bf16(&tb, W, a.K, a.n_valid, C::BK, BN)) return SAL_ECUDA;  // rows >= n_valid: zeros
+  // rows >= n_valid read as zeros; a pair's CTAs each load BN / 2 rows
+  if (!make_tmap_2d_bf16(&tb, W, a.K, a.n_valid, C::BK, C::BNL)) return SAL_ECUDA;
   if constexpr (C::QKV) {
     tc = ta;  // unused
   } else if constexpr (C::F32_OUT) {
@@ -523,15 +619,27 @@ sal_status launch_bn(const GemmArgs& a, const void* A, const void* W, cudaStream
   } else {
     if (!make_tmap_2d_bf16(&tc, a.out, a.N, a.M, C::CW, 32)) return SAL_ECUDA;
   }
-  const int tiles = static_cast<int>((a.M + C::BM - 1) / C::BM) * (a.N / BN) * a.splits;
-  const int grid = tiles < num_sms() ? tiles : num_sms();
-  return launch_kernel(gemm_kernel<BN, EPI>, dim3(grid), dim3(192), C::SMEM, s, ta, tb, tc, a) == cudaSuccess
-             ? SAL_OK
-             : SAL_ECUDA;
+  if constexpr (PAIR) {
+    // one cluster of two CTAs per pair of SMs, walking 256-row work units
+    const int units = static_cast<int>((a.M + 2 * C::BM - 1) / (2 * C::BM)) * (a.N / BN) * a.splits;
+    const int pairs = units < num_sms() / 2 ? units : num_sms() / 2;
+    return launch_kernel_cluster(gemm_kernel<BN, EPI, true>, dim3(2 * pairs), dim3(192), C::SMEM, s, 2u, ta, tb,
+                                 tc, a) == cudaSuccess
+               ? SAL_OK
+               : SAL_ECUDA;
+  } else {
+    const int tiles = static_cast<int>((a.M + C::BM - 1) / C::BM) * (a.N / BN) * a.splits;
+    const int grid = tiles < num_sms() ? tiles : num_sms();
+    return launch_kernel(gemm_kernel<BN, EPI, false>, dim3(grid), dim3(192), C::SMEM, s, ta, tb, tc, a) ==
+                   cudaSuccess
+               ? SAL_OK
+               : SAL_ECUDA;
+  }
 }
 
 template <int EPI>
-sal_status launch_epi(int BN, const GemmArgs& a, const void* A, const void* W, cudaStream_t s) {
+sal_status launch_epi(int BN, bool pair, const GemmArgs& a, const void* A, const void* W, cudaStream_t s) {
+  if (pair) return BN == 256 ? launch_bn<256, EPI, true>(a, A, W, s) : SAL_ESHAPE;
   if constexpr (EPI == kEpiQkv) {  // one or two heads per tile
     return BN == 256 ? launch_bn<256, EPI>(a, A, W, s) : (BN == 128 ? launch_bn<128, EPI>(a, A, W, s) : SAL_ESHAPE);
   } else {
@@ -555,6 +663,18 @@ int pick_bn(int64_t M, int N, bool qkv) {
   if (N % 256 == 0 && mt * (N / 256) >= num_sms()) return 256;
   if (N % 128 == 0) return 128;
   return 64;
+}
+
+// CTA pairs (256 x 256 work units over two SMs) for 256-wide tiles without a K split, once
+// the pairs' units alone fill every pair of SMs. SAL_GEMM_PAIR=0 / 1 in the environment
+// forces them off / on (where the shape allows them), for measurement.
+bool use_pair(int64_t M, int N, int BN, int splits) {
+  static const int mode = [] {
+    const char* e = std::getenv("SAL_GEMM_PAIR");
+    return e && e[0] == '0' ? 0 : (e && e[0] == '1' ? 1 : -1);
+  }();
+  if (mode != 1 || BN != 256 || splits != 1 || N % 256) return false;
+  return (M + 255) / 256 * (N / 256) >= 1;
 }
 
 }  // namespace
@@ -602,12 +722,13 @@ sal_status gemm_launch(int epilogue, const void* A, int64_t M, int K, const void
            a.splits < 8)
       a.splits *= 2;
   }
+  const bool pair = use_pair(M, N, BN, a.splits);
   switch (epilogue) {
-    case SAL_EPI_STORE_F32: return launch_epi<SAL_EPI_STORE_F32>(BN, a, A, W, s);
-    case SAL_EPI_STORE_BF16: return launch_epi<SAL_EPI_STORE_BF16>(BN, a, A, W, s);
-    case SAL_EPI_GELU_BF16: return launch_epi<SAL_EPI_GELU_BF16>(BN, a, A, W, s);
-    case SAL_EPI_RESID_F32: return launch_epi<SAL_EPI_RESID_F32>(BN, a, A, W, s);
-    case kEpiQkv: return launch_epi<kEpiQkv>(BN, a, A, W, s);
+    case SAL_EPI_STORE_F32: return launch_epi<SAL_EPI_STORE_F32>(BN, pair, a, A, W, s);
+    case SAL_EPI_STORE_BF16: return launch_epi<SAL_EPI_STORE_BF16>(BN, pair, a, A, W, s);
+    case SAL_EPI_GELU_BF16: return launch_epi<SAL_EPI_GELU_BF16>(BN, pair, a, A, W, s);
+    case SAL_EPI_RESID_F32: return launch_epi<SAL_EPI_RESID_F32>(BN, pair, a, A, W, s);
+    case kEpiQkv: return launch_epi<kEpiQkv>(BN, pair, a, A, W, s);
     default: return SAL_EINVAL;
   }
 }

@@ -16,6 +16,12 @@
 // speaker kernel K[s, 2i] = sin(s w_i), K[s, 2i+1] = cos(s w_i), w_i = 10000^(-2i/1280)
 // (scale 1), and added to the encoder state. One warp per position; K (40 KB, built in
 // fp64 on the host) sits in shared memory.
+//
+// Serving windows (section "Local encoder windows, recording-wide language context", the
+// paragraph on the serving path): the gather copies each context-extended window of a
+// recording's residual stream into its own left-aligned slot range of a windowed batch
+// (zeroing the slots past the window's length); the scatter copies every window's core
+// rows back in order, dropping the context rows. One warp per row, 16-byte accesses.
 #include <cuda_bf16.h>
 #include <math.h>
 
@@ -161,6 +167,59 @@ __global__ void __launch_bounds__(256) speaker_fuse_kernel(const __nv_bfloat16* 
   }
 }
 
+// First position of window w of a recording.
+__device__ __forceinline__ int64_t window_lo(const Windows& wn, int64_t w) {
+  const int64_t lo = w * wn.core - wn.ctx;
+  return lo > 0 ? lo : 0;
+}
+
+__global__ void __launch_bounds__(256) window_gather_kernel(const float* __restrict__ x, int batch, Windows wn,
+                                                            float* __restrict__ xw) {
+  const int lane = threadIdx.x & 31;
+  const int64_t rows = static_cast<int64_t>(batch) * wn.count * wn.slot;
+  const int64_t row = static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5);
+  pdl_wait();
+  pdl_trigger();
+  if (row >= rows) return;
+  const int64_t clip = row / wn.slot, i = row - clip * wn.slot;
+  const int64_t b = clip / wn.count, w = clip - b * wn.count;
+  const int64_t lo = window_lo(wn, w);
+  int64_t hi = (w + 1) * wn.core + wn.ctx;
+  if (hi > wn.total) hi = wn.total;
+  float4* dst = reinterpret_cast<float4*>(xw + row * kWidth);
+  if (lo + i < hi) {
+    const float4* src = reinterpret_cast<const float4*>(x + (b * wn.total + lo + i) * kWidth);
+#pragma unroll
+    for (int c = 0; c < kWidth / 128; ++c) dst[lane + 32 * c] = src[lane + 32 * c];
+  } else {
+#pragma unroll
+    for (int c = 0; c < kWidth / 128; ++c) dst[lane + 32 * c] = make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+}
+
+__global__ void __launch_bounds__(256) window_scatter_kernel(const __nv_bfloat16* __restrict__ embw,
+                                                             const float* __restrict__ xw, int batch, Windows wn,
+                                                             __nv_bfloat16* __restrict__ emb, float* __restrict__ x) {
+  const int lane = threadIdx.x & 31;
+  const int64_t rows = static_cast<int64_t>(batch) * wn.total;
+  const int64_t row = static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5);
+  pdl_wait();
+  pdl_trigger();
+  if (row >= rows) return;
+  const int64_t b = row / wn.total, t = row - b * wn.total;
+  const int64_t w = t / wn.core;  // the window whose core holds position t
+  const int64_t src_row = (b * wn.count + w) * wn.slot + (t - window_lo(wn, w));
+  const uint4* se = reinterpret_cast<const uint4*>(embw + src_row * kWidth);
+  uint4* de = reinterpret_cast<uint4*>(emb + row * kWidth);
+  for (int c = lane; c < kWidth / 8; c += 32) de[c] = se[c];
+  if (x) {
+    const float4* sx = reinterpret_cast<const float4*>(xw + src_row * kWidth);
+    float4* dx = reinterpret_cast<float4*>(x + row * kWidth);
+#pragma unroll
+    for (int c = 0; c < kWidth / 128; ++c) dx[lane + 32 * c] = sx[lane + 32 * c];
+  }
+}
+
 std::mutex g_spk_mu;
 bool g_spk_done[64] = {};
 
@@ -219,6 +278,26 @@ sal_status layernorm_launch(const float* x, int64_t rows, const void* g, const v
   else
     return SAL_ESHAPE;
   return e == cudaSuccess ? SAL_OK : SAL_ECUDA;
+}
+
+sal_status window_gather_launch(const float* x, int batch, const Windows& win, float* xw, cudaStream_t s) {
+  const int64_t rows = static_cast<int64_t>(batch) * win.count * win.slot;
+  if (rows == 0) return SAL_OK;
+  return launch_kernel(window_gather_kernel, dim3(static_cast<unsigned>((rows + 7) / 8)), dim3(256), 0, s, x, batch,
+                       win, xw) == cudaSuccess
+             ? SAL_OK
+             : SAL_ECUDA;
+}
+
+sal_status window_scatter_launch(const void* embw, const float* xw, int batch, const Windows& win, void* emb,
+                                 float* x, cudaStream_t s) {
+  const int64_t rows = static_cast<int64_t>(batch) * win.total;
+  if (rows == 0) return SAL_OK;
+  return launch_kernel(window_scatter_kernel, dim3(static_cast<unsigned>((rows + 7) / 8)), dim3(256), 0, s,
+                       static_cast<const __nv_bfloat16*>(embw), xw, batch, win, static_cast<__nv_bfloat16*>(emb),
+                       x) == cudaSuccess
+             ? SAL_OK
+             : SAL_ECUDA;
 }
 
 sal_status rope_table_launch(float* cs, int64_t T, cudaStream_t s) {

@@ -150,6 +150,23 @@ bool is_device_ptr(const void* p) {
 
 uint64_t wait_limit_ns() { return g_wait_limit_ns.load(); }
 
+Windows make_windows(int64_t total, int64_t core, int64_t ctx) {
+  Windows wn;
+  if (total <= 0 || core <= 0) return wn;
+  if (core > total) core = total;  // one window: the whole clip
+  if (ctx > total) ctx = total;    // context past the clip ends is clipped anyway
+  if (ctx < 0) ctx = 0;
+  wn.count = static_cast<int>((total + core - 1) / core);
+  wn.core = static_cast<int>(core);
+  wn.ctx = static_cast<int>(ctx);
+  wn.total = total;
+  for (int64_t w = 0; w < wn.count; ++w) {
+    const int64_t lo = std::max<int64_t>(0, w * core - ctx), hi = std::min<int64_t>(total, (w + 1) * core + ctx);
+    wn.slot = std::max(wn.slot, hi - lo);
+  }
+  return wn;
+}
+
 void count_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
 
 bool pdl_enabled() {
@@ -283,6 +300,24 @@ size_t sal_encoder_workspace_bytes(int batch, int64_t T) {
   return encoder_ws_layout(nullptr, batch, T).bytes;
 }
 
+namespace {
+bool windowed(const sal_forward_options* o) { return o && o->window_core > 0; }
+
+// Workspace of a windowed forward: the windowed fp32 stream and bf16 embeddings, then the
+// encoder workspace of the windowed batch.
+size_t windowed_ws_bytes(int batch, const Windows& wn) {
+  const size_t rows = static_cast<size_t>(batch) * wn.count * static_cast<size_t>(wn.slot);
+  return align256(rows * kWidth * 4) + align256(rows * kWidth * 2) +
+         encoder_ws_layout(nullptr, batch * wn.count, wn.slot).bytes;
+}
+}  // namespace
+
+size_t sal_encoder_workspace_bytes_ex(int batch, int64_t T, const sal_forward_options* opts) {
+  if (batch <= 0 || T <= 0) return 0;
+  if (!windowed(opts)) return sal_encoder_workspace_bytes(batch, T);
+  return windowed_ws_bytes(batch, make_windows(T, opts->window_core, opts->window_context));
+}
+
 sal_status sal_encoder_forward(float* x, int batch, int64_t T, const sal_weights* w, int n_layers, void* emb,
                                void* workspace, size_t ws_bytes, void* stream) {
   return sal_encoder_forward_ex(x, batch, T, w, n_layers, emb, workspace, ws_bytes, stream, nullptr);
@@ -317,11 +352,37 @@ struct Tracer {
     if (!tr.after(kind)) return SAL_ECUDA;                  \
   } while (0)
 
+namespace {
+// The layer sequence over `batch` clips of T positions, then the final LayerNorm into emb.
+// `win`: the clips are serving windows (attention only over each window's own length).
+sal_status run_layers(float* x, int batch, int64_t T, const sal_weights* w, int n_layers, void* emb,
+                      const EncoderWs& ws, int64_t chunk, const Windows* win, Tracer& tr, cudaStream_t s) {
+  const int64_t M = static_cast<int64_t>(batch) * T;
+  if (n_layers > 0) SAL_TRACED(SAL_KIND_ROPE_TABLE, rope_table_launch(ws.rope, chunk, s));
+  for (int i = 0; i < n_layers; ++i) {
+    const sal_layer& L = w->layers[i];
+    SAL_TRACED(SAL_KIND_LAYERNORM, layernorm_launch(x, M, L.ln1_g, L.ln1_b, ws.h, s));
+    QkvOut qo{ws.q, ws.k, ws.v, L.qn_g, L.kn_g, ws.rope, T, chunk};
+    SAL_TRACED(SAL_KIND_QKV, gemm_launch(kEpiQkv, ws.h, M, kWidth, L.w_qkv, 3 * kWidth, L.b_qkv, nullptr, &qo, s));
+    SAL_TRACED(SAL_KIND_ATTENTION, attention_launch(ws.q, ws.k, ws.v, batch, T, chunk, ws.o, s, win));
+    SAL_TRACED(SAL_KIND_OUT_PROJ,
+               gemm_launch(SAL_EPI_RESID_F32, ws.o, M, kWidth, L.w_o, kWidth, L.b_o, x, nullptr, s));
+    SAL_TRACED(SAL_KIND_LAYERNORM, layernorm_launch(x, M, L.ln2_g, L.ln2_b, ws.h, s));
+    SAL_TRACED(SAL_KIND_FFN_UP, gemm_launch(SAL_EPI_GELU_BF16, ws.h, M, kWidth, L.w1, kFfn, L.b1, ws.u, nullptr, s));
+    SAL_TRACED(SAL_KIND_FFN_DOWN,
+               gemm_launch(SAL_EPI_RESID_F32, ws.u, M, kFfn, L.w2, kWidth, L.b2, x, nullptr, s));
+  }
+  SAL_TRACED(SAL_KIND_LAYERNORM, layernorm_launch(x, M, w->lnf_g, w->lnf_b, emb, s));
+  return SAL_OK;
+}
+}  // namespace
+
 sal_status sal_encoder_forward_ex(float* x, int batch, int64_t T, const sal_weights* w, int n_layers, void* emb,
                                   void* workspace, size_t ws_bytes, void* stream, const sal_forward_options* opts) {
   const sal_trace* trace = opts ? opts->trace : nullptr;
   const int64_t chunk = (opts && opts->chunk > 0 && opts->chunk < T) ? opts->chunk : T;
   if (batch < 0 || T < 0 || !w || n_layers < 0 || n_layers > w->n_layers) return SAL_EINVAL;
+  if (windowed(opts) && (opts->chunk > 0 || opts->window_context < 0)) return SAL_EINVAL;
   if (T > SAL_MAX_POSITIONS) return SAL_ESHAPE;
   if (batch == 0 || T == 0) return SAL_OK;
   if (batch > 6553) return SAL_ESHAPE;  // attention grid.y = 10 * batch
@@ -334,28 +395,31 @@ sal_status sal_encoder_forward_ex(float* x, int batch, int64_t T, const sal_weig
   if (trace && (trace->kind < 0 || trace->kind >= SAL_KIND_COUNT || trace->n_events < 0 ||
                 (trace->n_events > 0 && !trace->events)))
     return SAL_EINVAL;
-  const EncoderWs ws = encoder_ws_layout(workspace, batch, T);
-  if (ws_bytes < ws.bytes) return SAL_EWORKSPACE;
-  SAL_TRY(check_device());
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   Tracer tr{trace, s};
-  const int64_t M = static_cast<int64_t>(batch) * T;
-  if (n_layers > 0) SAL_TRACED(SAL_KIND_ROPE_TABLE, rope_table_launch(ws.rope, chunk, s));
-  for (int i = 0; i < n_layers; ++i) {
-    const sal_layer& L = w->layers[i];
-    SAL_TRACED(SAL_KIND_LAYERNORM, layernorm_launch(x, M, L.ln1_g, L.ln1_b, ws.h, s));
-    QkvOut qo{ws.q, ws.k, ws.v, L.qn_g, L.kn_g, ws.rope, T, chunk};
-    SAL_TRACED(SAL_KIND_QKV, gemm_launch(kEpiQkv, ws.h, M, kWidth, L.w_qkv, 3 * kWidth, L.b_qkv, nullptr, &qo, s));
-    SAL_TRACED(SAL_KIND_ATTENTION, attention_launch(ws.q, ws.k, ws.v, batch, T, chunk, ws.o, s));
-    SAL_TRACED(SAL_KIND_OUT_PROJ,
-               gemm_launch(SAL_EPI_RESID_F32, ws.o, M, kWidth, L.w_o, kWidth, L.b_o, x, nullptr, s));
-    SAL_TRACED(SAL_KIND_LAYERNORM, layernorm_launch(x, M, L.ln2_g, L.ln2_b, ws.h, s));
-    SAL_TRACED(SAL_KIND_FFN_UP, gemm_launch(SAL_EPI_GELU_BF16, ws.h, M, kWidth, L.w1, kFfn, L.b1, ws.u, nullptr, s));
-    SAL_TRACED(SAL_KIND_FFN_DOWN,
-               gemm_launch(SAL_EPI_RESID_F32, ws.u, M, kFfn, L.w2, kWidth, L.b2, x, nullptr, s));
+  if (!windowed(opts)) {
+    const EncoderWs ws = encoder_ws_layout(workspace, batch, T);
+    if (ws_bytes < ws.bytes) return SAL_EWORKSPACE;
+    SAL_TRY(check_device());
+    return run_layers(x, batch, T, w, n_layers, emb, ws, chunk, nullptr, tr, s);
   }
-  SAL_TRACED(SAL_KIND_LAYERNORM, layernorm_launch(x, M, w->lnf_g, w->lnf_b, emb, s));
-  return SAL_OK;
+  // Serving windows: gather every window into its own slots of a windowed batch, run the
+  // layers on it as independent sequences, scatter the core rows back.
+  const Windows wn = make_windows(T, opts->window_core, opts->window_context);
+  const int64_t bw = static_cast<int64_t>(batch) * wn.count;
+  if (bw > 6553) return SAL_ESHAPE;  // attention grid.y = 10 * windows
+  if (ws_bytes < windowed_ws_bytes(batch, wn)) return SAL_EWORKSPACE;
+  SAL_TRY(check_device());
+  const size_t rows = static_cast<size_t>(bw) * static_cast<size_t>(wn.slot);
+  char* p = static_cast<char*>(workspace);
+  float* xw = reinterpret_cast<float*>(p);
+  p += align256(rows * kWidth * 4);
+  void* embw = p;
+  p += align256(rows * kWidth * 2);
+  const EncoderWs ws = encoder_ws_layout(p, static_cast<int>(bw), wn.slot);
+  SAL_TRY(window_gather_launch(x, batch, wn, xw, s));
+  SAL_TRY(run_layers(xw, static_cast<int>(bw), wn.slot, w, n_layers, embw, ws, wn.slot, &wn, tr, s));
+  return window_scatter_launch(embw, xw, batch, wn, emb, x, s);
 }
 
 uint64_t sal_launch_count(void) { return g_launches.load(); }

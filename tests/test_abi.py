@@ -59,6 +59,21 @@ def test_workspace_sizes(api):
     assert lib.sal_encode_workspace_bytes(1, 480000) > lib.sal_encoder_workspace_bytes(1, 374)
 
 
+def test_windowed_workspace_sizes(api):
+    """Serving windows: the windowed fp32 stream and bf16 embeddings over every window's
+    slots, plus the encoder workspace of the windowed batch; no windows: the plain size."""
+    lib = api.lib()
+    plain = lib.sal_encoder_workspace_bytes(1, 44999)
+    assert lib.sal_encoder_workspace_bytes_ex(1, 44999, None) == plain
+    none = api.sal_forward_options(375, None, 0, 0)
+    assert lib.sal_encoder_workspace_bytes_ex(1, 44999, ctypes.byref(none)) == plain
+    o = api.sal_forward_options(0, None, 500, 50)
+    rows = 90 * 600  # 90 windows, the longest 600 positions
+    assert lib.sal_encoder_workspace_bytes_ex(1, 44999, ctypes.byref(o)) == (
+        rows * 1280 * 6 + lib.sal_encoder_workspace_bytes(90, 600))
+    assert lib.sal_encoder_workspace_bytes_ex(0, 44999, ctypes.byref(o)) == 0
+
+
 def test_argument_checks_before_any_cuda_call(api):
     lib = api.lib()
     assert lib.sal_frontend(0, 1000, -1, 0, 0, 0) == 1          # negative batch
@@ -93,7 +108,12 @@ def test_ctc_adapter_host_checks(api):
 def test_attention_plan_matches_the_stated_schedule(api):
     """The library's split of query tiles between the two attention kernels equals the
     rule its header states (list scheduling, written out in the GPU tests), over clip
-    lengths and batch sizes on both sides of every threshold."""
+    lengths and batch sizes on both sides of every threshold.
+
+    SAL_ATTN_PP in the environment forces the split (the library reads it once per
+    process), so the stated rule is only checked when it is unset."""
+    if os.environ.get("SAL_ATTN_PP"):
+        pytest.skip("SAL_ATTN_PP forces the split in this process")
     from test_gpu_kernels import _pairs_for_two_tile_kernel
     cases = [(b, T) for b in (1, 2, 8, 16, 30) for T in (1, 129, 749, 1000, 2000, 2047, 2048, 3000)]
     cases += [(b, T) for b in (1, 2) for T in (5000, 7499, 12000, 20000, 44999)]
@@ -101,3 +121,14 @@ def test_attention_plan_matches_the_stated_schedule(api):
         assert api.attention_plan(batch, T) == _pairs_for_two_tile_kernel(batch, T), (batch, T)
     assert api.attention_plan(1, 20000, heads=16, head_dim=64) == (0, 157)  # 64-wide heads: one-tile
     assert api.attention_plan(0, 100) == (0, 1)
+    p, q = ctypes.c_int(), ctypes.c_int()
+    assert api.lib().sal_attention_plan(1, 90001, 10, 128, 148, ctypes.byref(p), ctypes.byref(q)) == 2
+
+
+def test_withhold_hook_argument_checks(api):
+    lib = api.lib()
+    assert lib.sal_attention_withhold(0, 0, 0, 1, 512, 3, 2, 0, 0) == 1    # no such kernel
+    assert lib.sal_attention_withhold(0, 0, 0, 1, 512, 1, -1, 0, 0) == 1   # negative tile
+    assert lib.sal_attention_withhold(0, 0, 0, 1, 45001, 1, 2, 0, 0) == 2  # more than one hour
+    assert lib.sal_attention_withhold(0, 0, 0, 1, 0, 1, 2, 0, 0) == 0      # nothing to do
+    assert lib.sal_attention_withhold(0, 0, 0, 1, 512, 1, 2, 0, 0) == 1    # null pointers

@@ -173,7 +173,12 @@ def test_attention(batch, T, scale):
     q, q64 = rand_bf16((batch, 10, T, 128), 50 + T, scale)
     k, k64 = rand_bf16((batch, 10, T, 128), 60 + T, 1.0)
     v, v64 = rand_bf16((batch, 10, T, 128), 70 + T, 1.0)
+    n0 = api.sal_launch_count()
     o = api.sal_attention(q, k, v)
+    # the launches match the plan: the two-tile kernel and, when it leaves query tiles
+    # over, the one-tile kernel behind it
+    P = expect.get((batch, T), (0, n_qt))[0]
+    assert api.sal_launch_count() - n0 == (2 if 0 < P and 2 * P < n_qt else 1)
     got = to64(o).reshape(batch, T, 10, 128)
     for b in range(batch):
         ref = O.attention(q64[b], k64[b], v64[b]).transpose(1, 0, 2)
