@@ -516,9 +516,10 @@ def _traffic(kind: str, workload: str):
     kernel's source changed since that capture or the capture was of another workload."""
     import hashlib
     try:
-        rec = json.load(open(os.path.join(ROOT, "profiles", "roofline_traffic.json")))[kind]
+        recs = json.load(open(os.path.join(ROOT, "profiles", "roofline_traffic.json")))
+        rec = recs.get(f"{kind}@{workload}", recs.get(kind))
         src = open(os.path.join(ROOT, rec["source"]), "rb").read()
-    except (OSError, KeyError, ValueError):
+    except (OSError, KeyError, ValueError, TypeError, AttributeError):
         return None
     if rec.get("workload") != workload or hashlib.sha256(src).hexdigest()[:16] != rec.get("sha256_16"):
         return None

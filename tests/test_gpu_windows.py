@@ -9,7 +9,7 @@ concatenated; 500 core and 50 context positions by default.
 The oracle takes the GPU's own residual stream x0 (upcast), so the front end is not part
 of the comparison. Bars as for the whole-clip encoder: embeddings within rel-L2 2e-2; the
 residual stream's update x - x0 (core rows, from the window that owns each row) within
-1e-2. Rows at window borders (the last core row of one window and the first of the next)
+1e-2 after one or two layers and 2e-2 after 32. Rows at window borders (the last core row of one window and the first of the next)
 are also checked on their own.
 """
 import numpy as np
