@@ -49,6 +49,11 @@ struct GemmArgs {
   unsigned int* status;
 };
 
+// Epilogue warps of the plain kinds (4 or 8; see Cfg::EPW), a build-time knob for measurement.
+#ifndef SAL_GEMM_EPW
+#define SAL_GEMM_EPW 8
+#endif
+
 // PAIR: a cluster of two CTAs computes a 256 x BN tile with tcgen05.mma.cta_group::2. Each
 // CTA loads its own 128 rows of A and its own BN / 2 rows of W (no multicast), holds its 128
 // rows of the accumulator in its TMEM and runs the epilogue on them; the even CTA issues
@@ -61,7 +66,12 @@ struct Cfg {
   // epilogue shared memory: QKV stages a whole head per warp (32 rows x 128 fp32); the
   // other kinds stage 128-byte-wide output boxes for TMA, two per warp
   static constexpr int CW = F32_OUT ? 32 : 64;  // output columns per 128-byte box row
-  static constexpr int SCR_BYTES = QKV ? 4 * 32 * 128 * 4 + 4 * 32 * 4 : 4 * 2 * 4096;
+  // epilogue warps: four (one per TMEM lane quarter), or eight for the plain kinds of
+  // 128- and 256-wide tiles (two per lane quarter, each on half of the columns, one
+  // staging box each), so that two warps per SM sub-partition hide each other's latency
+  static constexpr int EPW = (QKV || BN < 128) ? 4 : SAL_GEMM_EPW;
+  static constexpr int THREADS = 64 + 32 * EPW;
+  static constexpr int SCR_BYTES = QKV ? 4 * 32 * 128 * 4 + 4 * 32 * 4 : 8 * 4096;
   static constexpr int BNL = PAIR ? BN / 2 : BN;  // rows of W this CTA loads per tile
   static constexpr int STAGES = PAIR ? (QKV ? 5 : 6)
                                      : (QKV ? (BN == 256 ? 3 : 4) : (BN == 256 ? 4 : (BN == 128 ? 6 : 8)));
@@ -74,8 +84,25 @@ struct Cfg {
   static_assert(!PAIR || BN == 256, "CTA pairs use 256-wide tiles");
 };
 
+// Exact-erf GELU 0.5 x (1 + erf(x / sqrt 2)), with erf from the rational approximation of
+// Abramowitz and Stegun, Handbook of Mathematical Functions, formula 7.1.26 (after
+// Hastings): for z >= 0, erf z = 1 - t (a1 + t (a2 + t (a3 + t (a4 + t a5)))) e^(-z^2),
+// t = 1 / (1 + p z), |error| <= 1.5e-7; odd in z. Evaluated in fp32 (reciprocal and
+// exponential on the SFU) it stays within 6e-7 of erf over the whole line, branch-free;
+// the GELU output is then rounded to bf16 (2^-9 relative).
 __device__ __forceinline__ float gelu_erf(float x) {
-  return 0.5f * x * (1.0f + erff(x * 0.70710678118654752f));
+  const float z = fabsf(x) * 0.70710678118654752f;
+  float t;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(t) : "f"(fmaf(0.3275911f, z, 1.0f)));
+  float q = fmaf(1.061405429f, t, -1.453152027f);
+  q = fmaf(q, t, 1.421413741f);
+  q = fmaf(q, t, -0.284496736f);
+  q = fmaf(q, t, 0.254829592f);
+  q *= t;
+  const float e = fast_exp2(-1.4426950408889634f * z * z);
+  const float erf_z = copysignf(fmaf(-q, e, 1.0f), x);  // erf(x / sqrt 2)
+  const float h = 0.5f * x;
+  return fmaf(h, erf_z, h);
 }
 
 __device__ __forceinline__ float bf16_at(const __nv_bfloat16* p, int i) { return __bfloat162float(p[i]); }
@@ -99,14 +126,8 @@ __device__ __forceinline__ void stage_chunk(float4* scr, int lane, int cc, const
                     __uint_as_float(r[4 * i + 3]));
 }
 
-__device__ __forceinline__ float warp_sum(float v) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-  return v;
-}
-
 template <int BN, int EPI, bool PAIR>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(Cfg<BN, EPI, PAIR>::THREADS, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                 const __grid_constant__ CUtensorMap tmC, const GemmArgs args) {
   using C = Cfg<BN, EPI, PAIR>;
@@ -138,7 +159,8 @@ __global__ void __launch_bounds__(192, 1)
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&tfull[a], 1);
-      mbar_init(&tempty[a], PAIR ? 8 : 128);  // pairs: one arrival per epilogue warp of both CTAs
+      // one arrival per epilogue thread; pairs: one per epilogue warp of both CTAs
+      mbar_init(&tempty[a], PAIR ? 2 * C::EPW : 32 * C::EPW);
     }
     mbar_init(drain, 1);
     mbar_init(bye, 1);
@@ -441,7 +463,12 @@ __global__ void __launch_bounds__(192, 1)
       // them into a 128B-swizzled 32-row box in shared memory (two boxes per warp, used in
       // turn); one lane then issues a TMA store of the box, or a TMA reduce-add into the
       // fp32 residual stream, while the warp moves on to the next chunk.
-      uint8_t* stg = reinterpret_cast<uint8_t*>(scratch) + (warp - 2) * 8192;
+      // EPW 4: two boxes per warp, used in turn; EPW 8: one box per warp, and warps
+      // 2-5 / 6-9 take the first / second half of the tile's columns
+      constexpr int kBoxes = C::EPW == 4 ? 2 : 1;
+      uint8_t* stg = reinterpret_cast<uint8_t*>(scratch) + (warp - 2) * kBoxes * 4096;
+      const int c_begin = C::EPW == 4 ? 0 : ((warp - 2) >> 2) * (BN / 2);
+      const int c_end = C::EPW == 4 ? BN : c_begin + BN / 2;
       uint32_t kbuf = 0;
       for (int tile = first_tile; tile < num_tiles; tile += tile_step) {
         const int sp = tile % args.splits;
@@ -452,17 +479,22 @@ __global__ void __launch_bounds__(192, 1)
         const int y = m * C::BM + quarter * 32;
         const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + acc * BN;
 #pragma unroll 1
-        for (int c = 0; c < BN; c += C::CW) {
-          uint8_t* buf = stg + (kbuf & 1) * 4096;
-          if (kbuf >= 2) {  // the store issued from this box two chunks ago has read it
-            if (lane == 0) bulk_wait_read<1>();
+        for (int c = c_begin; c < c_end; c += C::CW) {
+          uint8_t* buf = stg + (kbuf % kBoxes) * 4096;
+          if (kbuf >= kBoxes) {  // the store issued from this box kBoxes chunks ago has read it
+            if (lane == 0) {
+              if constexpr (kBoxes == 2)
+                bulk_wait_read<1>();
+              else
+                bulk_wait_read<0>();
+            }
             __syncwarp();
           }
           uint32_t r[C::CW];
           tmem_ld32(taddr + c, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
           if constexpr (C::CW == 64) tmem_ld32(taddr + c + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
           tmem_wait_ld();
-          if (c + C::CW == BN) release_acc(acc);  // accumulator no longer needed
+          if (c + C::CW == c_end) release_acc(acc);  // this warp's part of the accumulator is read
           const int col0 = n * BN + c;
           const bool add_bias = !(EPI == SAL_EPI_RESID_F32 && sp != 0);
           const uint4* bias8 = reinterpret_cast<const uint4*>(args.bias + col0);
@@ -623,14 +655,14 @@ sal_status launch_bn(const GemmArgs& a, const void* A, const void* W, cudaStream
     // one cluster of two CTAs per pair of SMs, walking 256-row work units
     const int units = static_cast<int>((a.M + 2 * C::BM - 1) / (2 * C::BM)) * (a.N / BN) * a.splits;
     const int pairs = units < num_sms() / 2 ? units : num_sms() / 2;
-    return launch_kernel_cluster(gemm_kernel<BN, EPI, true>, dim3(2 * pairs), dim3(192), C::SMEM, s, 2u, ta, tb,
-                                 tc, a) == cudaSuccess
+    return launch_kernel_cluster(gemm_kernel<BN, EPI, true>, dim3(2 * pairs), dim3(C::THREADS), C::SMEM, s, 2u, ta,
+                                 tb, tc, a) == cudaSuccess
                ? SAL_OK
                : SAL_ECUDA;
   } else {
     const int tiles = static_cast<int>((a.M + C::BM - 1) / C::BM) * (a.N / BN) * a.splits;
     const int grid = tiles < num_sms() ? tiles : num_sms();
-    return launch_kernel(gemm_kernel<BN, EPI, false>, dim3(grid), dim3(192), C::SMEM, s, ta, tb, tc, a) ==
+    return launch_kernel(gemm_kernel<BN, EPI, false>, dim3(grid), dim3(C::THREADS), C::SMEM, s, ta, tb, tc, a) ==
                    cudaSuccess
                ? SAL_OK
                : SAL_ECUDA;
