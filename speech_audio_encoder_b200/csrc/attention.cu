@@ -811,7 +811,10 @@ __global__ void __launch_bounds__(kThreadsDb, 1)
   // waited for before its barrier can complete the next
   uint64_t* p_full = s_full + 4;                  // [2 query tiles][2 buffers]
   uint64_t* o_done = p_full + 4;                  // [2] one phase per P V
-  uint64_t* drain = o_done + 2;
+  // [2] the last P V of each query tile: the softmax waits for it without having waited
+  // for the phases before, so it needs a barrier of its own (one phase)
+  uint64_t* o_final = o_done + 2;
+  uint64_t* drain = o_final + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -846,7 +849,10 @@ __global__ void __launch_bounds__(kThreadsDb, 1)
       mbar_init(&s_full[i], 1);
       mbar_init(&p_full[i], 128);
     }
-    for (int i = 0; i < 2; ++i) mbar_init(&o_done[i], 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&o_done[i], 1);
+      mbar_init(&o_final[i], 1);
+    }
     mbar_init(drain, 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -923,6 +929,7 @@ __global__ void __launch_bounds__(kThreadsDb, 1)
           umma_ts(tmem + 256 + 128 * i, tmem + db_col_s(i, j & 1) + kk * 8,
                   sdesc_mnmajor_sw128(v0 + kk * 2048, kDbKvBox), IDESC_O, (j > 0 || kk > 0));
         umma_commit(&o_done[i]);
+        if (j == n_kv - 1) umma_commit(&o_final[i]);
         if (i == 1) umma_commit(&v_empty[s]);
         return true;
       };
@@ -982,8 +989,9 @@ __global__ void __launch_bounds__(kThreadsDb, 1)
         rescale = true;
       }
       if (j > 0 && __any_sync(0xffffffffu, rescale)) {
-        // O must hold P(j - 1) V(j - 1) before it is scaled: wait for that product (the
-        // next one is issued only after this step's P arrives below)
+        // O must hold P(j - 1) V(j - 1) before it is scaled: wait for that product. The
+        // parity wait is exact: S(j) was issued after P(j - 2) V(j - 2), so that one is
+        // complete, and P(j) V(j) is issued only after this step's P arrives below.
         if (!mbar_wait_warp(&o_done[wg], (j - 1) & 1, guard)) {
           ok = false;
           break;
@@ -1020,7 +1028,7 @@ __global__ void __launch_bounds__(kThreadsDb, 1)
       tc_fence_before();
       mbar_arrive(&p_full[2 * wg + b]);
     }
-    if (ok && mbar_wait_warp(&o_done[wg], (n_kv - 1) & 1, guard)) {
+    if (ok && mbar_wait_warp(&o_final[wg], 0, guard)) {
       tc_fence_after();
       const int64_t t = static_cast<int64_t>(2 * qt2 + wg) * kTile + row;
       const int bb = bh / args.heads, h = bh % args.heads;

@@ -49,11 +49,6 @@ struct GemmArgs {
   unsigned int* status;
 };
 
-// Epilogue warps of the plain kinds (4 or 8; see Cfg::EPW), a build-time knob for measurement.
-#ifndef SAL_GEMM_EPW
-#define SAL_GEMM_EPW 8
-#endif
-
 // PAIR: a cluster of two CTAs computes a 256 x BN tile with tcgen05.mma.cta_group::2. Each
 // CTA loads its own 128 rows of A and its own BN / 2 rows of W (no multicast), holds its 128
 // rows of the accumulator in its TMEM and runs the epilogue on them; the even CTA issues
@@ -66,12 +61,9 @@ struct Cfg {
   // epilogue shared memory: QKV stages a whole head per warp (32 rows x 128 fp32); the
   // other kinds stage 128-byte-wide output boxes for TMA, two per warp
   static constexpr int CW = F32_OUT ? 32 : 64;  // output columns per 128-byte box row
-  // epilogue warps: four (one per TMEM lane quarter), or eight for the plain kinds of
-  // 128- and 256-wide tiles (two per lane quarter, each on half of the columns, one
-  // staging box each), so that two warps per SM sub-partition hide each other's latency
-  static constexpr int EPW = (QKV || BN < 128) ? 4 : SAL_GEMM_EPW;
+  static constexpr int EPW = 4;  // epilogue warps, one per TMEM lane quarter
   static constexpr int THREADS = 64 + 32 * EPW;
-  static constexpr int SCR_BYTES = QKV ? 4 * 32 * 128 * 4 + 4 * 32 * 4 : 8 * 4096;
+  static constexpr int SCR_BYTES = QKV ? 4 * 32 * 128 * 4 + 4 * 32 * 4 : 4 * 2 * 4096;
   static constexpr int BNL = PAIR ? BN / 2 : BN;  // rows of W this CTA loads per tile
   static constexpr int STAGES = PAIR ? (QKV ? 5 : 6)
                                      : (QKV ? (BN == 256 ? 3 : 4) : (BN == 256 ? 4 : (BN == 128 ? 6 : 8)));
@@ -463,12 +455,7 @@ __global__ void __launch_bounds__(Cfg<BN, EPI, PAIR>::THREADS, 1)
       // them into a 128B-swizzled 32-row box in shared memory (two boxes per warp, used in
       // turn); one lane then issues a TMA store of the box, or a TMA reduce-add into the
       // fp32 residual stream, while the warp moves on to the next chunk.
-      // EPW 4: two boxes per warp, used in turn; EPW 8: one box per warp, and warps
-      // 2-5 / 6-9 take the first / second half of the tile's columns
-      constexpr int kBoxes = C::EPW == 4 ? 2 : 1;
-      uint8_t* stg = reinterpret_cast<uint8_t*>(scratch) + (warp - 2) * kBoxes * 4096;
-      const int c_begin = C::EPW == 4 ? 0 : ((warp - 2) >> 2) * (BN / 2);
-      const int c_end = C::EPW == 4 ? BN : c_begin + BN / 2;
+      uint8_t* stg = reinterpret_cast<uint8_t*>(scratch) + (warp - 2) * 8192;
       uint32_t kbuf = 0;
       for (int tile = first_tile; tile < num_tiles; tile += tile_step) {
         const int sp = tile % args.splits;
@@ -479,22 +466,17 @@ __global__ void __launch_bounds__(Cfg<BN, EPI, PAIR>::THREADS, 1)
         const int y = m * C::BM + quarter * 32;
         const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + acc * BN;
 #pragma unroll 1
-        for (int c = c_begin; c < c_end; c += C::CW) {
-          uint8_t* buf = stg + (kbuf % kBoxes) * 4096;
-          if (kbuf >= kBoxes) {  // the store issued from this box kBoxes chunks ago has read it
-            if (lane == 0) {
-              if constexpr (kBoxes == 2)
-                bulk_wait_read<1>();
-              else
-                bulk_wait_read<0>();
-            }
+        for (int c = 0; c < BN; c += C::CW) {
+          uint8_t* buf = stg + (kbuf & 1) * 4096;
+          if (kbuf >= 2) {  // the store issued from this box two chunks ago has read it
+            if (lane == 0) bulk_wait_read<1>();
             __syncwarp();
           }
           uint32_t r[C::CW];
           tmem_ld32(taddr + c, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
           if constexpr (C::CW == 64) tmem_ld32(taddr + c + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
           tmem_wait_ld();
-          if (c + C::CW == c_end) release_acc(acc);  // this warp's part of the accumulator is read
+          if (c + C::CW == BN) release_acc(acc);  // accumulator no longer needed
           const int col0 = n * BN + c;
           const bool add_bias = !(EPI == SAL_EPI_RESID_F32 && sp != 0);
           const uint4* bias8 = reinterpret_cast<const uint4*>(args.bias + col0);
@@ -698,15 +680,19 @@ int pick_bn(int64_t M, int N, bool qkv) {
 }
 
 // CTA pairs (256 x 256 work units over two SMs) for 256-wide tiles without a K split, once
-// the pairs' units alone fill every pair of SMs. SAL_GEMM_PAIR=0 / 1 in the environment
-// forces them off / on (where the shape allows them), for measurement.
-bool use_pair(int64_t M, int N, int BN, int splits) {
+// the pairs' units alone fill every pair of SMs, for the plain epilogues. (Measured at
+// 11,984 and 44,999 rows: +5 to +12 % for FFN up, FFN down and the output projection;
+// the QKV epilogue, which stages a whole head per warp, runs 8 % slower at 11,984 rows and
+// even at 44,999, so it keeps one CTA per tile.) SAL_GEMM_PAIR=0 / 1 in the environment
+// forces pairs off / on where the shape allows them, for measurement.
+bool use_pair(int64_t M, int N, int BN, int splits, bool qkv) {
   static const int mode = [] {
     const char* e = std::getenv("SAL_GEMM_PAIR");
     return e && e[0] == '0' ? 0 : (e && e[0] == '1' ? 1 : -1);
   }();
-  if (mode != 1 || BN != 256 || splits != 1 || N % 256) return false;
-  return (M + 255) / 256 * (N / 256) >= 1;
+  if (mode == 0 || BN != 256 || splits != 1 || N % 256) return false;
+  if (mode == 1) return true;
+  return !qkv && (M + 255) / 256 * (N / 256) >= num_sms() / 2;
 }
 
 }  // namespace
@@ -754,7 +740,7 @@ sal_status gemm_launch(int epilogue, const void* A, int64_t M, int K, const void
            a.splits < 8)
       a.splits *= 2;
   }
-  const bool pair = use_pair(M, N, BN, a.splits);
+  const bool pair = use_pair(M, N, BN, a.splits, is_qkv);
   switch (epilogue) {
     case SAL_EPI_STORE_F32: return launch_epi<SAL_EPI_STORE_F32>(BN, pair, a, A, W, s);
     case SAL_EPI_STORE_BF16: return launch_epi<SAL_EPI_STORE_BF16>(BN, pair, a, A, W, s);
