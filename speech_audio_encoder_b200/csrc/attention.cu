@@ -45,16 +45,6 @@ constexpr float kRescaleThreshold = 8.0f;  // log2 units
 // The choice between the one-tile and two-tile kernels can be forced with SAL_ATTN_PP.
 // SAL_ATTN_PP: unset = choose by the wave model below, 0 = never the two-tile kernel,
 // 1 = always (where its grid has at least one query-tile pair); for measuring the choice.
-// SAL_ATTN_DB=1 runs the two-tile kernel with 64-key steps and double-buffered scores
-// (attention_db_kernel) in place of attention_pp_kernel, for measurement.
-bool attention_db_mode() {
-  static const bool on = [] {
-    const char* e = std::getenv("SAL_ATTN_DB");
-    return e && e[0] == '1';
-  }();
-  return on;
-}
-
 int attention_pp_mode() {
   static const int mode = [] {
     const char* e = std::getenv("SAL_ATTN_PP");
@@ -448,6 +438,7 @@ constexpr int kPolyPairsPP = SAL_PP_POLY_PAIRS;
 #define SAL_PP_SPLIT_P 0
 #endif
 constexpr bool kSplitP = SAL_PP_SPLIT_P != 0;
+
 constexpr int kThreadsPP = 384;
 constexpr int kRegsCtrl = 80, kRegsSoftmax = 208;
 constexpr int kRegsNeededPP = kRegsCtrl * 128 + kRegsSoftmax * 256;  // <= launch regs x 384
@@ -756,323 +747,6 @@ __global__ void __launch_bounds__(kThreadsPP, 1)
   }
 }
 
-// ---------------------------------------------------------------------------------
-// Two query tiles per CTA, keys in steps of 64 with two score buffers per query tile.
-// The one-CTA-per-SM TMEM (512 columns) holds O0 and O1 (128 columns each) and four 64-column
-// score buffers S(i, b): while query tile i's softmax works on S(i, j) the tensor core
-// has already computed S(i, j + 1) into the other buffer, so a softmax warpgroup goes from
-// one step to the next without waiting for its own P V and next S (P(i, j) overwrites the
-// scores of S(i, j) once read; S(i, j + 2) reuses the buffer after P(i, j) V(j) was issued).
-//   warp 0: TMA loads (Q0, Q1 once; K and V in 64-key tiles through kDbStages-deep rings)
-//   warp 1: tcgen05.mma issue: S(0,0) S(1,0) S(0,1) S(1,1) | P(0,j) V(j), S(0,j+2),
-//           P(1,j) V(j), S(1,j+2), ...
-//   warps 2-3: idle
-//   warps 4-7 / 8-11: softmax of query tile 0 / 1, one row per thread (64 scores a step)
-// TMEM: S(i, b) at 64 (2 i + b); O_i at 256 + 128 i.
-constexpr int kDbKeys = 64;
-constexpr int kDbStages = 4;
-constexpr int kDbKvBox = kDbKeys * 64 * 2;         // 8 KB: 64 keys x 64 columns
-constexpr int kDbKvBytes = 2 * kDbKvBox;           // a 64-key tile of K or V (16 KB)
-constexpr size_t kSmemDb = 1024 + 2 * kTileBytes + 2 * kDbStages * kDbKvBytes + 256;
-constexpr int kThreadsDb = 384;
-
-__device__ __forceinline__ uint32_t db_col_s(int i, int b) { return 64u * (2 * i + b); }
-
-// Maximum of a row of 64 scores held as raw fp32 bits: eight chains of four max3, merged.
-__device__ __forceinline__ float row_max64(const uint32_t (&r)[2][32]) {
-  float m[8];
-#pragma unroll
-  for (int k = 0; k < 8; ++k) {
-    const uint32_t* v = &r[k >> 2][(k & 3) * 8];
-    m[k] = fmaxf(__uint_as_float(v[0]), __uint_as_float(v[1]));
-#pragma unroll
-    for (int i = 2; i < 8; i += 2) m[k] = max3f(m[k], __uint_as_float(v[i]), __uint_as_float(v[i + 1]));
-  }
-  return max3f(max3f(m[0], m[1], m[2]), max3f(m[3], m[4], m[5]), fmaxf(m[6], m[7]));
-}
-
-__global__ void __launch_bounds__(kThreadsDb, 1)
-    attention_db_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                        const __grid_constant__ CUtensorMap tmV, const AttnArgs args) {
-  extern __shared__ unsigned char smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* sQ = smem;                                    // Q0, Q1 (128 rows each)
-  uint8_t* sK = smem + 2 * kTileBytes;                   // [kDbStages] 64-key tiles
-  uint8_t* sV = sK + kDbStages * kDbKvBytes;             // [kDbStages]
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sV + kDbStages * kDbKvBytes);
-  uint64_t* q_full = bars + 0;
-  uint64_t* k_full = bars + 1;                    // [kDbStages]
-  uint64_t* v_full = k_full + kDbStages;          // [kDbStages]
-  uint64_t* k_empty = v_full + kDbStages;         // [kDbStages]
-  uint64_t* v_empty = k_empty + kDbStages;        // [kDbStages]
-  uint64_t* s_full = v_empty + kDbStages;         // [2 query tiles][2 buffers]
-  // P(i, j) ready, per query tile and buffer: a softmax warpgroup can finish two steps
-  // before the MMA thread takes the first, so one barrier per buffer keeps each phase
-  // waited for before its barrier can complete the next
-  uint64_t* p_full = s_full + 4;                  // [2 query tiles][2 buffers]
-  uint64_t* o_done = p_full + 4;                  // [2] one phase per P V
-  // [2] the last P V of each query tile: the softmax waits for it without having waited
-  // for the phases before, so it needs a barrier of its own (one phase)
-  uint64_t* o_final = o_done + 2;
-  uint64_t* drain = o_final + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-
-  const int warp = threadIdx.x >> 5;
-  const int lane = threadIdx.x & 31;
-  const int64_t T = args.T;
-  const int bh = blockIdx.y;
-  const int qt2 = blockIdx.x;  // 256-row query block
-  const int64_t Tk = valid_len(args, bh / args.heads);
-  int j0, n_kv;  // in 64-key tiles
-  {
-    int64_t q_lo = static_cast<int64_t>(qt2) * 2 * kTile, q_hi = q_lo + 2 * kTile;
-    if (q_hi > Tk) q_hi = Tk;
-    if (q_lo > Tk - 1) q_lo = Tk - 1;
-    if (q_hi <= q_lo) q_hi = q_lo + 1;
-    const int64_t kv_lo = (q_lo / args.chunk) * args.chunk;
-    int64_t kv_hi = ((q_hi - 1) / args.chunk + 1) * args.chunk;
-    if (kv_hi > Tk) kv_hi = Tk;
-    j0 = static_cast<int>(kv_lo / kDbKeys);
-    n_kv = static_cast<int>((kv_hi + kDbKeys - 1) / kDbKeys) - j0;
-  }
-
-  if (threadIdx.x == 0) {
-    mbar_init(q_full, 1);
-    for (int s = 0; s < kDbStages; ++s) {
-      mbar_init(&k_full[s], 1);
-      mbar_init(&v_full[s], 1);
-      mbar_init(&k_empty[s], 1);
-      mbar_init(&v_empty[s], 1);
-    }
-    for (int i = 0; i < 4; ++i) {
-      mbar_init(&s_full[i], 1);
-      mbar_init(&p_full[i], 128);
-    }
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(&o_done[i], 1);
-      mbar_init(&o_final[i], 1);
-    }
-    mbar_init(drain, 1);
-    *abort_flag = 0;
-    fence_mbar_init();
-    tma_prefetch_desc(&tmQ);
-    tma_prefetch_desc(&tmK);
-    tma_prefetch_desc(&tmV);
-  }
-  if (warp == 1) {
-    tmem_alloc(tmem_slot, 512);
-    tmem_relinquish();
-  }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  pdl_wait();
-  pdl_trigger();
-  const uint32_t tmem = *tmem_slot;
-  const WaitGuard guard{abort_flag, args.limit_ns, args.status};
-  // the producer's record of the ring slots it loaded and their phases (for the wind-down)
-  uint32_t issued_k = 0, issued_v = 0, par_k = 0, par_v = 0;
-
-  if (warp == 0) {
-    if (lane == 0) {
-      mbar_arrive_expect_tx(q_full, 2 * kTileBytes);
-      for (int i = 0; i < 2; ++i) {
-        tma_load_3d(sQ + i * kTileBytes, &tmQ, q_full, 0, (2 * qt2 + i) * kTile, bh);
-        tma_load_3d(sQ + i * kTileBytes + kBox, &tmQ, q_full, 64, (2 * qt2 + i) * kTile, bh);
-      }
-      for (int j = 0; j < n_kv; ++j) {
-        const int s = j % kDbStages;
-        const uint32_t use_par = (j / kDbStages) & 1;
-        if (!mbar_wait(&k_empty[s], use_par ^ 1, guard)) break;
-        if (j == args.withhold) continue;  // test hook: nothing issued for this tile
-        mbar_arrive_expect_tx(&k_full[s], kDbKvBytes);
-        tma_load_3d(sK + s * kDbKvBytes, &tmK, &k_full[s], 0, (j0 + j) * kDbKeys, bh);
-        tma_load_3d(sK + s * kDbKvBytes + kDbKvBox, &tmK, &k_full[s], 64, (j0 + j) * kDbKeys, bh);
-        issued_k |= 1u << s;
-        par_k = (par_k & ~(1u << s)) | (use_par << s);
-        if (!mbar_wait(&v_empty[s], use_par ^ 1, guard)) break;
-        mbar_arrive_expect_tx(&v_full[s], kDbKvBytes);
-        tma_load_3d(sV + s * kDbKvBytes, &tmV, &v_full[s], 0, (j0 + j) * kDbKeys, bh);
-        tma_load_3d(sV + s * kDbKvBytes + kDbKvBox, &tmV, &v_full[s], 64, (j0 + j) * kDbKeys, bh);
-        issued_v |= 1u << s;
-        par_v = (par_v & ~(1u << s)) | (use_par << s);
-      }
-    }
-  } else if (warp == 1) {
-    if (lane == 0) {
-      constexpr uint32_t IDESC_S = idesc_bf16(128, kDbKeys, false, false);
-      constexpr uint32_t IDESC_O = idesc_bf16(128, 128, false, true);
-      bool any_mma = false;
-      auto issue_s = [&](int i, int j) -> bool {  // S(i, j) = Q_i K_j^T into buffer j & 1
-        const int s = j % kDbStages;
-        if (!mbar_wait(&k_full[s], (j / kDbStages) & 1, guard)) return false;
-        tc_fence_after();
-        const uint32_t q0 = smem_u32(sQ + i * kTileBytes), k0 = smem_u32(sK + s * kDbKvBytes);
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          umma_ss(tmem + db_col_s(i, j & 1), sdesc_kmajor_sw128(q0 + (kk >> 2) * kBox + (kk & 3) * 32),
-                  sdesc_kmajor_sw128(k0 + (kk >> 2) * kDbKvBox + (kk & 3) * 32), IDESC_S, kk > 0);
-        umma_commit(&s_full[2 * i + (j & 1)]);
-        if (i == 1) umma_commit(&k_empty[s]);  // both products with K_j issued
-        any_mma = true;
-        return true;
-      };
-      auto issue_pv = [&](int i, int j) -> bool {  // O_i += P(i, j) V_j
-        const int s = j % kDbStages;
-        if (!mbar_wait(&p_full[2 * i + (j & 1)], (j >> 1) & 1, guard)) return false;
-        if (!mbar_wait(&v_full[s], (j / kDbStages) & 1, guard)) return false;
-        tc_fence_after();
-        const uint32_t v0 = smem_u32(sV + s * kDbKvBytes);
-#pragma unroll
-        for (int kk = 0; kk < kDbKeys / 16; ++kk)
-          umma_ts(tmem + 256 + 128 * i, tmem + db_col_s(i, j & 1) + kk * 8,
-                  sdesc_mnmajor_sw128(v0 + kk * 2048, kDbKvBox), IDESC_O, (j > 0 || kk > 0));
-        umma_commit(&o_done[i]);
-        if (j == n_kv - 1) umma_commit(&o_final[i]);
-        if (i == 1) umma_commit(&v_empty[s]);
-        return true;
-      };
-      bool ok = mbar_wait(q_full, 0, guard);
-      for (int j = 0; ok && j < 2 && j < n_kv; ++j) ok = issue_s(0, j) && issue_s(1, j);
-      for (int j = 0; ok && j < n_kv; ++j) {
-        for (int i = 0; ok && i < 2; ++i) {
-          ok = issue_pv(i, j);
-          if (ok && j + 2 < n_kv) ok = issue_s(i, j + 2);
-        }
-      }
-      if (*abort_flag && any_mma) {
-        umma_commit(drain);
-        drain_wait(drain, 0);
-      }
-    }
-  } else if (warp >= 4) {
-    // ------------------------------------------------------------ softmax warpgroups
-    const int wg = (warp - 4) >> 2;  // query tile 0 or 1
-    const int quarter = warp & 3;
-    const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
-    const uint32_t colO = 256u + 128u * wg;
-    const int row = quarter * 32 + lane;
-    const float sl2 = args.scale_log2;
-    float m_ref = -INFINITY, l = 0.f;
-    bool ok = true;
-    int row_lo, row_hi;
-    row_range((2 * qt2 + wg) * kTile + row, static_cast<int>(T), static_cast<int>(Tk), static_cast<int>(args.chunk),
-              row_lo, row_hi);
-    for (int j = 0; j < n_kv; ++j) {
-      const int b = j & 1;
-      if (!mbar_wait_warp(&s_full[2 * wg + b], (j >> 1) & 1, guard)) {
-        ok = false;
-        break;
-      }
-      tc_fence_after();
-      uint32_t r[2][32];
-      tmem_ld32(tmem + lane_base + db_col_s(wg, b), r[0]);
-      tmem_ld32(tmem + lane_base + db_col_s(wg, b) + 32, r[1]);
-      tmem_wait_ld();
-      {  // keys of this 64-key tile outside the row's range become -inf
-        const int base = (j0 + j) * kDbKeys;
-        const int c_lo = min(max(row_lo - base, 0), kDbKeys), c_hi = min(max(row_hi - base, 0), kDbKeys);
-        if (!__all_sync(0xffffffffu, c_lo == 0 && c_hi == kDbKeys)) {
-          mask_chunk(r[0], 0, c_lo, c_hi);
-          mask_chunk(r[1], 32, c_lo, c_hi);
-        }
-      }
-      const float mx = row_max64(r) * sl2;
-      float alpha = 1.f;
-      bool rescale = false;
-      if (j == 0) {
-        m_ref = mx;
-      } else if (mx > m_ref + kRescaleThreshold) {
-        alpha = fast_exp2(m_ref - mx);
-        m_ref = mx;
-        rescale = true;
-      }
-      if (j > 0 && __any_sync(0xffffffffu, rescale)) {
-        // O must hold P(j - 1) V(j - 1) before it is scaled: wait for that product. The
-        // parity wait is exact: S(j) was issued after P(j - 2) V(j - 2), so that one is
-        // complete, and P(j) V(j) is issued only after this step's P arrives below.
-        if (!mbar_wait_warp(&o_done[wg], (j - 1) & 1, guard)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-#pragma unroll 1
-        for (int c = 0; c < 4; ++c) {
-          uint32_t o[32];
-          tmem_ld32(tmem + lane_base + colO + 32 * c, o);
-          tmem_wait_ld();
-#pragma unroll
-          for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-          tmem_st32(tmem + lane_base + colO + 32 * c, o);
-        }
-      }
-      const float m_use = m_ref == -INFINITY ? 0.f : m_ref;  // a row with no key seen yet
-      const uint64_t sl2_2 = f2_pack(sl2, sl2), negm_2 = f2_pack(-m_use, -m_use);
-      uint64_t sum2[2];
-#pragma unroll
-      for (int c = 0; c < 2; ++c)
-#pragma unroll
-        for (int i = 0; i < 32; i += 2) {
-          float x0, x1;
-          f2_unpack(f2_fma(f2_pack(__uint_as_float(r[c][i]), __uint_as_float(r[c][i + 1])), sl2_2, negm_2), x0, x1);
-          const float e0 = fast_exp2(x0), e1 = fast_exp2(x1);
-          sum2[c] = i == 0 ? f2_pack(e0, e1) : f2_add(sum2[c], f2_pack(e0, e1));
-          r[0][c * 16 + (i >> 1)] = pack_bf16x2(e0, e1);  // P over the scores already read
-        }
-      tmem_st32(tmem + lane_base + db_col_s(wg, b), r[0]);
-      float sum_lo, sum_hi;
-      f2_unpack(f2_add(sum2[0], sum2[1]), sum_lo, sum_hi);
-      l = l * alpha + (sum_lo + sum_hi);
-      tmem_wait_st();
-      tc_fence_before();
-      mbar_arrive(&p_full[2 * wg + b]);
-    }
-    if (ok && mbar_wait_warp(&o_final[wg], 0, guard)) {
-      tc_fence_after();
-      const int64_t t = static_cast<int64_t>(2 * qt2 + wg) * kTile + row;
-      const int bb = bh / args.heads, h = bh % args.heads;
-      const float inv_l = 1.0f / l;
-      __nv_bfloat16* dst = args.o + (static_cast<int64_t>(bb) * T + t) * (args.heads * kHeadDim) + h * kHeadDim;
-#pragma unroll 1
-      for (int c = 0; c < 4; ++c) {
-        uint32_t o[32];
-        tmem_ld32(tmem + lane_base + colO + 32 * c, o);
-        tmem_wait_ld();
-        if (t < T) {
-          uint4* d4 = reinterpret_cast<uint4*>(dst + 32 * c);
-#pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            uint4 u;
-            u.x = pack_bf16x2(__uint_as_float(o[8 * i + 0]) * inv_l, __uint_as_float(o[8 * i + 1]) * inv_l);
-            u.y = pack_bf16x2(__uint_as_float(o[8 * i + 2]) * inv_l, __uint_as_float(o[8 * i + 3]) * inv_l);
-            u.z = pack_bf16x2(__uint_as_float(o[8 * i + 4]) * inv_l, __uint_as_float(o[8 * i + 5]) * inv_l);
-            u.w = pack_bf16x2(__uint_as_float(o[8 * i + 6]) * inv_l, __uint_as_float(o[8 * i + 7]) * inv_l);
-            d4[i] = u;
-          }
-        }
-      }
-    }
-  }
-
-  tc_fence_before();
-  __syncthreads();
-  if (warp == 1) {
-    __syncwarp();
-    tc_fence_after();
-    tmem_dealloc(tmem, 512);
-  }
-  // Every role has finished, so the abort flag is final: let every load this CTA issued
-  // land before the CTA, and its shared memory, goes away.
-  if (warp == 0 && lane == 0 && *abort_flag) {
-    drain_wait(q_full, 0);
-    for (int s = 0; s < kDbStages; ++s) {
-      if (issued_k & (1u << s)) drain_wait(&k_full[s], (par_k >> s) & 1);
-      if (issued_v & (1u << s)) drain_wait(&v_full[s], (par_v >> s) & 1);
-    }
-  }
-}
-
 std::mutex g_mu;
 bool g_attr[64] = {};
 bool g_pp_ok[64] = {};  // the two-tile kernel's launch registers cover its warpgroup split
@@ -1151,9 +825,7 @@ sal_status attention_launch_heads(const void* q, const void* k, const void* v, i
           cudaFuncSetAttribute(attention_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                static_cast<int>(smem_one_tile(64))) != cudaSuccess ||
           cudaFuncSetAttribute(attention_pp_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               static_cast<int>(kSmemPP)) != cudaSuccess ||
-          cudaFuncSetAttribute(attention_db_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               static_cast<int>(kSmemDb)) != cudaSuccess)
+                               static_cast<int>(kSmemPP)) != cudaSuccess)
         return SAL_ECUDA;
       // setmaxnreg.inc waits until the registers it asks for are free: run the kernel only
       // if what warpgroup 0 gives back covers what the softmax warpgroups take (and the
@@ -1215,16 +887,8 @@ sal_status attention_launch_heads(const void* q, const void* k, const void* v, i
   const int pp_tiles = 2 * P < n_qt ? 2 * P : n_qt;
   if (P > 0) {
     const dim3 grid(static_cast<unsigned>(P), static_cast<unsigned>(bh));
-    if (attention_db_mode() && !hold) {
-      CUtensorMap tk64, tv64;  // 64-key tiles
-      if (!make_tmap_3d_bf16(&tk64, k, head_dim, T, bh, 64, kDbKeys, 1)) return SAL_ECUDA;
-      if (!make_tmap_3d_bf16(&tv64, v, head_dim, T, bh, 64, kDbKeys, 1)) return SAL_ECUDA;
-      if (launch_kernel(attention_db_kernel, grid, dim3(kThreadsDb), kSmemDb, s, tq, tk64, tv64, a) != cudaSuccess)
-        return SAL_ECUDA;
-    } else if (launch_kernel(attention_pp_kernel, grid, dim3(kThreadsPP), kSmemPP, s, tq, tk, tv, a) !=
-               cudaSuccess) {
+    if (launch_kernel(attention_pp_kernel, grid, dim3(kThreadsPP), kSmemPP, s, tq, tk, tv, a) != cudaSuccess)
       return SAL_ECUDA;
-    }
   }
   if (pp_tiles == n_qt) return SAL_OK;
   a.qt0 = pp_tiles;
