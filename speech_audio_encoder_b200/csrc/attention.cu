@@ -429,7 +429,7 @@ constexpr size_t kSmemPP = 1024 + 6 * kTileBytes + 256;
 // Of every 16 score pairs of a row chunk, this many take their exponentials on the FMA
 // pipe (exp2_pair_poly) instead of the SFU.
 #ifndef SAL_PP_POLY_PAIRS
-#define SAL_PP_POLY_PAIRS 0
+#define SAL_PP_POLY_PAIRS 2
 #endif
 constexpr int kPolyPairsPP = SAL_PP_POLY_PAIRS;
 // Each softmax warpgroup hands P to the tensor core in two halves of 64 keys, so the first
