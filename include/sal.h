@@ -102,28 +102,39 @@ typedef struct {
     const void *lnf_g, *lnf_b;
 } sal_weights;
 
-/* Front end: wave [batch, n_samples] float32 at 16 kHz ->
+/* Front end (page "Nemotron 3.5 Transcribe: From Recorded Speech to Dataset Audits",
+ * section "How audio and speakers reach the language model", exported-frontend
+ * paragraph: 16 kHz mono, 128 log-mel features, 25 ms Hann window, 512-point FFT, 10 ms
+ * hop, eight stacked frames): wave [batch, n_samples] float32 at 16 kHz ->
  *   logmel  [batch, F, 128] float32, natural-log mel energies (required), and
  *   stacked [batch, T, 1024] bf16, the frame-major stack of the first 8 T frames
  *           (the projection's input; may be NULL).
  * One kernel: framing, Hann window, 512-point real FFT, power, 128 Slaney mel filters,
- * log and the bf16 stacked copy. */
+ * log and the bf16 stacked copy. Errors: SAL_EINVAL (negative sizes, null or misaligned
+ * pointer), SAL_ESHAPE (T > 45,000 or batch > 65,535), SAL_EDEVICE, SAL_ECUDA. */
 sal_status sal_frontend(const float* wave, int64_t n_samples, int batch, float* logmel,
                         void* stacked, void* stream);
 
-/* Stack projection x0 = S P^T + p: stacked [batch * T, 1024] bf16 ->
- * x [batch * T, 1280] float32 (the encoder's residual stream). */
+/* Stack projection (same paragraph: the eight stacked frames are projected to width
+ * 1,280) x0 = S P^T + p: stacked [batch * T, 1024] bf16 -> x [batch * T, 1280] float32
+ * (the encoder's residual stream); w->w_proj [1280, 1024] and w->b_proj [1280] bf16.
+ * Errors: SAL_EINVAL, SAL_ESHAPE (T > 45,000), SAL_EDEVICE, SAL_ECUDA. */
 sal_status sal_stack_project(const void* stacked, int batch, int64_t T, const sal_weights* w,
                              float* x, void* stream);
 
 /* Bytes of scratch that sal_encoder_forward needs for `batch` clips of T positions. */
 size_t sal_encoder_workspace_bytes(int batch, int64_t T);
 
-/* Encoder: x [batch * T, 1280] float32 holds x0 on entry and the residual stream after
- * n_layers layers on return (clobbered); emb [batch * T, 1280] bf16 receives the final
- * LayerNorm of it. n_layers may be 0..w->n_layers. Positions restart at 0 in each clip
- * and attention never crosses clips. `workspace` is device scratch of ws_bytes >=
- * sal_encoder_workspace_bytes(batch, T), 256-byte aligned. */
+/* Encoder (same paragraph: 32 Transformer layers at width 1,280 with ten heads, QK
+ * normalisation, feed-forward expansion four and rotary position embeddings; the
+ * readings above for what it leaves open): x [batch * T, 1280] float32 holds x0 on
+ * entry and the residual stream after n_layers layers on return (clobbered); emb
+ * [batch * T, 1280] bf16 receives the final LayerNorm of it. n_layers may be
+ * 0..w->n_layers. Positions restart at 0 in each clip and attention never crosses clips.
+ * `workspace` is device scratch of ws_bytes >= sal_encoder_workspace_bytes(batch, T),
+ * 256-byte aligned. Errors: SAL_EINVAL (bad count, null or misaligned pointer, a layer
+ * with a null or misaligned parameter), SAL_ESHAPE (T > 45,000 or batch > 6,553),
+ * SAL_EWORKSPACE, SAL_EDEVICE, SAL_ECUDA. */
 sal_status sal_encoder_forward(float* x, int batch, int64_t T, const sal_weights* w, int n_layers,
                                void* emb, void* workspace, size_t ws_bytes, void* stream);
 
