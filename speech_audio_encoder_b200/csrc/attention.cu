@@ -411,33 +411,32 @@ __global__ void __launch_bounds__(192, 1)
 // ---------------------------------------------------------------------------------
 // Ping-pong variant for long clips: one CTA owns TWO 128-row query tiles of one
 // (clip, head), so each K / V tile loaded serves 256 queries, and two softmax warpgroups
-// alternate with the tensor core: while warpgroup 0 runs the softmax of S0_j, the
-// tensor core computes O1 += P1_{j-1} V_{j-1} and S1_j, and the other way round.
+// take turns with the tensor core.
 //   warp 0: TMA loads (Q0 and Q1 once; K_j and V_j through two-stage rings released
 //           separately: K after both S products, V after both P V products)
-//   warp 1: tcgen05.mma issue, in the order S0_0 S1_0 | PV0_j S0_{j+1} PV1_j S1_{j+1} ...
+//   warp 1: tcgen05.mma issue, in the order S0_0 S1_0 | S0_{j+1} PV0_j S1_{j+1} PV1_j ...
 //   warps 2-3: idle (they complete warpgroup 0, which gives registers away)
 //   warps 4-7 / 8-11: softmax of query tile 0 / 1, one row per thread
-// TMEM: S0 [0,128) S1 [128,256) O0 [256,384) O1 [384,512); P_i (bf16 pairs) overwrites
-// the first 64 columns of S_i once the row has been read. Because tcgen05.mma operations
-// of one thread complete in issue order, S_i(j) completing implies P_i(j-1) V_{j-1} has
-// completed, so the softmax may rescale O_i as soon as S_i(j) is ready.
+// TMEM: S [0,128) O0 [128,256) O1 [256,384) P0 [384,448) P1 [448,512). The one score
+// buffer S is shared by the two query tiles: a warpgroup copies its S_i(j) into registers
+// and hands the buffer back at once, so the next product (the other tile's S, then its
+// own S_i(j+1)) runs on the tensor core while its exponentials are computed. P_i (bf16
+// pairs) has a region of its own, so S_i(j+1) does not wait for P_i(j) V_j. The
+// warpgroup waits for P_i(j-1) V_{j-1} to complete before it rescales O_i or overwrites
+// P_i.
 // Warpgroup 0 (loads, MMA issue) shrinks to kRegsCtrl registers per thread and the two
 // softmax warpgroups grow to kRegsSoftmax, so each softmax thread holds its whole row of
 // S (128 scores) and reads it from TMEM in one round trip per tile.
 constexpr size_t kSmemPP = 1024 + 6 * kTileBytes + 256;
+constexpr uint32_t kColSPP = 0;
+__device__ __forceinline__ uint32_t col_o_pp(int i) { return 128u + 128u * i; }
+__device__ __forceinline__ uint32_t col_p_pp(int i) { return 384u + 64u * i; }
 // Of every 16 score pairs of a row chunk, this many take their exponentials on the FMA
 // pipe (exp2_pair_poly) instead of the SFU.
 #ifndef SAL_PP_POLY_PAIRS
 #define SAL_PP_POLY_PAIRS 2
 #endif
 constexpr int kPolyPairsPP = SAL_PP_POLY_PAIRS;
-// Each softmax warpgroup hands P to the tensor core in two halves of 64 keys, so the first
-// half of P V runs while the second half's exponentials are computed.
-#ifndef SAL_PP_SPLIT_P
-#define SAL_PP_SPLIT_P 0
-#endif
-constexpr bool kSplitP = SAL_PP_SPLIT_P != 0;
 
 constexpr int kThreadsPP = 384;
 constexpr int kRegsCtrl = 80, kRegsSoftmax = 208;
@@ -457,13 +456,15 @@ __global__ void __launch_bounds__(kThreadsPP, 1)
   uint64_t* v_full = bars + 3;    // [2]
   uint64_t* k_empty = bars + 5;   // [2]
   uint64_t* v_empty = bars + 7;   // [2]
-  uint64_t* s_full = bars + 9;    // [2] one per query tile
-  uint64_t* p_full = bars + 11;   // [2]
-  uint64_t* o_final = bars + 13;  // [2]
-  uint64_t* drain = bars + 15;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 16);
+  uint64_t* s_full = bars + 9;    // [2] S_i(j) is in the score buffer
+  uint64_t* p_full = bars + 11;   // [2] P_i(j) is in its region (O_i rescaled if needed)
+  uint64_t* pv_done = bars + 13;  // [2] P_i(j) V_j has completed
+  uint64_t* s_free = bars + 15;   // the score buffer has been read (one phase per S)
+  uint64_t* drain = bars + 16;     // wind-down of the S issuer
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 17);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  uint64_t* p_half1 = bars + 18;  // [2] second half of P (kSplitP; p_full then means the first)
+  uint64_t* drain_pv = bars + 18;  // wind-down of the P V issuer
+  volatile int* s_issued = reinterpret_cast<volatile int*>(bars + 19);  // S products issued so far
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -484,10 +485,12 @@ __global__ void __launch_bounds__(kThreadsPP, 1)
       mbar_init(&v_empty[s], 1);
       mbar_init(&s_full[s], 1);
       mbar_init(&p_full[s], 128);
-      mbar_init(&p_half1[s], 128);
-      mbar_init(&o_final[s], 1);
+      mbar_init(&pv_done[s], 1);
     }
+    mbar_init(s_free, 4);  // one arrival per warp of the warpgroup that read S
     mbar_init(drain, 1);
+    mbar_init(drain_pv, 1);
+    *s_issued = 0;
     *abort_flag = 0;
     fence_mbar_init();
     tma_prefetch_desc(&tmQ);
@@ -537,64 +540,84 @@ __global__ void __launch_bounds__(kThreadsPP, 1)
         }
       }
     } else if (warp == 1) {
+      // S issue: S_i(x) into the shared score buffer, in the order S0_0 S1_0 S0_1 S1_1 ...
       if (lane == 0) {
         constexpr uint32_t IDESC_S = idesc_bf16(128, 128, false, false);
-        constexpr uint32_t IDESC_O = idesc_bf16(128, 128, false, true);
         bool any_mma = false;
-        auto issue_s = [&](int i, int j) -> bool {  // S_i = Q_i K_j^T
-          const int s = j & 1;
-          if (!mbar_wait(&k_full[s], (j >> 1) & 1, guard)) return false;
+        bool ok = mbar_wait(q_full, 0, guard);
+        for (int q = 0; ok && q < 2 * n_kv; ++q) {
+          const int i = q & 1, x = q >> 1, s = x & 1;
+          // the previous S product has been read out of the buffer, and K_x has landed
+          ok = (q == 0 || mbar_wait(s_free, (q - 1) & 1, guard)) && mbar_wait(&k_full[s], (x >> 1) & 1, guard);
+          if (!ok) break;
           tc_fence_after();
           const uint32_t q0 = smem_u32(sQ + i * kTileBytes), k0 = smem_u32(sK + s * kTileBytes);
-  #pragma unroll
+#pragma unroll
           for (int kk = 0; kk < 8; ++kk) {
             const uint32_t off = (kk >> 2) * kBox + (kk & 3) * 32;
-            umma_ss(tmem + 128 * i, sdesc_kmajor_sw128(q0 + off), sdesc_kmajor_sw128(k0 + off), IDESC_S, kk > 0);
+            umma_ss(tmem + kColSPP, sdesc_kmajor_sw128(q0 + off), sdesc_kmajor_sw128(k0 + off), IDESC_S, kk > 0);
           }
           umma_commit(&s_full[i]);
-          if (i == 1) umma_commit(&k_empty[s]);  // both products with K_j issued
+          if (i == 1) umma_commit(&k_empty[s]);  // both products with K_x issued
           any_mma = true;
-          return true;
-        };
-        auto issue_pv = [&](int i, int j) -> bool {  // O_i += P_i V_j
-          const int s = j & 1;
-          if (!mbar_wait(&p_full[i], j & 1, guard)) return false;
-          if (!mbar_wait(&v_full[s], (j >> 1) & 1, guard)) return false;
-          tc_fence_after();
-          const uint32_t v0 = smem_u32(sV + s * kTileBytes);
-  #pragma unroll
-          for (int kk = 0; kk < 8; ++kk) {
-            if (kSplitP && kk == 4) {  // keys 64-127: their P is the second half
-              if (!mbar_wait(&p_half1[i], j & 1, guard)) return false;
-              tc_fence_after();
-            }
-            umma_ts(tmem + 256 + 128 * i, tmem + 128 * i + kk * 8, sdesc_mnmajor_sw128(v0 + kk * 2048, kBox), IDESC_O,
-                    (j > 0 || kk > 0));
-          }
-          if (i == 1) umma_commit(&v_empty[s]);
-          return true;
-        };
-        bool ok = mbar_wait(q_full, 0, guard) && issue_s(0, 0) && issue_s(1, 0);
-        for (int j = 0; ok && j < n_kv; ++j) {
-          ok = issue_pv(0, j);
-          if (!ok) break;
-          if (j + 1 < n_kv) {
-            ok = issue_s(0, j + 1);
-          } else {
-            umma_commit(&o_final[0]);
-          }
-          if (!ok) break;
-          ok = issue_pv(1, j);
-          if (!ok) break;
-          if (j + 1 < n_kv) {
-            ok = issue_s(1, j + 1);
-          } else {
-            umma_commit(&o_final[1]);
-          }
+          *s_issued = q + 1;
         }
         if (*abort_flag && any_mma) {
           umma_commit(drain);
           drain_wait(drain, 0);
+        }
+      }
+    } else if (warp == 2) {
+      // P V issue: O_i += P_i(j) V_j. A second issuing thread, because one thread alone
+      // spends longer issuing the 32 MMAs of a key tile than the tensor core takes to run
+      // them. The tensor core runs MMAs in issue order, and an S product is on the
+      // critical path (the score buffer is shared), so P_i(j) V_j waits until S_i(j+1)
+      // has been issued and then runs while warpgroup i reads S_i(j+1).
+      if (lane == 0) {
+        constexpr uint32_t IDESC_O = idesc_bf16(128, 128, false, true);
+        bool any_mma = false, ok = true;
+        for (int j = 0; ok && j < n_kv; ++j) {
+          const int s = j & 1;
+          for (int i = 0; i < 2; ++i) {
+            ok = mbar_wait(&p_full[i], j & 1, guard) && mbar_wait(&v_full[s], (j >> 1) & 1, guard);
+            if (!ok) break;
+            if (j + 1 < n_kv) {
+              // a plain spin (the wait is short and its end is on the critical path); the
+              // bound is checked every 64 polls
+              const int need = 2 * (j + 1) + i + 1;
+              uint64_t t0 = 0;
+              for (uint32_t spin = 1; *s_issued < need; ++spin) {
+                if ((spin & 63) != 0) continue;
+                if (*abort_flag) {
+                  ok = false;
+                  break;
+                }
+                const uint64_t now = globaltimer_ns();
+                if (t0 == 0) {
+                  t0 = now;
+                } else if (now - t0 > args.limit_ns) {
+                  *abort_flag = 1;
+                  atomicOr(args.status, kStatusTimeout);
+                  ok = false;
+                  break;
+                }
+              }
+              if (!ok) break;
+            }
+            tc_fence_after();
+            const uint32_t v0 = smem_u32(sV + s * kTileBytes);
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk)
+              umma_ts(tmem + col_o_pp(i), tmem + col_p_pp(i) + kk * 8, sdesc_mnmajor_sw128(v0 + kk * 2048, kBox),
+                      IDESC_O, (j > 0 || kk > 0));
+            umma_commit(&pv_done[i]);
+            any_mma = true;
+          }
+          if (ok) umma_commit(&v_empty[s]);
+        }
+        if (*abort_flag && any_mma) {
+          umma_commit(drain_pv);
+          drain_wait(drain_pv, 0);
         }
       }
     }
@@ -604,7 +627,7 @@ __global__ void __launch_bounds__(kThreadsPP, 1)
     const int wg = (warp - 4) >> 2;  // query tile 0 or 1
     const int quarter = warp & 3;
     const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
-    const uint32_t colS = 128u * wg, colO = 256u + 128u * wg;
+    const uint32_t colO = col_o_pp(wg), colP = col_p_pp(wg);
     const int row = quarter * 32 + lane;
     const float sl2 = args.scale_log2;
     float m_ref = -INFINITY, l = 0.f;
@@ -618,15 +641,18 @@ __global__ void __launch_bounds__(kThreadsPP, 1)
         break;
       }
       tc_fence_after();
-      int c_lo, c_hi;
-      tile_cols(row_lo, row_hi, j0 + j, c_lo, c_hi);
-      const bool masked = !__all_sync(0xffffffffu, c_lo == 0 && c_hi == kTile);
-      // the whole row of S in registers (one wait for four loads)
+      // the whole row of S in registers (one wait for four loads), then the buffer goes
+      // back to the tensor core for the next product
       uint32_t r[4][32];
 #pragma unroll
-      for (int c = 0; c < 4; ++c) tmem_ld32(tmem + lane_base + colS + 32 * c, r[c]);
+      for (int c = 0; c < 4; ++c) tmem_ld32(tmem + lane_base + kColSPP + 32 * c, r[c]);
       tmem_wait_ld();
-      if (masked) {
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(s_free);
+      int c_lo, c_hi;
+      tile_cols(row_lo, row_hi, j0 + j, c_lo, c_hi);
+      if (!__all_sync(0xffffffffu, c_lo == 0 && c_hi == kTile)) {
 #pragma unroll
         for (int c = 0; c < 4; ++c) mask_chunk(r[c], 32 * c, c_lo, c_hi);
       }
@@ -640,31 +666,12 @@ __global__ void __launch_bounds__(kThreadsPP, 1)
         m_ref = mx;
         rescale = true;
       }
-      // O_i(j-1) is complete (it was issued before S_i(j)); rescale it if the max moved.
-      // PV_i(j) is issued only after P arrives below, so this precedes it.
-      if (kSplitP && j > 0 && __any_sync(0xffffffffu, rescale)) {
-#pragma unroll 1
-        for (int c = 0; c < 4; ++c) {
-          uint32_t o[32];
-          tmem_ld32(tmem + lane_base + colO + 32 * c, o);
-          tmem_wait_ld();
-#pragma unroll
-          for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-          tmem_st32(tmem + lane_base + colO + 32 * c, o);
-        }
-      }
       // exponentials, row sum, bf16 P packed in place over the scores already consumed
       const float m_use = m_ref == -INFINITY ? 0.f : m_ref;  // a row with no key seen yet
       const uint64_t sl2_2 = f2_pack(sl2, sl2), negm_2 = f2_pack(-m_use, -m_use);
       uint64_t sum2[4];  // one running pair sum per 32-column chunk: four short chains
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
-        if (kSplitP && c == 2) {  // the first 64 keys' P is complete: hand it over
-          tmem_st32(tmem + lane_base + colS, r[0]);
-          tmem_wait_st();
-          tc_fence_before();
-          mbar_arrive(&p_full[wg]);
-        }
 #pragma unroll
         for (int i = 0; i < 32; i += 2) {
           float x0, x1;
@@ -680,11 +687,17 @@ __global__ void __launch_bounds__(kThreadsPP, 1)
           r[c >> 1][(c & 1) * 16 + (i >> 1)] = pack_bf16x2(e0, e1);
         }
       }
-      if (!kSplitP) tmem_st32(tmem + lane_base + colS, r[0]);
-      tmem_st32(tmem + lane_base + colS + 32, r[1]);
-      // O_i(j-1) is complete (it was issued before S_i(j)); rescale it if the max moved.
-      // PV_i(j) is issued only after p_full below, so this precedes it.
-      if (!kSplitP && j > 0 && __any_sync(0xffffffffu, rescale)) {
+      if (j > 0) {
+        // P_i(j-1) V_{j-1} must be complete before O_i is rescaled or P_i overwritten
+        if (!mbar_wait_warp(&pv_done[wg], (j - 1) & 1, guard)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+      }
+      tmem_st32(tmem + lane_base + colP, r[0]);
+      tmem_st32(tmem + lane_base + colP + 32, r[1]);
+      if (j > 0 && __any_sync(0xffffffffu, rescale)) {
 #pragma unroll 1
         for (int c = 0; c < 4; ++c) {
           uint32_t o[32];
@@ -700,9 +713,9 @@ __global__ void __launch_bounds__(kThreadsPP, 1)
       l = l * alpha + (sum_lo + sum_hi);
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(kSplitP ? &p_half1[wg] : &p_full[wg]);
+      mbar_arrive(&p_full[wg]);
     }
-    if (ok && mbar_wait_warp(&o_final[wg], 0, guard)) {
+    if (ok && mbar_wait_warp(&pv_done[wg], (n_kv - 1) & 1, guard)) {
       tc_fence_after();
       const int64_t t = static_cast<int64_t>(2 * qt2 + wg) * kTile + row;
       const int b = bh / args.heads, h = bh % args.heads;
@@ -753,7 +766,7 @@ bool g_pp_ok[64] = {};  // the two-tile kernel's launch registers cover its warp
 
 // Makespan of n2 two-tile CTAs (cost kPairCost each, in units of one one-tile CTA over the
 // same keys) followed by n1 one-tile CTAs, placed in launch order on the first free SM.
-constexpr double kPairCost = 1.55;  // measured: 1.41 - 1.57 over 3,000 - 12,000 positions
+constexpr double kPairCost = 1.35;  // measured: 1.20 - 1.39 over 12,000 - 44,999 positions
 constexpr int kMinSplitTiles = 16;  // query tiles per clip below which no split is tried
 
 double makespan(uint64_t n2, uint64_t n1, int sms) {

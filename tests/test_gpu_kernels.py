@@ -125,7 +125,7 @@ def test_qkv_rope(batch, T):
 
 # ---------------------------------------------------------------- attention
 
-def _pairs_for_two_tile_kernel(batch, T, sms=148, rho=1.55):
+def _pairs_for_two_tile_kernel(batch, T, sms=148, rho=1.35):
     """Query-tile pairs per (clip, head) that the library gives the two-tile kernel (the
     rest go to the one-tile kernel launched behind it): the count, among none, all, or the
     largest filling whole waves, whose greedy schedule (a two-tile CTA costing rho one-tile
