@@ -427,24 +427,39 @@ __global__ void __launch_bounds__(192, 1)
 // Warpgroup 0 (loads, MMA issue) shrinks to kRegsCtrl registers per thread and the two
 // softmax warpgroups grow to kRegsSoftmax, so each softmax thread holds its whole row of
 // S (128 scores) and reads it from TMEM in one round trip per tile.
-constexpr size_t kSmemPP = 1024 + 6 * kTileBytes + 256;
-constexpr uint32_t kColSPP = 0;
-__device__ __forceinline__ uint32_t col_o_pp(int i) { return 128u + 128u * i; }
-__device__ __forceinline__ uint32_t col_p_pp(int i) { return 384u + 64u * i; }
 // Of every 16 score pairs of a row chunk, this many take their exponentials on the FMA
-// pipe (exp2_pair_poly) instead of the SFU.
+// pipe (exp2_pair_poly) instead of the SFU (head dim 128; at head dim 64 the MMAs of a tile
+// take half the time and 6 of 16 go to the FMA pipe).
 #ifndef SAL_PP_POLY_PAIRS
 #define SAL_PP_POLY_PAIRS 2
 #endif
-constexpr int kPolyPairsPP = SAL_PP_POLY_PAIRS;
+// Layout of the two-tile kernel per head dim. At 128 the TMEM holds one score buffer
+// shared by the two query tiles: S [0,128) O0 [128,256) O1 [256,384) P0 [384,448)
+// P1 [448,512). At 64 the accumulators are half as wide and each query tile has a score
+// buffer of its own: S0 [0,128) S1 [128,256) O0 [256,320) O1 [320,384) P0 P1 as above.
+template <int HD>
+struct PPLayout {
+  static constexpr int kTileB = kTile * HD * 2;  // a 128-row tile of Q, K or V
+  static constexpr int kBoxes = HD / 64;         // 64-column boxes of a tile
+  static constexpr bool kSharedS = HD == 128;
+  static constexpr size_t kSmem = 1024 + 6 * static_cast<size_t>(kTileB) + 256;
+  static constexpr int kPoly = HD == 64 ? 6 : SAL_PP_POLY_PAIRS;
+  __device__ static uint32_t col_s(int i) { return kSharedS ? 0u : 128u * i; }
+  __device__ static uint32_t col_o(int i) { return kSharedS ? 128u + 128u * i : 256u + 64u * i; }
+  __device__ static uint32_t col_p(int i) { return 384u + 64u * i; }
+};
+static_assert(PPLayout<128>::kSmem <= 227 * 1024 && PPLayout<64>::kSmem <= 227 * 1024, "shared memory");
 
 constexpr int kThreadsPP = 384;
 constexpr int kRegsCtrl = 80, kRegsSoftmax = 208;
 constexpr int kRegsNeededPP = kRegsCtrl * 128 + kRegsSoftmax * 256;  // <= launch regs x 384
 
+template <int HD>
 __global__ void __launch_bounds__(kThreadsPP, 1)
     attention_pp_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                         const __grid_constant__ CUtensorMap tmV, const AttnArgs args) {
+  using L = PPLayout<HD>;
+  constexpr int kTileBytes = L::kTileB;
   extern __shared__ unsigned char smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sQ = smem;                       // Q0, Q1
@@ -459,7 +474,9 @@ __global__ void __launch_bounds__(kThreadsPP, 1)
   uint64_t* s_full = bars + 9;    // [2] S_i(j) is in the score buffer
   uint64_t* p_full = bars + 11;   // [2] P_i(j) is in its region (O_i rescaled if needed)
   uint64_t* pv_done = bars + 13;  // [2] P_i(j) V_j has completed
-  uint64_t* s_free = bars + 15;   // the score buffer has been read (one phase per S)
+  // a score buffer has been read (one phase per S product in it): [0] is the shared
+  // buffer (head dim 128), [i] the buffer of query tile i (head dim 64)
+  uint64_t* s_free[2] = {bars + 15, bars + 20};
   uint64_t* drain = bars + 16;     // wind-down of the S issuer
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 17);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
@@ -487,7 +504,8 @@ __global__ void __launch_bounds__(kThreadsPP, 1)
       mbar_init(&p_full[s], 128);
       mbar_init(&pv_done[s], 1);
     }
-    mbar_init(s_free, 4);  // one arrival per warp of the warpgroup that read S
+    mbar_init(s_free[0], 4);  // one arrival per warp of the warpgroup that read S
+    mbar_init(s_free[1], 4);
     mbar_init(drain, 1);
     mbar_init(drain_pv, 1);
     *s_issued = 0;
@@ -517,45 +535,50 @@ __global__ void __launch_bounds__(kThreadsPP, 1)
     if (warp == 0) {
       if (lane == 0) {
         mbar_arrive_expect_tx(q_full, 2 * kTileBytes);
-        for (int i = 0; i < 2; ++i) {
-          tma_load_3d(sQ + i * kTileBytes, &tmQ, q_full, 0, (2 * qt2 + i) * kTile, bh);
-          tma_load_3d(sQ + i * kTileBytes + kBox, &tmQ, q_full, 64, (2 * qt2 + i) * kTile, bh);
-        }
+        for (int i = 0; i < 2; ++i)
+          for (int b = 0; b < L::kBoxes; ++b)
+            tma_load_3d(sQ + i * kTileBytes + b * kBox, &tmQ, q_full, 64 * b, (2 * qt2 + i) * kTile, bh);
         for (int j = 0; j < n_kv; ++j) {
           const int s = j & 1;
           const uint32_t use_par = (j >> 1) & 1;
           if (!mbar_wait(&k_empty[s], use_par ^ 1, guard)) break;
           if (j == args.withhold) continue;  // nothing issued: stage s keeps its last tracked loads
           mbar_arrive_expect_tx(&k_full[s], kTileBytes);
-          tma_load_3d(sK + s * kTileBytes, &tmK, &k_full[s], 0, (j0 + j) * kTile, bh);
-          tma_load_3d(sK + s * kTileBytes + kBox, &tmK, &k_full[s], 64, (j0 + j) * kTile, bh);
+          for (int b = 0; b < L::kBoxes; ++b)
+            tma_load_3d(sK + s * kTileBytes + b * kBox, &tmK, &k_full[s], 64 * b, (j0 + j) * kTile, bh);
           issued_k |= 1u << s;
           par_k = (par_k & ~(1u << s)) | (use_par << s);
           if (!mbar_wait(&v_empty[s], use_par ^ 1, guard)) break;
           mbar_arrive_expect_tx(&v_full[s], kTileBytes);
-          tma_load_3d(sV + s * kTileBytes, &tmV, &v_full[s], 0, (j0 + j) * kTile, bh);
-          tma_load_3d(sV + s * kTileBytes + kBox, &tmV, &v_full[s], 64, (j0 + j) * kTile, bh);
+          for (int b = 0; b < L::kBoxes; ++b)
+            tma_load_3d(sV + s * kTileBytes + b * kBox, &tmV, &v_full[s], 64 * b, (j0 + j) * kTile, bh);
           issued_v |= 1u << s;
           par_v = (par_v & ~(1u << s)) | (use_par << s);
         }
       }
     } else if (warp == 1) {
-      // S issue: S_i(x) into the shared score buffer, in the order S0_0 S1_0 S0_1 S1_1 ...
+      // S issue: S_i(x) into its score buffer, in the order S0_0 S1_0 S0_1 S1_1 ...
       if (lane == 0) {
         constexpr uint32_t IDESC_S = idesc_bf16(128, 128, false, false);
         bool any_mma = false;
         bool ok = mbar_wait(q_full, 0, guard);
         for (int q = 0; ok && q < 2 * n_kv; ++q) {
           const int i = q & 1, x = q >> 1, s = x & 1;
-          // the previous S product has been read out of the buffer, and K_x has landed
-          ok = (q == 0 || mbar_wait(s_free, (q - 1) & 1, guard)) && mbar_wait(&k_full[s], (x >> 1) & 1, guard);
+          // the previous S product in the same buffer has been read out of it (the shared
+          // buffer: the previous product; own buffers: this tile's previous one), and K_x
+          // has landed
+          const bool reuse = L::kSharedS ? q > 0 : x > 0;
+          const uint32_t par = L::kSharedS ? (q - 1) & 1 : (x - 1) & 1;
+          ok = (!reuse || mbar_wait(s_free[L::kSharedS ? 0 : i], par, guard)) &&
+               mbar_wait(&k_full[s], (x >> 1) & 1, guard);
           if (!ok) break;
           tc_fence_after();
           const uint32_t q0 = smem_u32(sQ + i * kTileBytes), k0 = smem_u32(sK + s * kTileBytes);
 #pragma unroll
-          for (int kk = 0; kk < 8; ++kk) {
+          for (int kk = 0; kk < HD / 16; ++kk) {
             const uint32_t off = (kk >> 2) * kBox + (kk & 3) * 32;
-            umma_ss(tmem + kColSPP, sdesc_kmajor_sw128(q0 + off), sdesc_kmajor_sw128(k0 + off), IDESC_S, kk > 0);
+            umma_ss(tmem + L::col_s(i), sdesc_kmajor_sw128(q0 + off), sdesc_kmajor_sw128(k0 + off), IDESC_S,
+                    kk > 0);
           }
           umma_commit(&s_full[i]);
           if (i == 1) umma_commit(&k_empty[s]);  // both products with K_x issued
@@ -574,7 +597,7 @@ __global__ void __launch_bounds__(kThreadsPP, 1)
       // critical path (the score buffer is shared), so P_i(j) V_j waits until S_i(j+1)
       // has been issued and then runs while warpgroup i reads S_i(j+1).
       if (lane == 0) {
-        constexpr uint32_t IDESC_O = idesc_bf16(128, 128, false, true);
+        constexpr uint32_t IDESC_O = idesc_bf16(128, HD, false, true);
         bool any_mma = false, ok = true;
         for (int j = 0; ok && j < n_kv; ++j) {
           const int s = j & 1;
@@ -608,7 +631,7 @@ __global__ void __launch_bounds__(kThreadsPP, 1)
             const uint32_t v0 = smem_u32(sV + s * kTileBytes);
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk)
-              umma_ts(tmem + col_o_pp(i), tmem + col_p_pp(i) + kk * 8, sdesc_mnmajor_sw128(v0 + kk * 2048, kBox),
+              umma_ts(tmem + L::col_o(i), tmem + L::col_p(i) + kk * 8, sdesc_mnmajor_sw128(v0 + kk * 2048, kBox),
                       IDESC_O, (j > 0 || kk > 0));
             umma_commit(&pv_done[i]);
             any_mma = true;
@@ -627,7 +650,7 @@ __global__ void __launch_bounds__(kThreadsPP, 1)
     const int wg = (warp - 4) >> 2;  // query tile 0 or 1
     const int quarter = warp & 3;
     const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
-    const uint32_t colO = col_o_pp(wg), colP = col_p_pp(wg);
+    const uint32_t colS = L::col_s(wg), colO = L::col_o(wg), colP = L::col_p(wg);
     const int row = quarter * 32 + lane;
     const float sl2 = args.scale_log2;
     float m_ref = -INFINITY, l = 0.f;
@@ -645,11 +668,11 @@ __global__ void __launch_bounds__(kThreadsPP, 1)
       // back to the tensor core for the next product
       uint32_t r[4][32];
 #pragma unroll
-      for (int c = 0; c < 4; ++c) tmem_ld32(tmem + lane_base + kColSPP + 32 * c, r[c]);
+      for (int c = 0; c < 4; ++c) tmem_ld32(tmem + lane_base + colS + 32 * c, r[c]);
       tmem_wait_ld();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(s_free);
+      if (lane == 0) mbar_arrive(s_free[L::kSharedS ? 0 : wg]);
       int c_lo, c_hi;
       tile_cols(row_lo, row_hi, j0 + j, c_lo, c_hi);
       if (!__all_sync(0xffffffffu, c_lo == 0 && c_hi == kTile)) {
@@ -677,7 +700,7 @@ __global__ void __launch_bounds__(kThreadsPP, 1)
           float x0, x1;
           f2_unpack(f2_fma(f2_pack(__uint_as_float(r[c][i]), __uint_as_float(r[c][i + 1])), sl2_2, negm_2), x0, x1);
           float e0, e1;
-          if (kPolyPairsPP > 0 && ((i >> 1) & 15) < kPolyPairsPP) {
+          if (L::kPoly > 0 && ((i >> 1) & 15) < L::kPoly) {
             exp2_pair_poly(x0, x1, e0, e1);  // on the FMA pipe, leaving the SFU to the others
           } else {
             e0 = fast_exp2(x0);
@@ -699,7 +722,7 @@ __global__ void __launch_bounds__(kThreadsPP, 1)
       tmem_st32(tmem + lane_base + colP + 32, r[1]);
       if (j > 0 && __any_sync(0xffffffffu, rescale)) {
 #pragma unroll 1
-        for (int c = 0; c < 4; ++c) {
+        for (int c = 0; c < HD / 32; ++c) {
           uint32_t o[32];
           tmem_ld32(tmem + lane_base + colO + 32 * c, o);
           tmem_wait_ld();
@@ -720,9 +743,9 @@ __global__ void __launch_bounds__(kThreadsPP, 1)
       const int64_t t = static_cast<int64_t>(2 * qt2 + wg) * kTile + row;
       const int b = bh / args.heads, h = bh % args.heads;
       const float inv_l = 1.0f / l;
-      __nv_bfloat16* dst = args.o + (static_cast<int64_t>(b) * T + t) * (args.heads * kHeadDim) + h * kHeadDim;
+      __nv_bfloat16* dst = args.o + (static_cast<int64_t>(b) * T + t) * (args.heads * HD) + h * HD;
 #pragma unroll 1
-      for (int c = 0; c < 4; ++c) {
+      for (int c = 0; c < HD / 32; ++c) {
         uint32_t o[32];
         tmem_ld32(tmem + lane_base + colO + 32 * c, o);
         tmem_wait_ld();
@@ -762,7 +785,8 @@ __global__ void __launch_bounds__(kThreadsPP, 1)
 
 std::mutex g_mu;
 bool g_attr[64] = {};
-bool g_pp_ok[64] = {};  // the two-tile kernel's launch registers cover its warpgroup split
+bool g_pp_ok[64] = {};    // the two-tile kernel's launch registers cover its warpgroup split
+bool g_pp_ok64[64] = {};  // the same for its head-dim-64 form
 
 // Makespan of n2 two-tile CTAs (cost kPairCost each, in units of one one-tile CTA over the
 // same keys) followed by n1 one-tile CTAs, placed in launch order on the first free SM.
@@ -837,15 +861,20 @@ sal_status attention_launch_heads(const void* q, const void* k, const void* v, i
                                static_cast<int>(smem_one_tile(128))) != cudaSuccess ||
           cudaFuncSetAttribute(attention_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                static_cast<int>(smem_one_tile(64))) != cudaSuccess ||
-          cudaFuncSetAttribute(attention_pp_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               static_cast<int>(kSmemPP)) != cudaSuccess)
+          cudaFuncSetAttribute(attention_pp_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               static_cast<int>(PPLayout<128>::kSmem)) != cudaSuccess ||
+          cudaFuncSetAttribute(attention_pp_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               static_cast<int>(PPLayout<64>::kSmem)) != cudaSuccess)
         return SAL_ECUDA;
       // setmaxnreg.inc waits until the registers it asks for are free: run the kernel only
       // if what warpgroup 0 gives back covers what the softmax warpgroups take (and the
       // launch count is one that 384 threads can get at all: at most 168)
-      cudaFuncAttributes fa{};
-      if (cudaFuncGetAttributes(&fa, attention_pp_kernel) != cudaSuccess) return SAL_ECUDA;
+      cudaFuncAttributes fa{}, fa64{};
+      if (cudaFuncGetAttributes(&fa, attention_pp_kernel<128>) != cudaSuccess ||
+          cudaFuncGetAttributes(&fa64, attention_pp_kernel<64>) != cudaSuccess)
+        return SAL_ECUDA;
       g_pp_ok[dev] = fa.numRegs * kThreadsPP >= kRegsNeededPP && fa.numRegs <= 168;
+      g_pp_ok64[dev] = fa64.numRegs * kThreadsPP >= kRegsNeededPP && fa64.numRegs <= 168;
       g_attr[dev] = true;
     }
   }
@@ -871,11 +900,26 @@ sal_status attention_launch_heads(const void* q, const void* k, const void* v, i
     a.win_total = win->total;
   }
   const dim3 grid1(static_cast<unsigned>((T + kTile - 1) / kTile), static_cast<unsigned>(bh));
-  if (head_dim == 64)
+  if (head_dim == 64) {
+    // the CTC adapter's heads: every query-tile pair to the two-tile kernel (the second
+    // tile of an odd count is empty), unless it is unavailable or switched off
+    bool pp64 = false;
+    {
+      std::lock_guard<std::mutex> lk(g_mu);
+      pp64 = dev >= 0 && dev < 64 && g_pp_ok64[dev];
+    }
+    if (pp64 && attention_pp_mode() != 0) {
+      const dim3 grid(static_cast<unsigned>((T + 2 * kTile - 1) / (2 * kTile)), static_cast<unsigned>(bh));
+      return launch_kernel(attention_pp_kernel<64>, grid, dim3(kThreadsPP), PPLayout<64>::kSmem, s, tq, tk, tv,
+                           a) == cudaSuccess
+                 ? SAL_OK
+                 : SAL_ECUDA;
+    }
     return launch_kernel(attention_kernel<64>, grid1, dim3(192), smem_one_tile(64), s, tq, tk, tv, a) ==
                    cudaSuccess
                ? SAL_OK
                : SAL_ECUDA;
+  }
   // Split the query tiles between the kernels: the two-tile kernel takes the first P pairs
   // of every (clip, head), the one-tile kernel the rest, launched right behind it so its
   // CTAs fill the SMs that two-tile CTAs leave. P is chosen by list scheduling (below).
@@ -900,7 +944,8 @@ sal_status attention_launch_heads(const void* q, const void* k, const void* v, i
   const int pp_tiles = 2 * P < n_qt ? 2 * P : n_qt;
   if (P > 0) {
     const dim3 grid(static_cast<unsigned>(P), static_cast<unsigned>(bh));
-    if (launch_kernel(attention_pp_kernel, grid, dim3(kThreadsPP), kSmemPP, s, tq, tk, tv, a) != cudaSuccess)
+    if (launch_kernel(attention_pp_kernel<128>, grid, dim3(kThreadsPP), PPLayout<128>::kSmem, s, tq, tk, tv, a) !=
+        cudaSuccess)
       return SAL_ECUDA;
   }
   if (pp_tiles == n_qt) return SAL_OK;

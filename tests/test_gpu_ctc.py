@@ -42,8 +42,10 @@ def _centred(a):
     return a - a.mean(axis=-1, keepdims=True)
 
 
-@pytest.mark.parametrize("batch,T", [(1, 1), (1, 127), (2, 300), (1, 749)])
+@pytest.mark.parametrize("batch,T", [(1, 1), (1, 127), (2, 300), (1, 749), (2, 640), (1, 1100)])
 def test_attention_16_heads_of_64(batch, T):
+    """Query tiles go to the two-tile kernel in pairs: odd tile counts (1, 127, 300, 640,
+    1,100 positions) leave the second tile of the last pair empty."""
     api = _api()
     q, q64 = rand_bf16((batch, 16, T, 64), 300 + T, 2.0)
     k, k64 = rand_bf16((batch, 16, T, 64), 310 + T, 1.0)
