@@ -996,9 +996,13 @@ extern "C" sal_status sal_attention_plan(int batch, int64_t T, int heads, int he
   const int n_qt = static_cast<int>((T + kTile - 1) / kTile);
   *query_tiles = n_qt;
   *pairs = 0;
-  if (head_dim != 128 || batch == 0 || T == 0 || heads == 0) return SAL_OK;
+  if ((head_dim != 128 && head_dim != 64) || batch == 0 || T == 0 || heads == 0) return SAL_OK;
   const uint64_t bh = static_cast<uint64_t>(batch) * heads;
   const int mode = attention_pp_mode();
+  if (head_dim == 64) {  // every pair to the two-tile kernel unless it is switched off
+    *pairs = mode == 0 ? 0 : (n_qt + 1) / 2;
+    return SAL_OK;
+  }
   *pairs = mode == 0 ? 0 : (mode == 1 ? (n_qt + 1) / 2 : choose_pairs(n_qt, bh, sms));
   return SAL_OK;
 }

@@ -119,7 +119,7 @@ def test_attention_plan_matches_the_stated_schedule(api):
     cases += [(b, T) for b in (1, 2) for T in (5000, 7499, 12000, 20000, 44999)]
     for batch, T in cases:
         assert api.attention_plan(batch, T) == _pairs_for_two_tile_kernel(batch, T), (batch, T)
-    assert api.attention_plan(1, 20000, heads=16, head_dim=64) == (0, 157)  # 64-wide heads: one-tile
+    assert api.attention_plan(1, 20000, heads=16, head_dim=64) == (79, 157)  # 64-wide heads: all pairs
     assert api.attention_plan(0, 100) == (0, 1)
     p, q = ctypes.c_int(), ctypes.c_int()
     assert api.lib().sal_attention_plan(1, 90001, 10, 128, 148, ctypes.byref(p), ctypes.byref(q)) == 2
