@@ -428,10 +428,15 @@ __global__ void __launch_bounds__(192, 1)
 // softmax warpgroups grow to kRegsSoftmax, so each softmax thread holds its whole row of
 // S (128 scores) and reads it from TMEM in one round trip per tile.
 // Of every 16 score pairs of a row chunk, this many take their exponentials on the FMA
-// pipe (exp2_pair_poly) instead of the SFU (head dim 128; at head dim 64 the MMAs of a tile
-// take half the time and 6 of 16 go to the FMA pipe).
+// pipe (exp2_pair_poly) instead of the SFU. Head dim 128: none, since the polynomial's
+// extra instructions slow the MMA-issuing threads that share the softmax warps' SM
+// sub-partitions (measured 3-5 % slower at 2 of 16). Head dim 64 (the MMAs of a tile take
+// half the time, the softmax is the bound): SAL_PP_POLY_PAIRS_HD64 of 16.
 #ifndef SAL_PP_POLY_PAIRS
-#define SAL_PP_POLY_PAIRS 2
+#define SAL_PP_POLY_PAIRS 0
+#endif
+#ifndef SAL_PP_POLY_PAIRS_HD64
+#define SAL_PP_POLY_PAIRS_HD64 6
 #endif
 // Layout of the two-tile kernel per head dim. At 128 the TMEM holds one score buffer
 // shared by the two query tiles: S [0,128) O0 [128,256) O1 [256,384) P0 [384,448)
@@ -443,7 +448,7 @@ struct PPLayout {
   static constexpr int kBoxes = HD / 64;         // 64-column boxes of a tile
   static constexpr bool kSharedS = HD == 128;
   static constexpr size_t kSmem = 1024 + 6 * static_cast<size_t>(kTileB) + 256;
-  static constexpr int kPoly = HD == 64 ? 6 : SAL_PP_POLY_PAIRS;
+  static constexpr int kPoly = HD == 64 ? SAL_PP_POLY_PAIRS_HD64 : SAL_PP_POLY_PAIRS;
   __device__ static uint32_t col_s(int i) { return kSharedS ? 0u : 128u * i; }
   __device__ static uint32_t col_o(int i) { return kSharedS ? 128u + 128u * i : 256u + 64u * i; }
   __device__ static uint32_t col_p(int i) { return 384u + 64u * i; }

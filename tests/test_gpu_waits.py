@@ -62,3 +62,19 @@ def test_withhold_beyond_the_last_tile_changes_nothing():
     assert api.sal_last_device_status() == 0
     b = api.sal_attention(q, k, v)
     assert np.array_equal(to64(a), to64(b))
+
+
+def test_one_and_two_tile_kernels_agree_bit_for_bit():
+    """With no tile withheld (an index past every CTA's key tiles), the hook forces the
+    one-tile kernel (1) or the two-tile kernel for every query-tile pair (2). At head dim 128
+    both do the same per-row arithmetic in the same order, so their outputs are equal bit
+    for bit; 1,000 positions give 8 query tiles (4 pairs) over 8 key tiles."""
+    from speech_audio_encoder_b200 import api
+    T = 1000
+    q, _ = rand_bf16((1, 10, T, 128), 91, 1.0)
+    k, _ = rand_bf16((1, 10, T, 128), 92, 1.0)
+    v, _ = rand_bf16((1, 10, T, 128), 93, 1.0)
+    one = to64(api.sal_attention_withhold(q, k, v, 1, 1000))
+    two = to64(api.sal_attention_withhold(q, k, v, 2, 1000))
+    assert api.sal_last_device_status() == 0
+    assert np.array_equal(one, two)
