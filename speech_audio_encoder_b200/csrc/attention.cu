@@ -409,21 +409,27 @@ __global__ void __launch_bounds__(192, 1)
 }
 
 // ---------------------------------------------------------------------------------
-// Ping-pong variant for long clips: one CTA owns TWO 128-row query tiles of one
+// Two-tile variant for long clips: one CTA owns TWO 128-row query tiles of one
 // (clip, head), so each K / V tile loaded serves 256 queries, and two softmax warpgroups
 // take turns with the tensor core.
 //   warp 0: TMA loads (Q0 and Q1 once; K_j and V_j through two-stage rings released
 //           separately: K after both S products, V after both P V products)
-//   warp 1: tcgen05.mma issue, in the order S0_0 S1_0 | S0_{j+1} PV0_j S1_{j+1} PV1_j ...
-//   warps 2-3: idle (they complete warpgroup 0, which gives registers away)
+//   warp 1: issues the S products, S0_0 S1_0 S0_1 S1_1 ..., each as soon as its score
+//           buffer is free
+//   warp 2: issues the P V products, P_i(j) V_j once P_i(j) is stored and S_i(j+1) has
+//           been issued (the tensor core runs MMAs in issue order: an S product, on the
+//           critical path, never waits behind a P V product). Two issuing threads,
+//           because one thread takes nearly as long to issue a 128 x 128 x 16 MMA as the
+//           tensor core takes to run it.
+//   warp 3: idle (it completes warpgroup 0, which gives registers away)
 //   warps 4-7 / 8-11: softmax of query tile 0 / 1, one row per thread
-// TMEM: S [0,128) O0 [128,256) O1 [256,384) P0 [384,448) P1 [448,512). The one score
-// buffer S is shared by the two query tiles: a warpgroup copies its S_i(j) into registers
-// and hands the buffer back at once, so the next product (the other tile's S, then its
-// own S_i(j+1)) runs on the tensor core while its exponentials are computed. P_i (bf16
-// pairs) has a region of its own, so S_i(j+1) does not wait for P_i(j) V_j. The
+// TMEM at head dim 128: S [0,128) O0 [128,256) O1 [256,384) P0 [384,448) P1 [448,512).
+// The one score buffer S is shared by the two query tiles: a warpgroup copies its S_i(j)
+// into registers and hands the buffer back at once, so the next product (the other tile's
+// S, then its own S_i(j+1)) runs on the tensor core while its exponentials are computed.
+// P_i (bf16 pairs) has a region of its own, so S_i(j+1) does not wait for P_i(j) V_j. The
 // warpgroup waits for P_i(j-1) V_{j-1} to complete before it rescales O_i or overwrites
-// P_i.
+// P_i. At head dim 64 each query tile has a score buffer of its own (PPLayout).
 // Warpgroup 0 (loads, MMA issue) shrinks to kRegsCtrl registers per thread and the two
 // softmax warpgroups grow to kRegsSoftmax, so each softmax thread holds its whole row of
 // S (128 scores) and reads it from TMEM in one round trip per tile.
