@@ -352,13 +352,16 @@ sal_status sal_attention_heads(const void* q, const void* k, const void* v, int 
                                int head_dim, void* o, void* stream);
 
 /* The kernels sal_attention would launch for 128-wide heads on a GPU with `sms` SMs:
- * *pairs query-tile pairs (of 128 rows) per (clip, head) go to the two-tile kernel and the
- * remaining of the *query_tiles tiles to the one-tile kernel launched behind it. P is the
+ * *pairs query-tile pairs (of 128 rows) per (clip, head) go to the two-tile kernel, out of
+ * *query_tiles tiles. P is the
  * count among none, all and the largest filling whole waves whose greedy schedule ends
  * first (a two-tile CTA counted as 1.35 one-tile CTAs); splits are tried from 16 query
- * tiles up. For head_dim 64 every pair goes to the two-tile kernel (*pairs = all). In both
- * cases SAL_ATTN_PP=0/1 in the environment forces none/all. Host arithmetic only: no
- * device is needed. */
+ * tiles up. The tiles past the pairs go to split-mode CTAs of the same launch (a tile's keys
+ * split between the CTA's two warpgroups), counted as 0.75 one-tile CTAs; with no pairs
+ * the one-tile kernel takes every tile. For head_dim 64 every pair goes to the two-tile
+ * kernel and an odd last tile to a split-mode CTA. SAL_ATTN_PP=0/1 in the environment
+ * forces none/all; SAL_ATTN_PAIRS=n forces n pairs and split mode for the rest. Host
+ * arithmetic only: no device is needed. */
 sal_status sal_attention_plan(int batch, int64_t T, int heads, int head_dim, int sms, int* pairs, int* query_tiles);
 /* (sal_attention_plan returns SAL_ESHAPE for T > 90,000, as sal_attention_heads does.) */
 

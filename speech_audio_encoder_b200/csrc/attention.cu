@@ -34,7 +34,6 @@ namespace {
 
 constexpr int kTile = 128;
 constexpr int kBox = kTile * 64 * 2;       // one 64-column half of a 128 x 128 bf16 tile
-constexpr int kTileBytes = 2 * kBox;       // 32 KB
 constexpr uint32_t kColO = 256;
 __device__ __forceinline__ uint32_t col_s(int s) { return s ? 128u : 0u; }    // score buffers
 __device__ __forceinline__ uint32_t col_p(int s) { return s ? 448u : 384u; }  // bf16 P buffers
@@ -53,9 +52,22 @@ int attention_pp_mode() {
   return mode;
 }
 
+// SAL_ATTN_PAIRS=n (n >= 0) in the environment forces the two-tile kernel with n pairs per
+// (clip, head), clamped to all of them, and every other tile in split mode (n = 0: every
+// tile split). For measuring the split cost; -1 when unset.
+int attention_pairs_forced() {
+  static const int n = [] {
+    const char* e = std::getenv("SAL_ATTN_PAIRS");
+    return e && e[0] >= '0' && e[0] <= '9' ? std::atoi(e) : -1;
+  }();
+  return n;
+}
+
 struct AttnArgs {
-  int qt0 = 0;    // one-tile kernel: first query tile of this launch
-  int tail = 0;   // one-tile kernel launched behind the two-tile kernel (see attention_launch_heads)
+  // two-tile kernel: CTAs x < pairs take the query-tile pair (2x, 2x + 1); each CTA past
+  // them takes one query tile, 2 pairs + (x - pairs), split over the keys between its two
+  // warpgroups (key tiles 0, 2, 4, ... and 1, 3, 5, ...) and merged at the end
+  int pairs = 0;
   int64_t T;
   int64_t chunk;  // attention stays inside chunks of this many positions (T: whole clip)
   int heads;
@@ -166,7 +178,7 @@ __global__ void __launch_bounds__(192, 1)
   const int lane = threadIdx.x & 31;
   const int64_t T = args.T;
   const int bh = blockIdx.y;
-  const int qt = blockIdx.x + args.qt0;
+  const int qt = blockIdx.x;
   const int64_t Tk = valid_len(args, bh / args.heads);  // key positions of this clip
   int j0, n_kv;
   kv_tile_range(static_cast<int64_t>(qt) * kTile, static_cast<int64_t>(qt) * kTile + kTile, Tk, args.chunk, j0,
@@ -196,10 +208,7 @@ __global__ void __launch_bounds__(192, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  // A tail launch reads only what the two-tile kernel ahead of it had already waited for
-  // (its CTAs start after every two-tile CTA passed griddepcontrol.wait), so it starts at
-  // once and waits for that kernel at exit instead, before its own completion.
-  if (!args.tail) pdl_wait();
+  pdl_wait();
   pdl_trigger();
   const uint32_t tmem = *tmem_slot;
   const WaitGuard guard{abort_flag, args.limit_ns, args.status};
@@ -405,15 +414,16 @@ __global__ void __launch_bounds__(192, 1)
         drain_wait(&v_full[s], (par_k >> s) & 1);
       }
   }
-  if (args.tail) pdl_wait();
 }
 
 // ---------------------------------------------------------------------------------
 // Two-tile variant for long clips: one CTA owns TWO 128-row query tiles of one
 // (clip, head), so each K / V tile loaded serves 256 queries, and two softmax warpgroups
-// take turns with the tensor core.
-//   warp 0: TMA loads (Q0 and Q1 once; K_j and V_j through two-stage rings released
-//           separately: K after both S products, V after both P V products)
+// take turns with the tensor core. CTAs past args.pairs take one query tile in split mode:
+// both warpgroups work on it, on alternate key tiles, and merge their results at the end.
+//   warp 0: TMA loads of Q0 and Q1 once and of K_j through a two-stage ring, released
+//           after the S products that read it
+//   warp 3: TMA loads of V_j through a two-stage ring, released after its P V products
 //   warp 1: issues the S products, S0_0 S1_0 S0_1 S1_1 ..., each as soon as its score
 //           buffer is free
 //   warp 2: issues the P V products, P_i(j) V_j once P_i(j) is stored and S_i(j+1) has
@@ -421,7 +431,6 @@ __global__ void __launch_bounds__(192, 1)
 //           critical path, never waits behind a P V product). Two issuing threads,
 //           because one thread takes nearly as long to issue a 128 x 128 x 16 MMA as the
 //           tensor core takes to run it.
-//   warp 3: idle (it completes warpgroup 0, which gives registers away)
 //   warps 4-7 / 8-11: softmax of query tile 0 / 1, one row per thread
 // TMEM at head dim 128: S [0,128) O0 [128,256) O1 [256,384) P0 [384,448) P1 [448,512).
 // The one score buffer S is shared by the two query tiles: a warpgroup copies its S_i(j)
@@ -453,7 +462,7 @@ struct PPLayout {
   static constexpr int kTileB = kTile * HD * 2;  // a 128-row tile of Q, K or V
   static constexpr int kBoxes = HD / 64;         // 64-column boxes of a tile
   static constexpr bool kSharedS = HD == 128;
-  static constexpr size_t kSmem = 1024 + 6 * static_cast<size_t>(kTileB) + 256;
+  static constexpr size_t kSmem = 1024 + 6 * static_cast<size_t>(kTileB) + 256 + 2048;  // + split-mode merge
   static constexpr int kPoly = HD == 64 ? SAL_PP_POLY_PAIRS_HD64 : SAL_PP_POLY_PAIRS;
   __device__ static uint32_t col_s(int i) { return kSharedS ? 0u : 128u * i; }
   __device__ static uint32_t col_o(int i) { return kSharedS ? 128u + 128u * i : 256u + 64u * i; }
@@ -461,11 +470,27 @@ struct PPLayout {
 };
 static_assert(PPLayout<128>::kSmem <= 227 * 1024 && PPLayout<64>::kSmem <= 227 * 1024, "shared memory");
 
+// 32 consecutive output columns of one row: bf16(a * x[i] + b * y[i]), 64 bytes.
+__device__ __forceinline__ void store_row32(__nv_bfloat16* dst, const uint32_t (&x)[32], float a, float b,
+                                            const uint32_t (&y)[32]) {
+  uint4* d4 = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    float v[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) v[e] = fmaf(__uint_as_float(y[8 * i + e]), b, __uint_as_float(x[8 * i + e]) * a);
+    d4[i] = make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]), pack_bf16x2(v[4], v[5]),
+                       pack_bf16x2(v[6], v[7]));
+  }
+}
+
 constexpr int kThreadsPP = 384;
-constexpr int kRegsCtrl = 80, kRegsSoftmax = 208;
+constexpr int kRegsCtrl = 104, kRegsSoftmax = 200;
 constexpr int kRegsNeededPP = kRegsCtrl * 128 + kRegsSoftmax * 256;  // <= launch regs x 384
 
-template <int HD>
+// SPLIT: the launch may hold split-mode CTAs. A launch of pairs only runs the form without
+// the split-mode code, whose registers and branches it would otherwise carry.
+template <int HD, bool SPLIT>
 __global__ void __launch_bounds__(kThreadsPP, 1)
     attention_pp_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                         const __grid_constant__ CUtensorMap tmV, const AttnArgs args) {
@@ -493,16 +518,25 @@ __global__ void __launch_bounds__(kThreadsPP, 1)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   uint64_t* drain_pv = bars + 18;  // wind-down of the P V issuer
   volatile int* s_issued = reinterpret_cast<volatile int*>(bars + 19);  // S products issued so far
+  uint64_t* merge_bar = bars + 21;  // split mode: both warpgroups' final (m, l) are written
+  float* merge_ml = reinterpret_cast<float*>(smem + 6 * kTileBytes + 256);  // [2][128][2]
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int64_t T = args.T;
   const int bh = blockIdx.y;
-  const int qt2 = blockIdx.x;  // 256-row query block
+  const bool split = SPLIT && static_cast<int>(blockIdx.x) >= args.pairs;
+  const int qt2 = blockIdx.x;                                    // pair mode: 256-row query block
+  const int qt1 = 2 * args.pairs + (static_cast<int>(blockIdx.x) - args.pairs);  // split mode: query tile
   const int64_t Tk = valid_len(args, bh / args.heads);  // key positions of this clip
   int j0, n_kv;
-  kv_tile_range(static_cast<int64_t>(qt2) * 2 * kTile, static_cast<int64_t>(qt2) * 2 * kTile + 2 * kTile, Tk,
-                args.chunk, j0, n_kv);
+  {
+    const int64_t q_lo = split ? static_cast<int64_t>(qt1) * kTile : static_cast<int64_t>(qt2) * 2 * kTile;
+    kv_tile_range(q_lo, q_lo + (split ? kTile : 2 * kTile), Tk, args.chunk, j0, n_kv);
+  }
+  // S products (and P V products) of the CTA, q = 2 x + i for warpgroup i's x-th: over
+  // key tile x (pair mode) or key tile q (split mode)
+  const int n_prod = split ? n_kv : 2 * n_kv;
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
@@ -519,6 +553,7 @@ __global__ void __launch_bounds__(kThreadsPP, 1)
     mbar_init(s_free[1], 4);
     mbar_init(drain, 1);
     mbar_init(drain_pv, 1);
+    mbar_init(merge_bar, 256);
     *s_issued = 0;
     *abort_flag = 0;
     fence_mbar_init();
@@ -545,10 +580,12 @@ __global__ void __launch_bounds__(kThreadsPP, 1)
     setmaxnreg_dec<kRegsCtrl>();
     if (warp == 0) {
       if (lane == 0) {
-        mbar_arrive_expect_tx(q_full, 2 * kTileBytes);
-        for (int i = 0; i < 2; ++i)
+        const int nq = split ? 1 : 2;  // split mode: both warpgroups use Q0
+        mbar_arrive_expect_tx(q_full, nq * kTileBytes);
+        for (int i = 0; i < nq; ++i)
           for (int b = 0; b < L::kBoxes; ++b)
-            tma_load_3d(sQ + i * kTileBytes + b * kBox, &tmQ, q_full, 64 * b, (2 * qt2 + i) * kTile, bh);
+            tma_load_3d(sQ + i * kTileBytes + b * kBox, &tmQ, q_full, 64 * b, (split ? qt1 : 2 * qt2 + i) * kTile,
+                        bh);
         for (int j = 0; j < n_kv; ++j) {
           const int s = j & 1;
           const uint32_t use_par = (j >> 1) & 1;
@@ -559,7 +596,28 @@ __global__ void __launch_bounds__(kThreadsPP, 1)
             tma_load_3d(sK + s * kTileBytes + b * kBox, &tmK, &k_full[s], 64 * b, (j0 + j) * kTile, bh);
           issued_k |= 1u << s;
           par_k = (par_k & ~(1u << s)) | (use_par << s);
+          if constexpr (!SPLIT) {  // pairs only: V_j right behind K_j from the same thread
+            if (!mbar_wait(&v_empty[s], use_par ^ 1, guard)) break;
+            mbar_arrive_expect_tx(&v_full[s], kTileBytes);
+            for (int b = 0; b < L::kBoxes; ++b)
+              tma_load_3d(sV + s * kTileBytes + b * kBox, &tmV, &v_full[s], 64 * b, (j0 + j) * kTile, bh);
+            issued_v |= 1u << s;
+            par_v = (par_v & ~(1u << s)) | (use_par << s);
+          }
+        }
+      }
+    } else if (warp == 3) {
+      // With split-mode CTAs in the launch, V loads come from a thread of their own: a V
+      // stage frees up only after its P V product, which must not hold back the next K tile
+      // (in split mode each stage serves one warpgroup, and V_j's stage is free only after
+      // that warpgroup's P V of tile j - 2). Without them a second polling thread costs the
+      // softmax warps that share its SM sub-partition more than it gains.
+      if (SPLIT && lane == 0) {
+        for (int j = 0; j < n_kv; ++j) {
+          const int s = j & 1;
+          const uint32_t use_par = (j >> 1) & 1;
           if (!mbar_wait(&v_empty[s], use_par ^ 1, guard)) break;
+          if (j == args.withhold) continue;  // nothing issued: stage s keeps its last tracked load
           mbar_arrive_expect_tx(&v_full[s], kTileBytes);
           for (int b = 0; b < L::kBoxes; ++b)
             tma_load_3d(sV + s * kTileBytes + b * kBox, &tmV, &v_full[s], 64 * b, (j0 + j) * kTile, bh);
@@ -573,18 +631,20 @@ __global__ void __launch_bounds__(kThreadsPP, 1)
         constexpr uint32_t IDESC_S = idesc_bf16(128, 128, false, false);
         bool any_mma = false;
         bool ok = mbar_wait(q_full, 0, guard);
-        for (int q = 0; ok && q < 2 * n_kv; ++q) {
-          const int i = q & 1, x = q >> 1, s = x & 1;
+        for (int q = 0; ok && q < n_prod; ++q) {
+          const int i = q & 1, x = q >> 1;
+          const int jk = split ? q : x;  // key tile (from j0), in stage jk & 1
+          const int s = jk & 1;
           // the previous S product in the same buffer has been read out of it (the shared
           // buffer: the previous product; own buffers: this tile's previous one), and K_x
           // has landed
           const bool reuse = L::kSharedS ? q > 0 : x > 0;
           const uint32_t par = L::kSharedS ? (q - 1) & 1 : (x - 1) & 1;
           ok = (!reuse || mbar_wait(s_free[L::kSharedS ? 0 : i], par, guard)) &&
-               mbar_wait(&k_full[s], (x >> 1) & 1, guard);
+               mbar_wait(&k_full[s], (jk >> 1) & 1, guard);
           if (!ok) break;
           tc_fence_after();
-          const uint32_t q0 = smem_u32(sQ + i * kTileBytes), k0 = smem_u32(sK + s * kTileBytes);
+          const uint32_t q0 = smem_u32(sQ + (split ? 0 : i) * kTileBytes), k0 = smem_u32(sK + s * kTileBytes);
 #pragma unroll
           for (int kk = 0; kk < HD / 16; ++kk) {
             const uint32_t off = (kk >> 2) * kBox + (kk & 3) * 32;
@@ -592,7 +652,7 @@ __global__ void __launch_bounds__(kThreadsPP, 1)
                     kk > 0);
           }
           umma_commit(&s_full[i]);
-          if (i == 1) umma_commit(&k_empty[s]);  // both products with K_x issued
+          if (split || i == 1) umma_commit(&k_empty[s]);  // every product with this K tile issued
           any_mma = true;
           *s_issued = q + 1;
         }
@@ -610,15 +670,61 @@ __global__ void __launch_bounds__(kThreadsPP, 1)
       if (lane == 0) {
         constexpr uint32_t IDESC_O = idesc_bf16(128, HD, false, true);
         bool any_mma = false, ok = true;
-        for (int j = 0; ok && j < n_kv; ++j) {
-          const int s = j & 1;
-          for (int i = 0; i < 2; ++i) {
-            ok = mbar_wait(&p_full[i], j & 1, guard) && mbar_wait(&v_full[s], (j >> 1) & 1, guard);
+        if constexpr (!SPLIT && HD == 64) {
+          // head dim 64, pairs only: per key tile, P0 V then P1 V. A P V MMA is 32 cycles of
+          // tensor work here, and this nested form issues faster than the flat loop below
+          // (measured 10.1 against 11.2 ms at 44,999 positions); at head dim 128 the flat
+          // loop measured faster.
+          for (int j = 0; ok && j < n_kv; ++j) {
+            const int s = j & 1;
+            for (int i = 0; i < 2; ++i) {
+              ok = mbar_wait(&p_full[i], j & 1, guard) && mbar_wait(&v_full[s], (j >> 1) & 1, guard);
+              if (!ok) break;
+              if (j + 1 < n_kv) {
+                // a plain spin (the wait is short and its end is on the critical path); the
+                // bound is checked every 64 polls
+                const int need = 2 * (j + 1) + i + 1;
+                uint64_t t0 = 0;
+                for (uint32_t spin = 1; *s_issued < need; ++spin) {
+                  if ((spin & 63) != 0) continue;
+                  if (*abort_flag) {
+                    ok = false;
+                    break;
+                  }
+                  const uint64_t now = globaltimer_ns();
+                  if (t0 == 0) {
+                    t0 = now;
+                  } else if (now - t0 > args.limit_ns) {
+                    *abort_flag = 1;
+                    atomicOr(args.status, kStatusTimeout);
+                    ok = false;
+                    break;
+                  }
+                }
+                if (!ok) break;
+              }
+              tc_fence_after();
+              const uint32_t v0 = smem_u32(sV + s * kTileBytes);
+#pragma unroll
+              for (int kk = 0; kk < 8; ++kk)
+                umma_ts(tmem + L::col_o(i), tmem + L::col_p(i) + kk * 8, sdesc_mnmajor_sw128(v0 + kk * 2048, kBox),
+                        IDESC_O, (j > 0 || kk > 0));
+              umma_commit(&pv_done[i]);
+              any_mma = true;
+            }
+            if (ok) umma_commit(&v_empty[s]);
+          }
+        } else {
+          for (int q = 0; ok && q < n_prod; ++q) {
+            const int i = q & 1, x = q >> 1;
+            const int jk = split ? q : x;  // key tile (from j0), in stage jk & 1
+            const int s = jk & 1;
+            ok = mbar_wait(&p_full[i], x & 1, guard) && mbar_wait(&v_full[s], (jk >> 1) & 1, guard);
             if (!ok) break;
-            if (j + 1 < n_kv) {
-              // a plain spin (the wait is short and its end is on the critical path); the
-              // bound is checked every 64 polls
-              const int need = 2 * (j + 1) + i + 1;
+            if (q + 2 < n_prod) {
+              // S_i(x+1) (product q + 2) must have been issued; a plain spin (the wait is short
+              // and its end is on the critical path), the bound checked every 64 polls
+              const int need = q + 3;
               uint64_t t0 = 0;
               for (uint32_t spin = 1; *s_issued < need; ++spin) {
                 if ((spin & 63) != 0) continue;
@@ -643,11 +749,11 @@ __global__ void __launch_bounds__(kThreadsPP, 1)
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk)
               umma_ts(tmem + L::col_o(i), tmem + L::col_p(i) + kk * 8, sdesc_mnmajor_sw128(v0 + kk * 2048, kBox),
-                      IDESC_O, (j > 0 || kk > 0));
+                      IDESC_O, (x > 0 || kk > 0));
             umma_commit(&pv_done[i]);
+            if (split || i == 1) umma_commit(&v_empty[s]);  // every product with this V tile issued
             any_mma = true;
           }
-          if (ok) umma_commit(&v_empty[s]);
         }
         if (*abort_flag && any_mma) {
           umma_commit(drain_pv);
@@ -667,9 +773,12 @@ __global__ void __launch_bounds__(kThreadsPP, 1)
     float m_ref = -INFINITY, l = 0.f;
     bool ok = true;
     int row_lo, row_hi;
-    row_range((2 * qt2 + wg) * kTile + row, static_cast<int>(T), static_cast<int>(Tk), static_cast<int>(args.chunk),
-              row_lo, row_hi);
-    for (int j = 0; j < n_kv; ++j) {
+    row_range((split ? qt1 : 2 * qt2 + wg) * kTile + row, static_cast<int>(T), static_cast<int>(Tk),
+              static_cast<int>(args.chunk), row_lo, row_hi);
+    // this warpgroup's key tiles: all n_kv (pair mode), or every other one from wg (split)
+    const int n_my = split ? (n_kv + 1 - wg) / 2 : n_kv;
+    for (int j = 0; j < n_my; ++j) {
+      const int jk = split ? 2 * j + wg : j;  // key tile (from j0)
       if (!mbar_wait_warp(&s_full[wg], j & 1, guard)) {
         ok = false;
         break;
@@ -685,7 +794,7 @@ __global__ void __launch_bounds__(kThreadsPP, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(s_free[L::kSharedS ? 0 : wg]);
       int c_lo, c_hi;
-      tile_cols(row_lo, row_hi, j0 + j, c_lo, c_hi);
+      tile_cols(row_lo, row_hi, j0 + jk, c_lo, c_hi);
       if (!__all_sync(0xffffffffu, c_lo == 0 && c_hi == kTile)) {
 #pragma unroll
         for (int c = 0; c < 4; ++c) mask_chunk(r[c], 32 * c, c_lo, c_hi);
@@ -749,28 +858,50 @@ __global__ void __launch_bounds__(kThreadsPP, 1)
       tc_fence_before();
       mbar_arrive(&p_full[wg]);
     }
-    if (ok && mbar_wait_warp(&pv_done[wg], (n_kv - 1) & 1, guard)) {
-      tc_fence_after();
-      const int64_t t = static_cast<int64_t>(2 * qt2 + wg) * kTile + row;
-      const int b = bh / args.heads, h = bh % args.heads;
-      const float inv_l = 1.0f / l;
-      __nv_bfloat16* dst = args.o + (static_cast<int64_t>(b) * T + t) * (args.heads * HD) + h * HD;
+    const int b = bh / args.heads, h = bh % args.heads;
+    if (!split) {
+      if (ok && mbar_wait_warp(&pv_done[wg], (n_my - 1) & 1, guard)) {
+        tc_fence_after();
+        const int64_t t = static_cast<int64_t>(2 * qt2 + wg) * kTile + row;
+        const float inv_l = 1.0f / l;
+        __nv_bfloat16* dst = args.o + (static_cast<int64_t>(b) * T + t) * (args.heads * HD) + h * HD;
 #pragma unroll 1
-      for (int c = 0; c < HD / 32; ++c) {
-        uint32_t o[32];
-        tmem_ld32(tmem + lane_base + colO + 32 * c, o);
-        tmem_wait_ld();
-        if (t < T) {
-          uint4* d4 = reinterpret_cast<uint4*>(dst + 32 * c);
-#pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            uint4 u;
-            u.x = pack_bf16x2(__uint_as_float(o[8 * i + 0]) * inv_l, __uint_as_float(o[8 * i + 1]) * inv_l);
-            u.y = pack_bf16x2(__uint_as_float(o[8 * i + 2]) * inv_l, __uint_as_float(o[8 * i + 3]) * inv_l);
-            u.z = pack_bf16x2(__uint_as_float(o[8 * i + 4]) * inv_l, __uint_as_float(o[8 * i + 5]) * inv_l);
-            u.w = pack_bf16x2(__uint_as_float(o[8 * i + 6]) * inv_l, __uint_as_float(o[8 * i + 7]) * inv_l);
-            d4[i] = u;
-          }
+        for (int c = 0; c < HD / 32; ++c) {
+          uint32_t o[32];
+          tmem_ld32(tmem + lane_base + colO + 32 * c, o);
+          tmem_wait_ld();
+          if (t < T) store_row32(dst + 32 * c, o, inv_l, 0.f, o);
+        }
+      }
+    } else {
+      // Both warpgroups hold a partial result for the same rows (the keys split between
+      // them). Once both are final, each writes half of the columns of
+      //   O = (O0 2^(m0 - m) + O1 2^(m1 - m)) / (l0 2^(m0 - m) + l1 2^(m1 - m)), m = max(m0, m1),
+      // reading both accumulators (every warp reaches both regions in its lane quarter).
+      // Every softmax thread arrives on merge_bar once, aborted or not.
+      const bool mine = ok && (n_my == 0 || mbar_wait_warp(&pv_done[wg], (n_my - 1) & 1, guard));
+      merge_ml[(wg * 128 + row) * 2 + 0] = m_ref;
+      merge_ml[(wg * 128 + row) * 2 + 1] = mine ? l : 0.f;
+      mbar_arrive(merge_bar);
+      if (mine && mbar_wait_warp(merge_bar, 0, guard) && !*abort_flag) {
+        tc_fence_after();
+        const float m0 = merge_ml[row * 2], l0 = merge_ml[row * 2 + 1];
+        const float m1 = merge_ml[(128 + row) * 2], l1 = merge_ml[(128 + row) * 2 + 1];
+        const float m = fmaxf(m0, m1);
+        // a part that saw no key has l = 0 (and m = -inf): its weight is 0
+        const float a0 = l0 > 0.f ? fast_exp2(m0 - m) : 0.f, a1 = l1 > 0.f ? fast_exp2(m1 - m) : 0.f;
+        const float lsum = l0 * a0 + l1 * a1;
+        const float inv = lsum > 0.f ? 1.0f / lsum : 0.f;
+        const int64_t t = static_cast<int64_t>(qt1) * kTile + row;
+        __nv_bfloat16* dst = args.o + (static_cast<int64_t>(b) * T + t) * (args.heads * HD) + h * HD;
+#pragma unroll 1
+        for (int c = 0; c < HD / 64; ++c) {
+          const uint32_t col = static_cast<uint32_t>(wg * (HD / 2) + 32 * c);
+          uint32_t o0[32], o1[32];
+          tmem_ld32(tmem + lane_base + L::col_o(0) + col, o0);
+          tmem_ld32(tmem + lane_base + L::col_o(1) + col, o1);
+          tmem_wait_ld();
+          if (t < T) store_row32(dst + col, o0, a0 * inv, a1 * inv, o1);
         }
       }
     }
@@ -785,8 +916,8 @@ __global__ void __launch_bounds__(kThreadsPP, 1)
   }
   // Every role has finished, so the abort flag is final: let every load this CTA issued
   // land before the CTA, and its shared memory, goes away.
-  if (warp == 0 && lane == 0 && *abort_flag) {
-    drain_wait(q_full, 0);
+  if (lane == 0 && (warp == 0 || warp == 3) && *abort_flag) {  // each producer drains its own loads
+    if (warp == 0) drain_wait(q_full, 0);
     for (int s = 0; s < 2; ++s) {
       if (issued_k & (1u << s)) drain_wait(&k_full[s], (par_k >> s) & 1);
       if (issued_v & (1u << s)) drain_wait(&v_full[s], (par_v >> s) & 1);
@@ -797,32 +928,59 @@ __global__ void __launch_bounds__(kThreadsPP, 1)
 std::mutex g_mu;
 bool g_attr[64] = {};
 bool g_pp_ok[64] = {};    // the two-tile kernel's launch registers cover its warpgroup split
-bool g_pp_ok64[64] = {};  // the same for its head-dim-64 form
+bool g_pp_ok64[64] = {};  // the same for its head-dim-64 forms
 
-// Makespan of n2 two-tile CTAs (cost kPairCost each, in units of one one-tile CTA over the
-// same keys) followed by n1 one-tile CTAs, placed in launch order on the first free SM.
-constexpr double kPairCost = 1.35;  // measured: 1.20 - 1.39 over 12,000 - 44,999 positions
-constexpr int kMinSplitTiles = 16;  // query tiles per clip below which no split is tried
+template <int HD, bool SPLIT>
+bool pp_attr() {
+  return cudaFuncSetAttribute(attention_pp_kernel<HD, SPLIT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              static_cast<int>(PPLayout<HD>::kSmem)) == cudaSuccess;
+}
+// Adds 1 to `ok_count` when this form's launch registers cover its warpgroup split; false
+// if the attributes cannot be read.
+template <int HD, bool SPLIT>
+bool pp_regs_ok(int& ok_count) {
+  cudaFuncAttributes fa{};
+  if (cudaFuncGetAttributes(&fa, attention_pp_kernel<HD, SPLIT>) != cudaSuccess) return false;
+  ok_count += fa.numRegs * kThreadsPP >= kRegsNeededPP && fa.numRegs <= 168;
+  return true;
+}
 
-double makespan(uint64_t n2, uint64_t n1, int sms) {
+// Makespan, in units of one one-tile CTA over the same keys, of the launch the library
+// makes: for every (clip, head) in launch order, P two-tile CTAs (cost kPairCost each) and
+// then its R = n_qt - 2P split-mode CTAs (kSplitCost), each placed on the first free SM;
+// with P = -1, n_qt one-tile CTAs per (clip, head).
+constexpr double kPairCost = 1.35;   // measured: 1.20 - 1.39 over 12,000 - 44,999 positions
+constexpr double kSplitCost = 0.75;  // half a pair's key walk plus the merge
+constexpr int kMinSplitTiles = 16;   // query tiles per clip below which only none / all are tried
+
+double makespan(int n_qt, int P, uint64_t bh, int sms) {
   std::priority_queue<double, std::vector<double>, std::greater<double>> free_at;
   for (int i = 0; i < sms; ++i) free_at.push(0.0);
   double end = 0.0;
-  auto place = [&](uint64_t n, double cost) {
-    for (uint64_t i = 0; i < n; ++i) {
+  auto place = [&](int n, double cost) {
+    for (int i = 0; i < n; ++i) {
       const double t = free_at.top() + cost;
       free_at.pop();
       free_at.push(t);
       end = t > end ? t : end;
     }
   };
-  place(n2, kPairCost);
-  place(n1, 1.0);
+  const int R = n_qt - 2 * P > 0 ? n_qt - 2 * P : 0;
+  for (uint64_t c = 0; c < bh; ++c) {
+    if (P < 0) {
+      place(n_qt, 1.0);
+    } else {
+      place(P, kPairCost);
+      place(R, kSplitCost);
+    }
+  }
   return end;
 }
 
-// Pairs per (clip, head) for the two-tile kernel: 0 (one-tile only), all of them, or the
-// largest count whose CTAs fill whole waves, whichever schedules shortest. Cached per shape.
+// Pairs per (clip, head) for the two-tile kernel, the rest of the tiles in split mode, or
+// -1 for the one-tile kernel: whichever of one-tile only, all pairs and (from
+// kMinSplitTiles query tiles up) no pairs or the largest count of pairs filling whole waves
+// schedules shortest. Cached per shape.
 int choose_pairs(int n_qt, uint64_t bh, int sms) {
   static std::mutex mu;
   static std::map<std::tuple<int, uint64_t, int>, int> cache;
@@ -833,19 +991,20 @@ int choose_pairs(int n_qt, uint64_t bh, int sms) {
     if (it != cache.end()) return it->second;
   }
   const int all = (n_qt + 1) / 2;
-  int best = 0;
-  double best_t = makespan(0, static_cast<uint64_t>(n_qt) * bh, sms);
+  int best = -1;
+  double best_t = makespan(n_qt, -1, bh, sms);
   std::vector<int> cands{all};
-  // Splitting only pays where every CTA walks many key tiles: the cost ratio was measured
-  // on 24 - 94 tiles, and at 6 tiles (16 clips of 60 s) a split ran 11 % slower than all
-  // pairs. Shorter clips choose between none and all.
-  if (n_qt >= kMinSplitTiles)
+  // The cost ratios were measured on 24 - 352 key tiles per CTA; on shorter clips (6 tiles
+  // for 16 clips of 60 s) a mix ran slower than all pairs, so they choose between one-tile
+  // and all pairs.
+  if (n_qt >= kMinSplitTiles) {
+    cands.push_back(0);
     for (uint64_t w = 1; w * sms <= static_cast<uint64_t>(all) * bh; ++w)
       cands.push_back(static_cast<int>(w * sms / bh));
+  }
   for (int P : cands) {
-    if (P <= 0 || static_cast<uint64_t>(P) * bh < 120) continue;  // too few CTAs to pair tiles
-    const int rest = n_qt - 2 * P > 0 ? n_qt - 2 * P : 0;
-    const double t = makespan(static_cast<uint64_t>(P) * bh, static_cast<uint64_t>(rest) * bh, sms);
+    if (P > 0 && static_cast<uint64_t>(P) * bh < 120) continue;  // too few CTAs to pair tiles
+    const double t = makespan(n_qt, P, bh, sms);
     if (t < best_t - 1e-9) {
       best_t = t;
       best = P;
@@ -872,20 +1031,17 @@ sal_status attention_launch_heads(const void* q, const void* k, const void* v, i
                                static_cast<int>(smem_one_tile(128))) != cudaSuccess ||
           cudaFuncSetAttribute(attention_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                static_cast<int>(smem_one_tile(64))) != cudaSuccess ||
-          cudaFuncSetAttribute(attention_pp_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               static_cast<int>(PPLayout<128>::kSmem)) != cudaSuccess ||
-          cudaFuncSetAttribute(attention_pp_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               static_cast<int>(PPLayout<64>::kSmem)) != cudaSuccess)
+          !pp_attr<128, false>() || !pp_attr<128, true>() || !pp_attr<64, false>() || !pp_attr<64, true>())
         return SAL_ECUDA;
       // setmaxnreg.inc waits until the registers it asks for are free: run the kernel only
       // if what warpgroup 0 gives back covers what the softmax warpgroups take (and the
       // launch count is one that 384 threads can get at all: at most 168)
-      cudaFuncAttributes fa{}, fa64{};
-      if (cudaFuncGetAttributes(&fa, attention_pp_kernel<128>) != cudaSuccess ||
-          cudaFuncGetAttributes(&fa64, attention_pp_kernel<64>) != cudaSuccess)
+      int r128 = 0, r64 = 0;
+      if (!pp_regs_ok<128, false>(r128) || !pp_regs_ok<128, true>(r128) || !pp_regs_ok<64, false>(r64) ||
+          !pp_regs_ok<64, true>(r64))
         return SAL_ECUDA;
-      g_pp_ok[dev] = fa.numRegs * kThreadsPP >= kRegsNeededPP && fa.numRegs <= 168;
-      g_pp_ok64[dev] = fa64.numRegs * kThreadsPP >= kRegsNeededPP && fa64.numRegs <= 168;
+      g_pp_ok[dev] = r128 == 2;
+      g_pp_ok64[dev] = r64 == 2;
       g_attr[dev] = true;
     }
   }
@@ -912,28 +1068,33 @@ sal_status attention_launch_heads(const void* q, const void* k, const void* v, i
   }
   const dim3 grid1(static_cast<unsigned>((T + kTile - 1) / kTile), static_cast<unsigned>(bh));
   if (head_dim == 64) {
-    // the CTC adapter's heads: every query-tile pair to the two-tile kernel (the second
-    // tile of an odd count is empty), unless it is unavailable or switched off
+    // the CTC adapter's heads: every query-tile pair to the two-tile kernel and an odd last
+    // tile to a split-mode CTA of the same launch, unless it is unavailable or switched off
     bool pp64 = false;
     {
       std::lock_guard<std::mutex> lk(g_mu);
       pp64 = dev >= 0 && dev < 64 && g_pp_ok64[dev];
     }
     if (pp64 && attention_pp_mode() != 0) {
-      const dim3 grid(static_cast<unsigned>((T + 2 * kTile - 1) / (2 * kTile)), static_cast<unsigned>(bh));
-      return launch_kernel(attention_pp_kernel<64>, grid, dim3(kThreadsPP), PPLayout<64>::kSmem, s, tq, tk, tv,
-                           a) == cudaSuccess
-                 ? SAL_OK
-                 : SAL_ECUDA;
+      const int n_qt = static_cast<int>((T + kTile - 1) / kTile);
+      a.pairs = n_qt / 2;
+      const dim3 grid(static_cast<unsigned>(n_qt / 2 + n_qt % 2), static_cast<unsigned>(bh));
+      const cudaError_t e =
+          n_qt % 2 ? launch_kernel(attention_pp_kernel<64, true>, grid, dim3(kThreadsPP), PPLayout<64>::kSmem, s,
+                                   tq, tk, tv, a)
+                   : launch_kernel(attention_pp_kernel<64, false>, grid, dim3(kThreadsPP), PPLayout<64>::kSmem, s,
+                                   tq, tk, tv, a);
+      return e == cudaSuccess ? SAL_OK : SAL_ECUDA;
     }
     return launch_kernel(attention_kernel<64>, grid1, dim3(192), smem_one_tile(64), s, tq, tk, tv, a) ==
                    cudaSuccess
                ? SAL_OK
                : SAL_ECUDA;
   }
-  // Split the query tiles between the kernels: the two-tile kernel takes the first P pairs
-  // of every (clip, head), the one-tile kernel the rest, launched right behind it so its
-  // CTAs fill the SMs that two-tile CTAs leave. P is chosen by list scheduling (below).
+  // The two-tile kernel takes the first P query-tile pairs of every (clip, head) and the
+  // remaining tiles one CTA each in split mode (the keys split between its warpgroups),
+  // all in one launch; with P = 0 the one-tile kernel takes every tile. P is chosen by
+  // list scheduling (choose_pairs).
   int sms = 148;
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const int n_qt = static_cast<int>((T + kTile - 1) / kTile);
@@ -943,27 +1104,29 @@ sal_status attention_launch_heads(const void* q, const void* k, const void* v, i
     pp_ok = dev >= 0 && dev < 64 && g_pp_ok[dev];
   }
   const int mode = attention_pp_mode();
-  int P = 0;  // query-tile pairs per (clip, head) for the two-tile kernel
+  int P = -1;  // query-tile pairs per (clip, head) for the two-tile kernel; -1: the one-tile kernel
   if (hold) {
     if (hold->kernel == 2 && !pp_ok) return SAL_EDEVICE;
-    P = hold->kernel == 2 ? (n_qt + 1) / 2 : 0;
+    P = hold->kernel == 2 ? (n_qt + 1) / 2 : -1;
   } else if (pp_ok && mode == 1) {
     P = (n_qt + 1) / 2;
   } else if (pp_ok && mode != 0) {
     P = choose_pairs(n_qt, bh, sms);
   }
-  const int pp_tiles = 2 * P < n_qt ? 2 * P : n_qt;
-  if (P > 0) {
-    const dim3 grid(static_cast<unsigned>(P), static_cast<unsigned>(bh));
-    if (launch_kernel(attention_pp_kernel<128>, grid, dim3(kThreadsPP), PPLayout<128>::kSmem, s, tq, tk, tv, a) !=
-        cudaSuccess)
-      return SAL_ECUDA;
+  const int forced = hold || !pp_ok ? -1 : attention_pairs_forced();
+  if (forced >= 0) P = forced < (n_qt + 1) / 2 ? forced : (n_qt + 1) / 2;
+  if (P >= 0) {
+    const int rest = n_qt - 2 * P > 0 ? n_qt - 2 * P : 0;
+    a.pairs = P;
+    const dim3 grid(static_cast<unsigned>(P + rest), static_cast<unsigned>(bh));
+    const cudaError_t e =
+        rest > 0 ? launch_kernel(attention_pp_kernel<128, true>, grid, dim3(kThreadsPP), PPLayout<128>::kSmem, s,
+                                 tq, tk, tv, a)
+                 : launch_kernel(attention_pp_kernel<128, false>, grid, dim3(kThreadsPP), PPLayout<128>::kSmem, s,
+                                 tq, tk, tv, a);
+    return e == cudaSuccess ? SAL_OK : SAL_ECUDA;
   }
-  if (pp_tiles == n_qt) return SAL_OK;
-  a.qt0 = pp_tiles;
-  a.tail = P > 0 ? 1 : 0;
-  const dim3 grid_rest(static_cast<unsigned>(n_qt - pp_tiles), static_cast<unsigned>(bh));
-  return launch_kernel(attention_kernel<128>, grid_rest, dim3(192), smem_one_tile(128), s, tq, tk, tv, a) ==
+  return launch_kernel(attention_kernel<128>, grid1, dim3(192), smem_one_tile(128), s, tq, tk, tv, a) ==
                  cudaSuccess
              ? SAL_OK
              : SAL_ECUDA;
@@ -1010,10 +1173,13 @@ extern "C" sal_status sal_attention_plan(int batch, int64_t T, int heads, int he
   if ((head_dim != 128 && head_dim != 64) || batch == 0 || T == 0 || heads == 0) return SAL_OK;
   const uint64_t bh = static_cast<uint64_t>(batch) * heads;
   const int mode = attention_pp_mode();
-  if (head_dim == 64) {  // every pair to the two-tile kernel unless it is switched off
-    *pairs = mode == 0 ? 0 : (n_qt + 1) / 2;
+  if (head_dim == 64) {  // every pair to the two-tile kernel, an odd last tile split
+    *pairs = mode == 0 ? 0 : n_qt / 2;
     return SAL_OK;
   }
-  *pairs = mode == 0 ? 0 : (mode == 1 ? (n_qt + 1) / 2 : choose_pairs(n_qt, bh, sms));
+  int P = mode == 0 ? -1 : (mode == 1 ? (n_qt + 1) / 2 : choose_pairs(n_qt, bh, sms));
+  const int forced = attention_pairs_forced();
+  if (forced >= 0) P = forced < (n_qt + 1) / 2 ? forced : (n_qt + 1) / 2;
+  *pairs = P > 0 ? P : 0;
   return SAL_OK;
 }

@@ -112,14 +112,14 @@ def test_attention_plan_matches_the_stated_schedule(api):
 
     SAL_ATTN_PP in the environment forces the split (the library reads it once per
     process), so the stated rule is only checked when it is unset."""
-    if os.environ.get("SAL_ATTN_PP"):
-        pytest.skip("SAL_ATTN_PP forces the split in this process")
+    if os.environ.get("SAL_ATTN_PP") or os.environ.get("SAL_ATTN_PAIRS"):
+        pytest.skip("SAL_ATTN_PP / SAL_ATTN_PAIRS force the split in this process")
     from test_gpu_kernels import _pairs_for_two_tile_kernel
     cases = [(b, T) for b in (1, 2, 8, 16, 30) for T in (1, 129, 749, 1000, 2000, 2047, 2048, 3000)]
     cases += [(b, T) for b in (1, 2) for T in (5000, 7499, 12000, 20000, 44999)]
     for batch, T in cases:
         assert api.attention_plan(batch, T) == _pairs_for_two_tile_kernel(batch, T), (batch, T)
-    assert api.attention_plan(1, 20000, heads=16, head_dim=64) == (79, 157)  # 64-wide heads: all pairs
+    assert api.attention_plan(1, 20000, heads=16, head_dim=64) == (78, 157)  # 64-wide heads: pairs + 1 split
     assert api.attention_plan(0, 100) == (0, 1)
     p, q = ctypes.c_int(), ctypes.c_int()
     assert api.lib().sal_attention_plan(1, 90001, 10, 128, 148, ctypes.byref(p), ctypes.byref(q)) == 2

@@ -125,49 +125,55 @@ def test_qkv_rope(batch, T):
 
 # ---------------------------------------------------------------- attention
 
-def _pairs_for_two_tile_kernel(batch, T, sms=148, rho=1.35):
+def _pairs_for_two_tile_kernel(batch, T, sms=148, rho=1.35, sigma=0.75):
     """Query-tile pairs per (clip, head) that the library gives the two-tile kernel (the
-    rest go to the one-tile kernel launched behind it): the count, among none, all, or the
-    largest filling whole waves, whose greedy schedule (a two-tile CTA costing rho one-tile
-    CTAs) ends first; at least 120 two-tile CTAs."""
+    remaining tiles go to split-mode CTAs of the same launch), 0 also when the one-tile
+    kernel takes every tile: the choice among one-tile only, all pairs and (from 16 query
+    tiles up) no pairs or the largest count of pairs filling whole waves whose greedy
+    schedule ends first; at least 120 two-tile CTAs when there are pairs. The schedule
+    places, for every (clip, head) in launch order, its pairs (rho one-tile CTAs each) and
+    then its split tiles (sigma each); one-tile CTAs cost 1."""
     import heapq
 
-    def makespan(n2, n1):
+    bh, n_qt = 10 * batch, -(-T // 128)
+
+    def makespan(P):
         h = [0.0] * sms
         end = 0.0
-        for n, c in ((n2, rho), (n1, 1.0)):
-            for _ in range(n):
-                t = heapq.heappop(h) + c
-                heapq.heappush(h, t)
-                end = max(end, t)
+        jobs = [(n_qt, 1.0)] if P < 0 else [(P, rho), (max(n_qt - 2 * P, 0), sigma)]
+        for _ in range(bh):
+            for n, c in jobs:
+                for _ in range(n):
+                    t = heapq.heappop(h) + c
+                    heapq.heappush(h, t)
+                    end = max(end, t)
         return end
 
-    bh, n_qt = 10 * batch, -(-T // 128)
     everything = (n_qt + 1) // 2
     cands = [everything]
-    if n_qt >= 16:  # shorter clips: none or all pairs
-        cands += [w * sms // bh for w in range(1, everything * bh // sms + 1)]
-    best, best_t = 0, makespan(0, n_qt * bh)
+    if n_qt >= 16:  # shorter clips: one-tile or all pairs
+        cands += [0] + [w * sms // bh for w in range(1, everything * bh // sms + 1)]
+    best, best_t = -1, makespan(-1)
     for P in cands:
-        if P <= 0 or P * bh < 120:
+        if P > 0 and P * bh < 120:
             continue
-        t = makespan(P * bh, max(n_qt - 2 * P, 0) * bh)
+        t = makespan(P)
         if t < best_t - 1e-9:
             best, best_t = P, t
-    return best, n_qt
+    return max(best, 0), n_qt
 
 
 # The first eight cases run the one-tile kernel only; (30, 129), (8, 1000), (1, 3000) and
-# (16, 749) the two-tile kernel only; (1, 5000) splits the query tiles between the two
+# (16, 749) the two-tile kernel only; (1, 4000) gives it 14 pairs and 4 split-mode tiles
 # (checked below). T = 129: a second query tile with one valid row and a last key tile
 # with one valid column.
 @pytest.mark.parametrize("batch,T,scale", [(1, 1, 1.0), (2, 7, 1.0), (1, 128, 1.0), (1, 129, 1.0),
                                            (2, 383, 1.0), (1, 749, 1.0), (1, 749, 8.0), (1, 2000, 3.0),
                                            (30, 129, 1.0), (8, 1000, 1.0), (1, 3000, 8.0), (16, 749, 1.0),
-                                           (1, 5000, 2.0)])
+                                           (1, 4000, 2.0)])
 def test_attention(batch, T, scale):
     api = _api()
-    expect = {(30, 129): (1, 2), (1, 3000): (12, 24), (8, 1000): (4, 8), (16, 749): (3, 6), (1, 5000): (14, 40)}
+    expect = {(30, 129): (1, 2), (1, 3000): (12, 24), (8, 1000): (4, 8), (16, 749): (3, 6), (1, 4000): (14, 32)}
     n_qt = -(-T // 128)
     assert api.attention_plan(batch, T) == expect.get((batch, T), (0, n_qt))
     q, q64 = rand_bf16((batch, 10, T, 128), 50 + T, scale)
@@ -175,10 +181,9 @@ def test_attention(batch, T, scale):
     v, v64 = rand_bf16((batch, 10, T, 128), 70 + T, 1.0)
     n0 = api.sal_launch_count()
     o = api.sal_attention(q, k, v)
-    # the launches match the plan: the two-tile kernel and, when it leaves query tiles
-    # over, the one-tile kernel behind it
-    P = expect.get((batch, T), (0, n_qt))[0]
-    assert api.sal_launch_count() - n0 == (2 if 0 < P and 2 * P < n_qt else 1)
+    # one launch: the two-tile kernel (its pairs, then any split-mode tiles) or, with no
+    # pairs, the one-tile kernel
+    assert api.sal_launch_count() - n0 == 1
     got = to64(o).reshape(batch, T, 10, 128)
     for b in range(batch):
         ref = O.attention(q64[b], k64[b], v64[b]).transpose(1, 0, 2)
