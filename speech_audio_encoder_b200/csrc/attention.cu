@@ -947,11 +947,14 @@ bool pp_regs_ok(int& ok_count) {
 
 // Makespan, in units of one one-tile CTA over the same keys, of the launch the library
 // makes: for every (clip, head) in launch order, P two-tile CTAs (cost kPairCost each) and
-// then its R = n_qt - 2P split-mode CTAs (kSplitCost), each placed on the first free SM;
+// then its R = n_qt - 2P split-mode CTAs (split_cost), each placed on the first free SM;
 // with P = -1, n_qt one-tile CTAs per (clip, head).
-constexpr double kPairCost = 1.35;   // measured: 1.20 - 1.39 over 12,000 - 44,999 positions
-constexpr double kSplitCost = 0.75;  // half a pair's key walk plus the merge
-constexpr int kMinSplitTiles = 16;   // query tiles per clip below which only none / all are tried
+constexpr double kPairCost = 1.35;  // measured: 1.20 - 1.39 over 12,000 - 44,999 positions
+constexpr int kMinSplitTiles = 16;  // query tiles per clip below which no mix is tried
+// A split CTA walks half of a pair's keys, plus a fixed part (its start and the merge) that
+// weighs more on short clips: fitted to 0.757 at 59 query tiles (7,499 positions, every
+// tile split against all pairs) and 0.92 at 6 (16 clips of 749).
+double split_cost(int n_qt) { return 0.74 + 1.09 / (n_qt > 0 ? n_qt : 1); }
 
 double makespan(int n_qt, int P, uint64_t bh, int sms) {
   std::priority_queue<double, std::vector<double>, std::greater<double>> free_at;
@@ -971,16 +974,16 @@ double makespan(int n_qt, int P, uint64_t bh, int sms) {
       place(n_qt, 1.0);
     } else {
       place(P, kPairCost);
-      place(R, kSplitCost);
+      place(R, split_cost(n_qt));
     }
   }
   return end;
 }
 
 // Pairs per (clip, head) for the two-tile kernel, the rest of the tiles in split mode, or
-// -1 for the one-tile kernel: whichever of one-tile only, all pairs and (from
-// kMinSplitTiles query tiles up) no pairs or the largest count of pairs filling whole waves
-// schedules shortest. Cached per shape.
+// -1 for the one-tile kernel: whichever of one-tile only, all pairs, no pairs (every tile
+// split) and (from kMinSplitTiles query tiles up) the largest counts of pairs filling
+// whole waves schedules shortest. Cached per shape.
 int choose_pairs(int n_qt, uint64_t bh, int sms) {
   static std::mutex mu;
   static std::map<std::tuple<int, uint64_t, int>, int> cache;
@@ -993,15 +996,12 @@ int choose_pairs(int n_qt, uint64_t bh, int sms) {
   const int all = (n_qt + 1) / 2;
   int best = -1;
   double best_t = makespan(n_qt, -1, bh, sms);
-  std::vector<int> cands{all};
-  // The cost ratios were measured on 24 - 352 key tiles per CTA; on shorter clips (6 tiles
-  // for 16 clips of 60 s) a mix ran slower than all pairs, so they choose between one-tile
-  // and all pairs.
-  if (n_qt >= kMinSplitTiles) {
-    cands.push_back(0);
+  std::vector<int> cands{all, 0};
+  // The pair cost was measured on 24 - 352 key tiles per CTA; on shorter clips (6 tiles
+  // for 16 clips of 60 s) a mix of pairs and one-tile CTAs ran slower than all pairs.
+  if (n_qt >= kMinSplitTiles)
     for (uint64_t w = 1; w * sms <= static_cast<uint64_t>(all) * bh; ++w)
       cands.push_back(static_cast<int>(w * sms / bh));
-  }
   for (int P : cands) {
     if (P > 0 && static_cast<uint64_t>(P) * bh < 120) continue;  // too few CTAs to pair tiles
     const double t = makespan(n_qt, P, bh, sms);

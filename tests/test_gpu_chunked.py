@@ -23,9 +23,9 @@ def _api():
 
 # (batch, T, chunk): chunk = 1 (a chunk per position), chunks not aligned to 128-row tiles,
 # chunks aligned to tiles, the 30-second chunk of 375 positions; (8, 1000) and (1, 3000) run
-# the two-tile kernel in pairs, (1, 4000) in 14 pairs and 4 split-mode tiles (the
-# warpgroups of a split tile take alternate key tiles of its chunks, with masked borders),
-# the others the one-tile kernel.
+# the two-tile kernel in pairs, (1, 4000) in 14 pairs and 4 split-mode tiles, (1, 749) with
+# every tile in split mode (the warpgroups of a split tile take alternate key tiles of its
+# chunks, with masked borders), the others the one-tile kernel.
 @pytest.mark.parametrize("batch,T,chunk", [(1, 129, 1), (2, 383, 100), (1, 749, 128), (1, 749, 375),
                                            (8, 1000, 375), (1, 3000, 375), (1, 4000, 375), (1, 4000, 1000)])
 def test_attention_chunked(batch, T, chunk):

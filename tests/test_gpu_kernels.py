@@ -125,17 +125,18 @@ def test_qkv_rope(batch, T):
 
 # ---------------------------------------------------------------- attention
 
-def _pairs_for_two_tile_kernel(batch, T, sms=148, rho=1.35, sigma=0.75):
+def _pairs_for_two_tile_kernel(batch, T, sms=148, rho=1.35):
     """Query-tile pairs per (clip, head) that the library gives the two-tile kernel (the
     remaining tiles go to split-mode CTAs of the same launch), 0 also when the one-tile
-    kernel takes every tile: the choice among one-tile only, all pairs and (from 16 query
-    tiles up) no pairs or the largest count of pairs filling whole waves whose greedy
+    kernel takes every tile: the choice among one-tile only, all pairs, no pairs and (from
+    16 query tiles up) the largest counts of pairs filling whole waves whose greedy
     schedule ends first; at least 120 two-tile CTAs when there are pairs. The schedule
     places, for every (clip, head) in launch order, its pairs (rho one-tile CTAs each) and
-    then its split tiles (sigma each); one-tile CTAs cost 1."""
+    then its split tiles (0.74 + 1.09 / query tiles each); one-tile CTAs cost 1."""
     import heapq
 
     bh, n_qt = 10 * batch, -(-T // 128)
+    sigma = 0.74 + 1.09 / n_qt
 
     def makespan(P):
         h = [0.0] * sms
@@ -150,9 +151,9 @@ def _pairs_for_two_tile_kernel(batch, T, sms=148, rho=1.35, sigma=0.75):
         return end
 
     everything = (n_qt + 1) // 2
-    cands = [everything]
-    if n_qt >= 16:  # shorter clips: one-tile or all pairs
-        cands += [0] + [w * sms // bh for w in range(1, everything * bh // sms + 1)]
+    cands = [everything, 0]
+    if n_qt >= 16:  # shorter clips: one-tile, all pairs or every tile split
+        cands += [w * sms // bh for w in range(1, everything * bh // sms + 1)]
     best, best_t = -1, makespan(-1)
     for P in cands:
         if P > 0 and P * bh < 120:
@@ -163,10 +164,11 @@ def _pairs_for_two_tile_kernel(batch, T, sms=148, rho=1.35, sigma=0.75):
     return max(best, 0), n_qt
 
 
-# The first eight cases run the one-tile kernel only; (30, 129), (8, 1000), (1, 3000) and
-# (16, 749) the two-tile kernel only; (1, 4000) gives it 14 pairs and 4 split-mode tiles
-# (checked below). T = 129: a second query tile with one valid row and a last key tile
-# with one valid column.
+# The first five cases run the one-tile kernel; (1, 749) and (1, 2000) the two-tile kernel
+# with every query tile in split mode (the keys split between its warpgroups); (30, 129),
+# (8, 1000), (1, 3000) and (16, 749) the two-tile kernel in pairs only; (1, 4000) 14 pairs
+# and 4 split-mode tiles. T = 129: a second query tile with one valid row and a last key
+# tile with one valid column.
 @pytest.mark.parametrize("batch,T,scale", [(1, 1, 1.0), (2, 7, 1.0), (1, 128, 1.0), (1, 129, 1.0),
                                            (2, 383, 1.0), (1, 749, 1.0), (1, 749, 8.0), (1, 2000, 3.0),
                                            (30, 129, 1.0), (8, 1000, 1.0), (1, 3000, 8.0), (16, 749, 1.0),
