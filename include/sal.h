@@ -33,8 +33,10 @@
  *   - bf16 tensors are IEEE bfloat16 bit patterns (uint16_t); parameters are bf16.
  *   - T > 45000 (more than one hour of audio per clip) is SAL_ESHAPE; N < 400 samples
  *     or T = 0 is a valid empty problem that launches nothing and returns SAL_OK.
- *   - The library allocates no device memory. Scratch space is the caller's
- *     `workspace`; sal_encoder_workspace_bytes() gives its size.
+ *   - The library allocates no device memory (the bounds-checked build excepted: a few
+ *     hundred bytes per device for its report). Scratch space is the caller's
+ *     `workspace`; sal_encoder_workspace_bytes() gives its size. sal_weights_file_load
+ *     allocates pinned host memory for its staging buffers while it runs.
  *   - Thread safety: calls on different streams may run concurrently.
  */
 #ifndef SAL_H_
@@ -54,7 +56,8 @@ typedef enum {
     SAL_EWORKSPACE = 3, /* workspace smaller than sal_encoder_workspace_bytes() */
     SAL_ECUDA = 4,      /* a CUDA runtime call or kernel launch failed */
     SAL_ETIMEOUT = 5,   /* a bounded device wait gave up (see sal_last_device_status) */
-    SAL_EDEVICE = 6     /* the current device is not a B200-class sm_100 GPU */
+    SAL_EDEVICE = 6,    /* the current device is not a B200-class sm_100 GPU */
+    SAL_EIO = 7         /* a file could not be opened or read */
 } sal_status;
 
 #define SAL_N_MELS 128
@@ -101,6 +104,40 @@ typedef struct {
     int n_layers;
     const void *lnf_g, *lnf_b;
 } sal_weights;
+
+/* ---------------------------------------------------------------------------------
+ * Flat weight file: this library's own format for the encoder's parameters (the pages'
+ * models ship in a third-party container format, which is not read here). Little-endian:
+ *   bytes [0, 8)    magic "SALENCW1"
+ *         [8, 12)   version 1            [12, 16) header bytes 256
+ *         [16, 20)  dtype 1 (bf16)       [20, 24) width 1280
+ *         [24, 28)  heads 10             [28, 32) head dim 128
+ *         [32, 36)  FFN width 5120       [36, 40) stack width 1024
+ *         [40, 44)  n_layers             [44, 48) alignment 256
+ *         [48, 56)  data bytes D (uint64)
+ *         [56, 256) zero
+ *   then D bytes: every tensor as row-major bf16 starting on a 256-byte boundary (zero
+ *   padding), in the order w_proj [1280, 1024], b_proj, lnf_g, lnf_b [1280], then for
+ *   each layer ln1_g, ln1_b [1280], w_qkv [3840, 1280], b_qkv [3840], qn_g, kn_g [128],
+ *   w_o [1280, 1280], b_o, ln2_g, ln2_b [1280], w1 [5120, 1280], b1 [5120],
+ *   w2 [1280, 5120], b2 [1280]. The file is exactly 256 + D bytes long.
+ * --------------------------------------------------------------------------------- */
+
+/* Reads the header of the file at `path` (host only, no CUDA call): *n_layers and the
+ * device buffer size *device_bytes (= D). Errors: SAL_EINVAL (null argument; bad magic,
+ * version, dtype, alignment, reserved bytes, data size or file length), SAL_ESHAPE (sizes
+ * other than this library's), SAL_EIO (cannot open or read); outputs 0 on error. */
+sal_status sal_weights_file_info(const char* path, int* n_layers, size_t* device_bytes);
+
+/* Loads the file into device_buffer (device memory, 256-byte aligned, >= D bytes: the
+ * tensors keep the file's layout) through pinned staging buffers on `stream`, and returns
+ * after the copies have completed. Fills layers[0 .. n_layers) (a host array of at least
+ * n_layers records, owned by the caller) and *w, whose pointers address device_buffer;
+ * w->layers = layers. Errors: as sal_weights_file_info, plus SAL_EINVAL (null buffer or
+ * record, misaligned buffer), SAL_EWORKSPACE (buffer_bytes < D or max_layers < n_layers),
+ * SAL_ECUDA; on error the contents of device_buffer are unspecified. */
+sal_status sal_weights_file_load(const char* path, void* device_buffer, size_t buffer_bytes,
+                                 sal_layer* layers, int max_layers, sal_weights* w, void* stream);
 
 /* Front end (page "Nemotron 3.5 Transcribe: From Recorded Speech to Dataset Audits",
  * section "How audio and speakers reach the language model", exported-frontend
@@ -223,6 +260,35 @@ sal_status sal_last_device_status(void* stream);
  * down: each CTA waits for its own TMA loads and MMAs still in flight, with a fixed bound
  * of 4 s that this limit does not shorten, then frees its tensor memory and returns. */
 void sal_set_wait_limit_ns(uint64_t ns);
+
+/* ---------------------------------------------------------------------------------
+ * Bounds-checked build. libsal_checked.so is this library compiled with SAL_CHECKED:
+ * the same entry points, in which every plain global load and store of every kernel is
+ * tested against the byte ranges of the buffers that launch was given (inputs read-only,
+ * outputs and workspace writable). An access outside them is not made: it is counted,
+ * the lowest such address is kept with the file and line of the access, and the kernel
+ * carries on (its outputs are then unspecified). TMA copies are clipped by the hardware
+ * to their tensor maps and are not counted. The checked build serialises every launch
+ * behind a small host-to-device copy, must be driven from one host thread and one stream
+ * at a time, and cannot be captured into a CUDA graph. Both libraries export these calls.
+ * --------------------------------------------------------------------------------- */
+
+/* 1 in libsal_checked.so, 0 in libsal.so. */
+int sal_checked_build(void);
+
+/* Synchronises the current device and reports, then clears, the accesses the checked
+ * build refused on it since the last report: their count, the lowest address, the source
+ * file of that access (1 frontend.cu, 2 rowops.cu, 3 gemm.cu, 4 attention.cu, 5 ctc.cu)
+ * and line, and the smallest sal_launch_count value before a launch that made one. All
+ * outputs are 0 when count is 0. SAL_EINVAL (outputs 0) from libsal.so or on a null
+ * pointer; SAL_ECUDA if the device cannot be reached. */
+sal_status sal_check_report(uint64_t* count, uint64_t* first_address, int* file, int* line,
+                            uint64_t* first_launch);
+
+/* Test hook of the checked build (no effect in libsal.so): every writable range declared
+ * from now on is taken `bytes` shorter at its end (0 restores the exact ranges), so the
+ * stores a kernel makes there are refused and reported instead of made. */
+void sal_check_shrink_writable(uint64_t bytes);
 
 /* ---------------------------------------------------------------------------------
  * Single-step entry points (the stages sal_encoder_forward chains; for tests and

@@ -7,6 +7,7 @@ device is not an sm_100 GPU, the calls raise.
 """
 from __future__ import annotations
 
+import contextlib
 import ctypes
 import os
 
@@ -15,6 +16,9 @@ import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libsal.so")
+# The bounds-checked build (sal.h, "Bounds-checked build"): same calls, every kernel's
+# plain global accesses tested against the buffers it was given.
+LIB_CHECKED_PATH = os.path.join(_HERE, "libsal_checked.so")
 
 N_MELS, STACK, STACK_DIM, WIDTH, HEADS, HEAD_DIM, FFN = 128, 8, 1024, 1280, 10, 128, 5120
 MAX_POSITIONS = 45000
@@ -88,6 +92,16 @@ EXPORTS = {
                                    ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_size_t,
                                    ctypes.c_void_p]),
     "sal_last_device_status": (ctypes.c_int, [ctypes.c_void_p]),
+    "sal_weights_file_info": (ctypes.c_int, [ctypes.c_char_p, ctypes.POINTER(ctypes.c_int),
+                                              ctypes.POINTER(ctypes.c_size_t)]),
+    "sal_weights_file_load": (ctypes.c_int, [ctypes.c_char_p, ctypes.c_void_p, ctypes.c_size_t,
+                                              ctypes.POINTER(sal_layer), ctypes.c_int, ctypes.POINTER(sal_weights),
+                                              ctypes.c_void_p]),
+    "sal_checked_build": (ctypes.c_int, []),
+    "sal_check_report": (ctypes.c_int, [ctypes.POINTER(ctypes.c_uint64), ctypes.POINTER(ctypes.c_uint64),
+                                         ctypes.POINTER(ctypes.c_int), ctypes.POINTER(ctypes.c_int),
+                                         ctypes.POINTER(ctypes.c_uint64)]),
+    "sal_check_shrink_writable": (None, [ctypes.c_uint64]),
     "sal_set_wait_limit_ns": (None, [ctypes.c_uint64]),
     "sal_layernorm": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int64, ctypes.c_void_p, ctypes.c_void_p,
                                       ctypes.c_void_p, ctypes.c_void_p]),
@@ -123,22 +137,39 @@ EXPORTS = {
                                         ctypes.c_size_t, ctypes.c_void_p]),
 }
 
-_lib = None
+_libs: dict = {}
+# SAL_LIB=checked routes every call of this module through the bounds-checked build.
+_active = LIB_CHECKED_PATH if os.environ.get("SAL_LIB") == "checked" else LIB_PATH
 
 
-def lib() -> ctypes.CDLL:
-    """The loaded libsal.so. Raises if it has not been built."""
-    global _lib
-    if _lib is None:
-        if not os.path.exists(LIB_PATH):
-            raise RuntimeError(f"{LIB_PATH} is missing: run `python -m speech_audio_encoder_b200.build`")
-        l = ctypes.CDLL(LIB_PATH)
+def _load(path: str) -> ctypes.CDLL:
+    if path not in _libs:
+        if not os.path.exists(path):
+            raise RuntimeError(f"{path} is missing: run `python -m speech_audio_encoder_b200.build`")
+        l = ctypes.CDLL(path)
         for name, (res, args) in EXPORTS.items():
             f = getattr(l, name)
             f.restype = res
             f.argtypes = args
-        _lib = l
-    return _lib
+        _libs[path] = l
+    return _libs[path]
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded library (libsal.so, or libsal_checked.so inside `checked_library()` or
+    with SAL_LIB=checked). Raises if it has not been built."""
+    return _load(_active)
+
+
+@contextlib.contextmanager
+def checked_library():
+    """Calls made inside this block go through libsal_checked.so."""
+    global _active
+    prev, _active = _active, LIB_CHECKED_PATH
+    try:
+        yield lib()
+    finally:
+        _active = prev
 
 
 def status_string(status: int) -> str:
@@ -213,6 +244,26 @@ class DeviceWeights:
         self.record = sal_weights(self.ptr[(None, "w_proj")], self.ptr[(None, "b_proj")],
                                   self._layers, self.n_layers, self.ptr[(None, "lnf_g")],
                                   self.ptr[(None, "lnf_b")])
+
+    @classmethod
+    def from_file(cls, path: str, device="cuda", stream=None) -> "DeviceWeights":
+        """Loads a flat weight file (sal_weights_file_load) into one device buffer."""
+        n_layers, nbytes = ctypes.c_int(), ctypes.c_size_t()
+        _check("sal_weights_file_info", lib().sal_weights_file_info(os.fsencode(path), ctypes.byref(n_layers),
+                                                                    ctypes.byref(nbytes)))
+        self = cls.__new__(cls)
+        self.buffer = torch.empty(nbytes.value, dtype=torch.uint8, device=device)
+        self.n_layers = n_layers.value
+        self._layers = (sal_layer * max(self.n_layers, 1))()
+        self.record = sal_weights()
+        _check("sal_weights_file_load",
+               lib().sal_weights_file_load(os.fsencode(path), self.buffer.data_ptr(), nbytes.value, self._layers,
+                                           self.n_layers, ctypes.byref(self.record), _stream(stream)))
+        self.ptr = {(None, k): getattr(self.record, k) for k in ("w_proj", "b_proj", "lnf_g", "lnf_b")}
+        for i in range(self.n_layers):
+            for k in LAYER_FIELDS:
+                self.ptr[(i, k)] = getattr(self._layers[i], k)
+        return self
 
     def layer(self, i: int) -> sal_layer:
         return self._layers[i]
@@ -451,6 +502,24 @@ def sal_last_device_status(stream=None) -> int:
 
 def sal_set_wait_limit_ns(ns: int) -> None:
     lib().sal_set_wait_limit_ns(int(ns))
+
+
+FILE_IDS = {1: "frontend.cu", 2: "rowops.cu", 3: "gemm.cu", 4: "attention.cu", 5: "ctc.cu"}
+
+
+def check_report() -> dict:
+    """Reads and clears the checked build's record of refused accesses (sal_check_report)."""
+    count, addr, seq = ctypes.c_uint64(), ctypes.c_uint64(), ctypes.c_uint64()
+    f, ln = ctypes.c_int(), ctypes.c_int()
+    _check("sal_check_report", lib().sal_check_report(ctypes.byref(count), ctypes.byref(addr), ctypes.byref(f),
+                                                       ctypes.byref(ln), ctypes.byref(seq)))
+    return {"count": count.value, "first_address": addr.value, "file": FILE_IDS.get(f.value, f.value),
+            "line": ln.value, "first_launch": seq.value}
+
+
+def check_shrink_writable(nbytes: int) -> None:
+    """Test hook of the checked build: writable ranges declared from now on end nbytes early."""
+    lib().sal_check_shrink_writable(int(nbytes))
 
 
 CTC_CLASSES = 23863

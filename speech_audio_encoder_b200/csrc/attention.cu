@@ -16,6 +16,7 @@
 //     the stale maximum keeps every p <= 256, exact in fp32 and bf16 range);
 //   * S_{j+1} is computed while the softmax of S_j runs.
 // TMEM columns: S0 [0,128), S1 [128,256), O [256,384), P0 [384,448), P1 [448,512).
+#define SAL_CK_FILE 4
 #include <cuda_bf16.h>
 #include <math.h>
 
@@ -389,7 +390,7 @@ __global__ void __launch_bounds__(192, 1)
             u.y = pack_bf16x2(__uint_as_float(o[8 * i + 2]) * inv_l, __uint_as_float(o[8 * i + 3]) * inv_l);
             u.z = pack_bf16x2(__uint_as_float(o[8 * i + 4]) * inv_l, __uint_as_float(o[8 * i + 5]) * inv_l);
             u.w = pack_bf16x2(__uint_as_float(o[8 * i + 6]) * inv_l, __uint_as_float(o[8 * i + 7]) * inv_l);
-            d4[i] = u;
+            *SAL_CK_ST(d4 + i, 16) = u;
           }
         }
       }
@@ -479,8 +480,8 @@ __device__ __forceinline__ void store_row32(__nv_bfloat16* dst, const uint32_t (
     float v[8];
 #pragma unroll
     for (int e = 0; e < 8; ++e) v[e] = fmaf(__uint_as_float(y[8 * i + e]), b, __uint_as_float(x[8 * i + e]) * a);
-    d4[i] = make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]), pack_bf16x2(v[4], v[5]),
-                       pack_bf16x2(v[6], v[7]));
+    *SAL_CK_ST(d4 + i, 16) = make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]),
+                                        pack_bf16x2(v[4], v[5]), pack_bf16x2(v[6], v[7]));
   }
 }
 
@@ -1067,6 +1068,11 @@ sal_status attention_launch_heads(const void* q, const void* k, const void* v, i
     a.win_total = win->total;
   }
   const dim3 grid1(static_cast<unsigned>((T + kTile - 1) / kTile), static_cast<unsigned>(bh));
+  const int64_t bytes = static_cast<int64_t>(bh) * T * head_dim * 2;  // each of q, k, v and o
+  ck_declare(q, bytes, false);
+  ck_declare(k, bytes, false);
+  ck_declare(v, bytes, false);
+  ck_declare(o, bytes, true);
   if (head_dim == 64) {
     // the CTC adapter's heads: every query-tile pair to the two-tile kernel and an odd last
     // tile to a split-mode CTA of the same launch, unless it is unavailable or switched off
@@ -1144,6 +1150,7 @@ sal_status attention_launch(const void* q, const void* k, const void* v, int bat
 extern "C" sal_status sal_attention_withhold(const void* q, const void* k, const void* v, int batch, int64_t T,
                                              int kernel, int tile, void* o, void* stream) {
   using namespace sal;
+  const NvtxRange nvtx_("sal_attention_withhold");
   if (batch < 0 || T < 0 || tile < 0 || (kernel != 1 && kernel != 2)) return SAL_EINVAL;
   if (T > SAL_MAX_POSITIONS) return SAL_ESHAPE;
   if (batch == 0 || T == 0) return SAL_OK;

@@ -15,6 +15,7 @@
 //   * log-softmax over the 23,863 classes of each 40 ms position: one CTA per row, an
 //     online maximum and sum of exponentials in one pass over the fp32 scores, then
 //     z - max - log(sum) written out.
+#define SAL_CK_FILE 5
 #include <cuda_bf16.h>
 #include <math.h>
 
@@ -45,31 +46,33 @@ __global__ void __launch_bounds__(256) ctc_qk_norm_rope_kernel(const float* __re
   pdl_trigger();
   if (row >= rows) return;
   const int64_t b = row / T, t = row - b * T;
-  const float c = cs[t * 64 + 2 * lane], s = cs[T * 64 + t * 64 + 2 * lane];
-  const float gq0 = __bfloat162float(qn_g[lane]), gq1 = __bfloat162float(qn_g[lane + 32]);
-  const float gk0 = __bfloat162float(kn_g[lane]), gk1 = __bfloat162float(kn_g[lane + 32]);
+  const float c = *SAL_CK_LD(cs + t * 64 + 2 * lane, 4), s = *SAL_CK_LD(cs + T * 64 + t * 64 + 2 * lane, 4);
+  const float gq0 = __bfloat162float(*SAL_CK_LD(qn_g + lane, 2));
+  const float gq1 = __bfloat162float(*SAL_CK_LD(qn_g + lane + 32, 2));
+  const float gk0 = __bfloat162float(*SAL_CK_LD(kn_g + lane, 2));
+  const float gk1 = __bfloat162float(*SAL_CK_LD(kn_g + lane + 32, 2));
   const float* src = qkv + row * (3 * kW);
 #pragma unroll 4
   for (int h = 0; h < kH; ++h) {
     const int64_t dst = ((b * kH + h) * T + t) * kHd;
     {  // q
-      float x0 = src[h * kHd + lane], x1 = src[h * kHd + 32 + lane];
+      float x0 = *SAL_CK_LD(src + h * kHd + lane, 4), x1 = *SAL_CK_LD(src + h * kHd + 32 + lane, 4);
       const float r = rsqrtf(warp_sum32(x0 * x0 + x1 * x1) * (1.0f / kHd) + 1e-6f);
       x0 *= r * gq0;
       x1 *= r * gq1;
-      q[dst + lane] = __float2bfloat16_rn(x0 * c - x1 * s);
-      q[dst + 32 + lane] = __float2bfloat16_rn(x1 * c + x0 * s);
+      *SAL_CK_ST(q + dst + lane, 2) = __float2bfloat16_rn(x0 * c - x1 * s);
+      *SAL_CK_ST(q + dst + 32 + lane, 2) = __float2bfloat16_rn(x1 * c + x0 * s);
     }
     {  // k
-      float x0 = src[kW + h * kHd + lane], x1 = src[kW + h * kHd + 32 + lane];
+      float x0 = *SAL_CK_LD(src + kW + h * kHd + lane, 4), x1 = *SAL_CK_LD(src + kW + h * kHd + 32 + lane, 4);
       const float r = rsqrtf(warp_sum32(x0 * x0 + x1 * x1) * (1.0f / kHd) + 1e-6f);
       x0 *= r * gk0;
       x1 *= r * gk1;
-      k[dst + lane] = __float2bfloat16_rn(x0 * c - x1 * s);
-      k[dst + 32 + lane] = __float2bfloat16_rn(x1 * c + x0 * s);
+      *SAL_CK_ST(k + dst + lane, 2) = __float2bfloat16_rn(x0 * c - x1 * s);
+      *SAL_CK_ST(k + dst + 32 + lane, 2) = __float2bfloat16_rn(x1 * c + x0 * s);
     }
-    v[dst + lane] = __float2bfloat16_rn(src[2 * kW + h * kHd + lane]);
-    v[dst + 32 + lane] = __float2bfloat16_rn(src[2 * kW + h * kHd + 32 + lane]);
+    *SAL_CK_ST(v + dst + lane, 2) = __float2bfloat16_rn(*SAL_CK_LD(src + 2 * kW + h * kHd + lane, 4));
+    *SAL_CK_ST(v + dst + 32 + lane, 2) = __float2bfloat16_rn(*SAL_CK_LD(src + 2 * kW + h * kHd + 32 + lane, 4));
   }
 }
 
@@ -93,7 +96,7 @@ __global__ void __launch_bounds__(kLsThreads) log_softmax_kernel(const float* __
   const float* zr = z + row * ld;
   float m = -INFINITY, s = 0.f;
   for (int i = threadIdx.x; i < n; i += kLsThreads) {
-    const float a = zr[i];  // kept in L2 for the second pass
+    const float a = *SAL_CK_LD(zr + i, 4);  // kept in L2 for the second pass
     if (a > m) {
       s = s * __expf(m - a) + 1.f;
       m = a;
@@ -125,7 +128,7 @@ __global__ void __launch_bounds__(kLsThreads) log_softmax_kernel(const float* __
   __syncthreads();
   const float lse = sm[0];
   float* orow = out + row * static_cast<int64_t>(n);
-  for (int i = threadIdx.x; i < n; i += kLsThreads) __stcs(orow + i, __ldcs(zr + i) - lse);
+  for (int i = threadIdx.x; i < n; i += kLsThreads) __stcs(SAL_CK_ST(orow + i, 4), __ldcs(SAL_CK_LD(zr + i, 4)) - lse);
 }
 
 }  // namespace
@@ -133,6 +136,13 @@ __global__ void __launch_bounds__(kLsThreads) log_softmax_kernel(const float* __
 sal_status ctc_qk_norm_rope_launch(const float* qkv, int64_t rows, int64_t T, const void* qn_g, const void* kn_g,
                                    const float* cs, void* q, void* k, void* v, cudaStream_t s) {
   if (rows == 0) return SAL_OK;
+  ck_declare(qkv, rows * 3 * kW * 4, false);
+  ck_declare(qn_g, kHd * 2, false);
+  ck_declare(kn_g, kHd * 2, false);
+  ck_declare(cs, 2 * T * 64 * 4, false);
+  ck_declare(q, rows * kW * 2, true);
+  ck_declare(k, rows * kW * 2, true);
+  ck_declare(v, rows * kW * 2, true);
   return launch_kernel(ctc_qk_norm_rope_kernel, dim3(static_cast<unsigned>((rows + 7) / 8)), dim3(256), 0, s, qkv,
                        rows, T, static_cast<const __nv_bfloat16*>(qn_g), static_cast<const __nv_bfloat16*>(kn_g), cs,
                        static_cast<__nv_bfloat16*>(q), static_cast<__nv_bfloat16*>(k),
@@ -144,6 +154,8 @@ sal_status ctc_qk_norm_rope_launch(const float* qkv, int64_t rows, int64_t T, co
 sal_status log_softmax_launch(const float* z, int64_t rows, int n, int64_t ld, float* out, cudaStream_t s) {
   if (rows == 0 || n == 0) return SAL_OK;
   if (rows > 0x7fffffff) return SAL_ESHAPE;
+  ck_declare(z, ((rows - 1) * ld + n) * 4, false);
+  ck_declare(out, rows * n * 4, true);
   return launch_kernel(log_softmax_kernel, dim3(static_cast<unsigned>(rows)), dim3(kLsThreads), 0, s, z, rows, n, ld,
                        out) == cudaSuccess
              ? SAL_OK

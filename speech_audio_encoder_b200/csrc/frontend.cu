@@ -29,6 +29,7 @@
 // of a sample or butterfly scales with the strong component (rounding only the window
 // product to fp32 already costs 2e-4 on the 1 s tone clip). The powers and the filter
 // sums round each value relative to itself and stay in fp32.
+#define SAL_CK_FILE 1
 #include <cuda_bf16.h>
 #include <math.h>
 
@@ -164,9 +165,9 @@ __device__ __forceinline__ void stage_pair(float* dst, const float* __restrict__
   const int n = f + 1 < F ? kPairSamples : kWin;
   const float* src = wave + clip * n_samples + kHop * f;
   if (vec) {
-    for (int i = lane; i < n / 4; i += 32) cp_async16(dst + 4 * i, src + 4 * i);
+    for (int i = lane; i < n / 4; i += 32) cp_async16(dst + 4 * i, SAL_CK_LD(src + 4 * i, 16));
   } else {
-    for (int i = lane; i < n; i += 32) cp_async4(dst + i, src + i);
+    for (int i = lane; i < n; i += 32) cp_async4(dst + i, SAL_CK_LD(src + i, 4));
   }
 }
 
@@ -189,7 +190,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   {  // tables (computed once on the host)
     const int4* src = reinterpret_cast<const int4*>(&g_front_tables);
     int4* dst = reinterpret_cast<int4*>(smem_raw);
-    for (int i = tid; i < static_cast<int>(sizeof(FrontTables) / 16); i += kThreads) dst[i] = src[i];
+    for (int i = tid; i < static_cast<int>(sizeof(FrontTables) / 16); i += kThreads) dst[i] = *SAL_CK_LD(src + i, 16);
   }
   __syncthreads();
   pdl_wait();
@@ -309,8 +310,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int j = 0; j < mel_taps(h); ++j) e = fmaf(wk[16 * j], pk[j], e);
         // __logf: absolute error ~1e-6 over the range of e, far inside the 1e-4 budget
         const float lm = __logf(fmaxf(e, 1e-10f));
-        __stcs(out + m, lm);
-        if (sout) sout[m] = __float2bfloat16_rn(lm);
+        __stcs(SAL_CK_ST(out + m, 4), lm);
+        if (sout) *SAL_CK_ST(sout + m, 2) = __float2bfloat16_rn(lm);
       }
     }
     __syncwarp();  // the samples buffer and the scratch are free again
@@ -376,6 +377,7 @@ bool build_tables(FrontTables* t) {
 std::mutex g_init_mu;
 bool g_init_done[64] = {};
 int g_sms[64] = {};
+const void* g_tables_addr[64] = {};  // device address of the tables
 
 sal_status ensure_tables() {
   int dev = 0;
@@ -395,6 +397,9 @@ sal_status ensure_tables() {
   int n = 0;
   if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) return SAL_ECUDA;
   g_sms[dev] = n;
+  void* addr = nullptr;
+  if (cudaGetSymbolAddress(&addr, g_front_tables) != cudaSuccess) return SAL_ECUDA;
+  g_tables_addr[dev] = addr;
   g_init_done[dev] = true;
   return SAL_OK;
 }
@@ -404,6 +409,13 @@ int sm_count() {
   cudaGetDevice(&dev);
   std::lock_guard<std::mutex> lk(g_init_mu);
   return (dev >= 0 && dev < 64 && g_sms[dev] > 0) ? g_sms[dev] : 1;
+}
+
+const void* tables_addr() {
+  int dev = 0;
+  cudaGetDevice(&dev);
+  std::lock_guard<std::mutex> lk(g_init_mu);
+  return (dev >= 0 && dev < 64) ? g_tables_addr[dev] : nullptr;
 }
 
 }  // namespace
@@ -417,6 +429,10 @@ sal_status frontend_launch(const float* wave, int64_t n_samples, int batch, int6
   const int64_t sms = sm_count();
   const dim3 grid(static_cast<unsigned>(ctas < sms ? ctas : sms));
   const int64_t n_stack = stacked ? positions * kStack : 0;
+  ck_declare(wave, batch * n_samples * 4, false);
+  ck_declare(logmel, batch * frames * kMels * 4, true);
+  ck_declare(stacked, batch * n_stack * kMels * 2, true);
+  ck_declare(tables_addr(), sizeof(FrontTables), false);
   return launch_kernel(frontend_kernel, grid, dim3(kThreads), kSmemBytes, s, wave, n_samples, batch, frames, n_stack,
                        logmel, static_cast<__nv_bfloat16*>(stacked)) == cudaSuccess
              ? SAL_OK

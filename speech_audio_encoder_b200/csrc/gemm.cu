@@ -20,6 +20,7 @@
 // Every mbarrier wait is bounded; a wait that gives up flags the device status word
 // and the CTA winds down (waiting, bounded, for its own TMA loads and MMAs in flight)
 // before it frees its TMEM and exits.
+#define SAL_CK_FILE 3
 #include <cuda_bf16.h>
 #include <math.h>
 
@@ -97,7 +98,7 @@ __device__ __forceinline__ float gelu_erf(float x) {
   return fmaf(h, erf_z, h);
 }
 
-__device__ __forceinline__ float bf16_at(const __nv_bfloat16* p, int i) { return __bfloat162float(p[i]); }
+__device__ __forceinline__ float bf16_at(const __nv_bfloat16* p, int i) { return __bfloat162float(*SAL_CK_LD(p + i, 2)); }
 
 // Warp scratch: 32 rows x W fp32 columns, row r at r * W floats; the 16-byte chunk j of a
 // row sits at chunk position (j & ~7) | ((j ^ r) & 7), so a thread-per-row store of 8
@@ -342,8 +343,8 @@ __global__ void __launch_bounds__(Cfg<BN, EPI, PAIR>::THREADS, 1)
       const float sg = lane >= 16 ? 1.f : -1.f;  // i < 64: a c - b s;  i >= 64: b c + a s
       float4 c1 = make_float4(1.f, 1.f, 1.f, 1.f), s1 = make_float4(0.f, 0.f, 0.f, 0.f);
       if (args.rope_rows > 1) {  // table row 1 holds cos / sin of theta_i itself
-        c1 = __ldg(reinterpret_cast<const float4*>(args.rope_cs + 64) + q4);
-        s1 = __ldg(reinterpret_cast<const float4*>(args.rope_cs + (args.rope_rows + 1) * 64) + q4);
+        c1 = __ldg(SAL_CK_LD(reinterpret_cast<const float4*>(args.rope_cs + 64) + q4, 16));
+        s1 = __ldg(SAL_CK_LD(reinterpret_cast<const float4*>(args.rope_cs + (args.rope_rows + 1) * 64) + q4, 16));
       }
       for (int tile = first_tile; tile < num_tiles; tile += tile_step) {
         const int rest = tile / args.splits;
@@ -368,7 +369,7 @@ __global__ void __launch_bounds__(Cfg<BN, EPI, PAIR>::THREADS, 1)
             const uint4* b8 = reinterpret_cast<const uint4*>(args.bias + col0 + cc * 32);
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
-              const uint4 bb = __ldg(b8 + j);
+              const uint4 bb = __ldg(SAL_CK_LD(b8 + j, 16));
               const uint32_t bw[4] = {bb.x, bb.y, bb.z, bb.w};
 #pragma unroll
               for (int e = 0; e < 4; ++e) {
@@ -396,7 +397,7 @@ __global__ void __launch_bounds__(Cfg<BN, EPI, PAIR>::THREADS, 1)
                 uint2 o;
                 o.x = pack_bf16x2(v.x, v.y);
                 o.y = pack_bf16x2(v.z, v.w);
-                reinterpret_cast<uint2*>(dst)[lane] = o;
+                *SAL_CK_ST(reinterpret_cast<uint2*>(dst) + lane, 8) = o;
                 dst += kHeadDim;
                 if (++t == args.T) {  // next clip
                   t = 0;
@@ -407,8 +408,9 @@ __global__ void __launch_bounds__(Cfg<BN, EPI, PAIR>::THREADS, 1)
             } else {
               const __nv_bfloat16* gp = (sec == 0 ? args.qn_g : args.kn_g) + 4 * lane;
               const float4 g4 = make_float4(bf16_at(gp, 0), bf16_at(gp, 1), bf16_at(gp, 2), bf16_at(gp, 3));
-              float4 c = __ldg(reinterpret_cast<const float4*>(args.rope_cs + pos * 64) + q4);
-              float4 sn = __ldg(reinterpret_cast<const float4*>(args.rope_cs + (args.rope_rows + pos) * 64) + q4);
+              float4 c = __ldg(SAL_CK_LD(reinterpret_cast<const float4*>(args.rope_cs + pos * 64) + q4, 16));
+              float4 sn =
+                  __ldg(SAL_CK_LD(reinterpret_cast<const float4*>(args.rope_cs + (args.rope_rows + pos) * 64) + q4, 16));
 #pragma unroll 4
               for (int r = 0; r < nrows; ++r) {
                 float4 v = scr[scr_chunk<128>(r, lane)];
@@ -422,7 +424,7 @@ __global__ void __launch_bounds__(Cfg<BN, EPI, PAIR>::THREADS, 1)
                 uint2 o;
                 o.x = pack_bf16x2(fmaf(sg * p.x, sn.x, v.x * c.x), fmaf(sg * p.y, sn.y, v.y * c.y));
                 o.y = pack_bf16x2(fmaf(sg * p.z, sn.z, v.z * c.z), fmaf(sg * p.w, sn.w, v.w * c.w));
-                reinterpret_cast<uint2*>(dst)[lane] = o;
+                *SAL_CK_ST(reinterpret_cast<uint2*>(dst) + lane, 8) = o;
                 dst += kHeadDim;
                 ++pos;
                 if (++t == args.T) {  // next clip: positions restart at 0
@@ -489,12 +491,12 @@ __global__ void __launch_bounds__(Cfg<BN, EPI, PAIR>::THREADS, 1)
               if (add_bias) {
                 const int cb = col0 + 4 * j;
                 if (cb + 4 <= args.n_valid) {
-                  bb = __ldg(reinterpret_cast<const uint2*>(bias8) + j);
+                  bb = __ldg(SAL_CK_LD(reinterpret_cast<const uint2*>(bias8) + j, 8));
                 } else {  // the last, partial bias chunk
                   const uint16_t* bu = reinterpret_cast<const uint16_t*>(args.bias);
                   uint32_t e[4];
 #pragma unroll
-                  for (int q = 0; q < 4; ++q) e[q] = cb + q < args.n_valid ? bu[cb + q] : 0u;
+                  for (int q = 0; q < 4; ++q) e[q] = cb + q < args.n_valid ? *SAL_CK_LD(bu + cb + q, 2) : 0u;
                   bb = make_uint2(e[0] | (e[1] << 16), e[2] | (e[3] << 16));
                 }
               }
@@ -508,12 +510,12 @@ __global__ void __launch_bounds__(Cfg<BN, EPI, PAIR>::THREADS, 1)
               uint4 bb;
               const int cb = col0 + 8 * j;
               if (cb + 8 <= args.n_valid) {
-                bb = __ldg(bias8 + j);
+                bb = __ldg(SAL_CK_LD(bias8 + j, 16));
               } else {  // the last, partial bias chunk
                 const uint16_t* bu = reinterpret_cast<const uint16_t*>(args.bias);
                 uint32_t e[8];
 #pragma unroll
-                for (int q = 0; q < 8; ++q) e[q] = cb + q < args.n_valid ? bu[cb + q] : 0u;
+                for (int q = 0; q < 8; ++q) e[q] = cb + q < args.n_valid ? *SAL_CK_LD(bu + cb + q, 2) : 0u;
                 bb = make_uint4(e[0] | (e[1] << 16), e[2] | (e[3] << 16), e[4] | (e[5] << 16), e[6] | (e[7] << 16));
               }
               const uint32_t bw[4] = {bb.x, bb.y, bb.z, bb.w};
@@ -741,6 +743,20 @@ sal_status gemm_launch(int epilogue, const void* A, int64_t M, int K, const void
       a.splits *= 2;
   }
   const bool pair = use_pair(M, N, BN, a.splits, is_qkv);
+  ck_declare(A, M * K * 2, false);
+  ck_declare(W, static_cast<int64_t>(n_valid) * K * 2, false);
+  ck_declare(bias, static_cast<int64_t>(n_valid) * 2, false);
+  if (is_qkv) {
+    ck_declare(a.q, M * kWidth * 2, true);
+    ck_declare(a.k, M * kWidth * 2, true);
+    ck_declare(a.v, M * kWidth * 2, true);
+    ck_declare(a.qn_g, kHeadDim * 2, false);
+    ck_declare(a.kn_g, kHeadDim * 2, false);
+    ck_declare(a.rope_cs, a.rope_rows * 2 * 64 * 4, false);
+  } else {
+    const bool f32 = epilogue == SAL_EPI_STORE_F32 || epilogue == SAL_EPI_RESID_F32;
+    ck_declare(out, M * N * (f32 ? 4 : 2), true);
+  }
   switch (epilogue) {
     case SAL_EPI_STORE_F32: return launch_epi<SAL_EPI_STORE_F32>(BN, pair, a, A, W, s);
     case SAL_EPI_STORE_BF16: return launch_epi<SAL_EPI_STORE_BF16>(BN, pair, a, A, W, s);

@@ -51,6 +51,7 @@ using namespace sal;
 
 extern "C" sal_status sal_qkv_rope_noalloc(const void* h, int batch, int64_t T, const sal_layer* layer, void* q,
                                            void* k, void* v, void* stream) {
+  const NvtxRange nvtx_("sal_qkv_rope_noalloc");
   if (batch < 0 || T < 0 || !layer) return SAL_EINVAL;
   if (T > kMaxT) return SAL_ESHAPE;
   if (batch == 0 || T == 0) return SAL_OK;

@@ -22,6 +22,7 @@
 // recording's residual stream into its own left-aligned slot range of a windowed batch
 // (zeroing the slots past the window's length); the scatter copies every window's core
 // rows back in order, dropping the context rows. One warp per row, 16-byte accesses.
+#define SAL_CK_FILE 2
 #include <cuda_bf16.h>
 #include <math.h>
 
@@ -59,7 +60,7 @@ __global__ void __launch_bounds__(256) layernorm_kernel(const float* __restrict_
   float s = 0.f;
 #pragma unroll
   for (int i = 0; i < kVec; ++i) {
-    v[i] = xr[lane + 32 * i];
+    v[i] = *SAL_CK_LD(xr + lane + 32 * i, 16);
     s += (v[i].x + v[i].y) + (v[i].z + v[i].w);
   }
   const float mean = warp_sum(s) * (1.0f / kW);
@@ -76,7 +77,7 @@ __global__ void __launch_bounds__(256) layernorm_kernel(const float* __restrict_
 #pragma unroll
   for (int i = 0; i < kVec; ++i) {
     const int c4 = lane + 32 * i;
-    const uint2 gg = __ldg(g2 + c4), bb = __ldg(b2 + c4);
+    const uint2 gg = __ldg(SAL_CK_LD(g2 + c4, 8)), bb = __ldg(SAL_CK_LD(b2 + c4, 8));
     const float o0 = (v[i].x - mean) * rstd * __uint_as_float(gg.x << 16) + __uint_as_float(bb.x << 16);
     const float o1 = (v[i].y - mean) * rstd * __uint_as_float(gg.x & 0xFFFF0000u) + __uint_as_float(bb.x & 0xFFFF0000u);
     const float o2 = (v[i].z - mean) * rstd * __uint_as_float(gg.y << 16) + __uint_as_float(bb.y << 16);
@@ -85,7 +86,7 @@ __global__ void __launch_bounds__(256) layernorm_kernel(const float* __restrict_
     uint2 out;
     out.x = *reinterpret_cast<uint32_t*>(&p0);
     out.y = *reinterpret_cast<uint32_t*>(&p1);
-    yr[c4] = out;
+    *SAL_CK_ST(yr + c4, 8) = out;
   }
 }
 
@@ -99,8 +100,8 @@ __global__ void rope_table_kernel(float* __restrict__ cs, int64_t T) {
   const double inv = pow(10000.0, -static_cast<double>(2 * i) / 128.0);
   double s, c;
   sincos(static_cast<double>(t) * inv, &s, &c);
-  cs[idx] = static_cast<float>(c);
-  cs[T * 64 + idx] = static_cast<float>(s);
+  *SAL_CK_ST(cs + idx, 4) = static_cast<float>(c);
+  *SAL_CK_ST(cs + T * 64 + idx, 4) = static_cast<float>(s);
 }
 
 constexpr int kSlots = 8;
@@ -118,19 +119,19 @@ __global__ void __launch_bounds__(256) speaker_fuse_kernel(const __nv_bfloat16* 
   {
     const float4* src = reinterpret_cast<const float4*>(&g_speaker_kernel);
     float4* dst = reinterpret_cast<float4*>(sk);
-    for (int i = threadIdx.x; i < kSlots * kWidth / 4; i += blockDim.x) dst[i] = src[i];
+    for (int i = threadIdx.x; i < kSlots * kWidth / 4; i += blockDim.x) dst[i] = *SAL_CK_LD(src + i, 16);
   }
   __syncthreads();
   pdl_wait();
   pdl_trigger();
   const int lane = threadIdx.x & 31;
   const int s = lane & 7;
-  const float gs = __bfloat162float(g[s]), bs = __bfloat162float(b[s]);
+  const float gs = __bfloat162float(*SAL_CK_LD(g + s, 2)), bs = __bfloat162float(*SAL_CK_LD(b + s, 2));
   const int64_t warps = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
   for (int64_t row = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5); row < rows;
        row += warps) {
     // every group of 8 lanes holds the 8 slots of this position
-    const float a = P[row * kSlots + s] > 0.5f ? 1.f : 0.f;
+    const float a = *SAL_CK_LD(P + row * kSlots + s, 4) > 0.5f ? 1.f : 0.f;
     float sum = a;
 #pragma unroll
     for (int o = 1; o < kSlots; o <<= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
@@ -147,7 +148,7 @@ __global__ void __launch_bounds__(256) speaker_fuse_kernel(const __nv_bfloat16* 
 #pragma unroll
     for (int i = 0; i < kWidth / 128; ++i) {
       const int c4 = lane + 32 * i;  // columns 4 c4 .. 4 c4 + 3
-      const uint2 hv = hr[c4];
+      const uint2 hv = *SAL_CK_LD(hr + c4, 8);
       float o0 = __uint_as_float(hv.x << 16), o1 = __uint_as_float(hv.x & 0xFFFF0000u);
       float o2 = __uint_as_float(hv.y << 16), o3 = __uint_as_float(hv.y & 0xFFFF0000u);
 #pragma unroll
@@ -162,7 +163,7 @@ __global__ void __launch_bounds__(256) speaker_fuse_kernel(const __nv_bfloat16* 
       uint2 ov;
       ov.x = *reinterpret_cast<uint32_t*>(&p0);
       ov.y = *reinterpret_cast<uint32_t*>(&p1);
-      orow[c4] = ov;
+      *SAL_CK_ST(orow + c4, 8) = ov;
     }
   }
 }
@@ -190,10 +191,10 @@ __global__ void __launch_bounds__(256) window_gather_kernel(const float* __restr
   if (lo + i < hi) {
     const float4* src = reinterpret_cast<const float4*>(x + (b * wn.total + lo + i) * kWidth);
 #pragma unroll
-    for (int c = 0; c < kWidth / 128; ++c) dst[lane + 32 * c] = src[lane + 32 * c];
+    for (int c = 0; c < kWidth / 128; ++c) *SAL_CK_ST(dst + lane + 32 * c, 16) = *SAL_CK_LD(src + lane + 32 * c, 16);
   } else {
 #pragma unroll
-    for (int c = 0; c < kWidth / 128; ++c) dst[lane + 32 * c] = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int c = 0; c < kWidth / 128; ++c) *SAL_CK_ST(dst + lane + 32 * c, 16) = make_float4(0.f, 0.f, 0.f, 0.f);
   }
 }
 
@@ -211,17 +212,18 @@ __global__ void __launch_bounds__(256) window_scatter_kernel(const __nv_bfloat16
   const int64_t src_row = (b * wn.count + w) * wn.slot + (t - window_lo(wn, w));
   const uint4* se = reinterpret_cast<const uint4*>(embw + src_row * kWidth);
   uint4* de = reinterpret_cast<uint4*>(emb + row * kWidth);
-  for (int c = lane; c < kWidth / 8; c += 32) de[c] = se[c];
+  for (int c = lane; c < kWidth / 8; c += 32) *SAL_CK_ST(de + c, 16) = *SAL_CK_LD(se + c, 16);
   if (x) {
     const float4* sx = reinterpret_cast<const float4*>(xw + src_row * kWidth);
     float4* dx = reinterpret_cast<float4*>(x + row * kWidth);
 #pragma unroll
-    for (int c = 0; c < kWidth / 128; ++c) dx[lane + 32 * c] = sx[lane + 32 * c];
+    for (int c = 0; c < kWidth / 128; ++c) *SAL_CK_ST(dx + lane + 32 * c, 16) = *SAL_CK_LD(sx + lane + 32 * c, 16);
   }
 }
 
 std::mutex g_spk_mu;
 bool g_spk_done[64] = {};
+const void* g_spk_addr[64] = {};  // device address of the speaker kernel table
 
 sal_status ensure_speaker_kernel() {
   int dev = 0;
@@ -239,6 +241,9 @@ sal_status ensure_speaker_kernel() {
   if (cudaFuncSetAttribute(speaker_fuse_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            static_cast<int>(sizeof(SpeakerKernel))) != cudaSuccess)
     return SAL_ECUDA;
+  void* addr = nullptr;
+  if (cudaGetSymbolAddress(&addr, g_speaker_kernel) != cudaSuccess) return SAL_ECUDA;
+  g_spk_addr[dev] = addr;
   g_spk_done[dev] = true;
   return SAL_OK;
 }
@@ -256,6 +261,12 @@ sal_status speaker_fuse_launch(const void* H, const float* P, int64_t rows, cons
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const int64_t want = (rows + 7) / 8;
   const unsigned grid = static_cast<unsigned>(want < 4 * sms ? want : 4 * sms);
+  ck_declare(H, rows * kWidth * 2, false);
+  ck_declare(P, rows * kSlots * 4, false);
+  ck_declare(g, kSlots * 2, false);
+  ck_declare(b, kSlots * 2, false);
+  ck_declare(out, rows * kWidth * 2, true);
+  ck_declare(g_spk_addr[dev], sizeof(SpeakerKernel), false);
   return launch_kernel(speaker_fuse_kernel, dim3(grid), dim3(256), sizeof(SpeakerKernel), s,
                        static_cast<const __nv_bfloat16*>(H), P, rows, static_cast<const __nv_bfloat16*>(g),
                        static_cast<const __nv_bfloat16*>(b), static_cast<__nv_bfloat16*>(out)) == cudaSuccess
@@ -270,6 +281,10 @@ sal_status layernorm_launch(const float* x, int64_t rows, const void* g, const v
   const auto gg = static_cast<const __nv_bfloat16*>(g);
   const auto bb = static_cast<const __nv_bfloat16*>(b);
   const auto yy = static_cast<__nv_bfloat16*>(y);
+  ck_declare(x, rows * width * 4, false);
+  ck_declare(g, width * 2, false);
+  ck_declare(b, width * 2, false);
+  ck_declare(y, rows * width * 2, true);
   cudaError_t e;
   if (width == kWidth)
     e = launch_kernel(layernorm_kernel<kWidth / 128>, dim3(grid), dim3(32 * kLnWarps), 0, s, x, rows, gg, bb, yy);
@@ -283,6 +298,8 @@ sal_status layernorm_launch(const float* x, int64_t rows, const void* g, const v
 sal_status window_gather_launch(const float* x, int batch, const Windows& win, float* xw, cudaStream_t s) {
   const int64_t rows = static_cast<int64_t>(batch) * win.count * win.slot;
   if (rows == 0) return SAL_OK;
+  ck_declare(x, batch * win.total * kWidth * 4, false);
+  ck_declare(xw, rows * kWidth * 4, true);
   return launch_kernel(window_gather_kernel, dim3(static_cast<unsigned>((rows + 7) / 8)), dim3(256), 0, s, x, batch,
                        win, xw) == cudaSuccess
              ? SAL_OK
@@ -293,6 +310,13 @@ sal_status window_scatter_launch(const void* embw, const float* xw, int batch, c
                                  float* x, cudaStream_t s) {
   const int64_t rows = static_cast<int64_t>(batch) * win.total;
   if (rows == 0) return SAL_OK;
+  const int64_t wrows = static_cast<int64_t>(batch) * win.count * win.slot;
+  ck_declare(embw, wrows * kWidth * 2, false);
+  ck_declare(emb, rows * kWidth * 2, true);
+  if (x) {
+    ck_declare(xw, wrows * kWidth * 4, false);
+    ck_declare(x, rows * kWidth * 4, true);
+  }
   return launch_kernel(window_scatter_kernel, dim3(static_cast<unsigned>((rows + 7) / 8)), dim3(256), 0, s,
                        static_cast<const __nv_bfloat16*>(embw), xw, batch, win, static_cast<__nv_bfloat16*>(emb),
                        x) == cudaSuccess
@@ -303,6 +327,7 @@ sal_status window_scatter_launch(const void* embw, const float* xw, int batch, c
 sal_status rope_table_launch(float* cs, int64_t T, cudaStream_t s) {
   if (T == 0) return SAL_OK;
   const int64_t n = T * 64;
+  ck_declare(cs, 2 * n * 4, true);
   return launch_kernel(rope_table_kernel, dim3(static_cast<unsigned>((n + 255) / 256)), dim3(256), 0, s, cs, T) ==
                  cudaSuccess
              ? SAL_OK

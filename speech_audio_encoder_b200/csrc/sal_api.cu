@@ -15,6 +15,7 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <cstdio>
 #include <cstdlib>
 #include <atomic>
 #include <mutex>
@@ -191,6 +192,75 @@ unsigned int* device_status_ptr() {
   return ptrs[dev];
 }
 
+#ifdef SAL_CHECKED
+// Bounds-checked build: the ranges declared on this thread since its last launch, the
+// test hook's shortening of writable ranges, and per device the report and the sink.
+namespace {
+struct CkPending {
+  CkTable t{};
+  bool overflow = false;
+};
+thread_local CkPending g_ck;
+std::atomic<uint64_t> g_ck_shrink{0};
+struct CkDevice {
+  CkReport* report = nullptr;
+  void* sink = nullptr;
+};
+CkDevice g_ck_dev[64];
+std::mutex g_ck_mu;
+constexpr CkReport kCkClear = {0ull, ~0ull, ~0ull};
+
+CkDevice* ck_device() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  std::lock_guard<std::mutex> lk(g_ck_mu);
+  CkDevice& d = g_ck_dev[dev];
+  if (!d.report) {
+    void *r = nullptr, *k = nullptr;
+    if (cudaMalloc(&r, sizeof(CkReport)) != cudaSuccess) return nullptr;
+    if (cudaMalloc(&k, kCkSinkBytes) != cudaSuccess ||
+        cudaMemcpy(r, &kCkClear, sizeof(CkReport), cudaMemcpyHostToDevice) != cudaSuccess) {
+      cudaFree(r);
+      if (k) cudaFree(k);
+      return nullptr;
+    }
+    d.report = static_cast<CkReport*>(r);
+    d.sink = k;
+  }
+  return &d;
+}
+}  // namespace
+
+void ck_declare(const void* p, uint64_t bytes, bool writable) {
+  if (!p) return;
+  CkPending& pnd = g_ck;
+  if (pnd.t.n >= kCkSpans) {
+    pnd.overflow = true;
+    return;
+  }
+  if (writable) {
+    const uint64_t sh = g_ck_shrink.load();
+    bytes = bytes > sh ? bytes - sh : 0;
+  }
+  const int i = pnd.t.n++;
+  pnd.t.lo[i] = reinterpret_cast<uintptr_t>(p);
+  pnd.t.hi[i] = pnd.t.lo[i] + bytes;
+  if (writable) pnd.t.writable |= 1u << i;
+}
+
+bool ck_take(CkTable* t) {
+  CkPending& pnd = g_ck;
+  CkDevice* d = ck_device();
+  const bool ok = d && !pnd.overflow;
+  *t = pnd.t;
+  t->seq = g_launches.load();
+  t->report = d ? d->report : nullptr;
+  t->sink = d ? d->sink : nullptr;
+  pnd = CkPending{};
+  return ok;
+}
+#endif
+
 bool make_tmap_2d_bf16(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer,
                        uint32_t box_inner, uint32_t box_outer) {
   auto fn = encode_fn();
@@ -240,6 +310,12 @@ using namespace sal;
     if (st_ != SAL_OK) return st_;    \
   } while (0)
 
+namespace {
+// Stage names, indexed by the SAL_KIND_* values.
+const char* const kKindNames[SAL_KIND_COUNT] = {"rope_table", "layernorm", "qkv", "attention",
+                                                "out_proj", "ffn_up", "ffn_down"};
+}  // namespace
+
 extern "C" {
 
 int64_t sal_frame_count(int64_t n) { return n < kWin ? 0 : 1 + (n - kWin) / kHop; }
@@ -255,11 +331,53 @@ const char* sal_status_string(int status) {
     case SAL_ECUDA: return "CUDA runtime error";
     case SAL_ETIMEOUT: return "a bounded device wait gave up";
     case SAL_EDEVICE: return "device is not an sm_100 GPU";
+    case SAL_EIO: return "a file could not be opened or read";
     default: return "unknown status";
   }
 }
 
 void sal_set_wait_limit_ns(uint64_t ns) { g_wait_limit_ns.store(ns ? ns : 1); }
+
+int sal_checked_build(void) {
+#ifdef SAL_CHECKED
+  return 1;
+#else
+  return 0;
+#endif
+}
+
+sal_status sal_check_report(uint64_t* count, uint64_t* first_address, int* file, int* line, uint64_t* first_launch) {
+  if (!count || !first_address || !file || !line || !first_launch) return SAL_EINVAL;
+  *count = *first_address = *first_launch = 0;
+  *file = *line = 0;
+#ifdef SAL_CHECKED
+  CkDevice* d = ck_device();
+  if (!d) return SAL_ECUDA;
+  if (cudaDeviceSynchronize() != cudaSuccess) return SAL_ECUDA;
+  CkReport r;
+  if (cudaMemcpy(&r, d->report, sizeof(r), cudaMemcpyDeviceToHost) != cudaSuccess ||
+      cudaMemcpy(d->report, &kCkClear, sizeof(r), cudaMemcpyHostToDevice) != cudaSuccess)
+    return SAL_ECUDA;
+  *count = r.count;
+  if (r.count) {
+    *first_address = r.min_key >> 16;
+    *file = static_cast<int>((r.min_key >> 12) & 15u);
+    *line = static_cast<int>(r.min_key & 4095u);
+    *first_launch = r.min_seq;
+  }
+  return SAL_OK;
+#else
+  return SAL_EINVAL;
+#endif
+}
+
+void sal_check_shrink_writable(uint64_t bytes) {
+#ifdef SAL_CHECKED
+  g_ck_shrink.store(bytes);
+#else
+  (void)bytes;
+#endif
+}
 
 sal_status sal_last_device_status(void* stream) {
   if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return SAL_ECUDA;
@@ -271,6 +389,7 @@ sal_status sal_last_device_status(void* stream) {
 
 sal_status sal_frontend(const float* wave, int64_t n_samples, int batch, float* logmel, void* stacked,
                         void* stream) {
+  const NvtxRange nvtx_("sal_frontend");
   if (batch < 0 || n_samples < 0) return SAL_EINVAL;
   const int64_t F = sal_frame_count(n_samples), T = F / kStack;
   if (T > SAL_MAX_POSITIONS) return SAL_ESHAPE;
@@ -284,6 +403,7 @@ sal_status sal_frontend(const float* wave, int64_t n_samples, int batch, float* 
 
 sal_status sal_stack_project(const void* stacked, int batch, int64_t T, const sal_weights* w, float* x,
                              void* stream) {
+  const NvtxRange nvtx_("sal_stack_project");
   if (batch < 0 || T < 0 || !w) return SAL_EINVAL;
   if (T > SAL_MAX_POSITIONS) return SAL_ESHAPE;
   if (batch == 0 || T == 0) return SAL_OK;
@@ -320,6 +440,7 @@ size_t sal_encoder_workspace_bytes_ex(int batch, int64_t T, const sal_forward_op
 
 sal_status sal_encoder_forward(float* x, int batch, int64_t T, const sal_weights* w, int n_layers, void* emb,
                                void* workspace, size_t ws_bytes, void* stream) {
+  const NvtxRange nvtx_("sal_encoder_forward");
   return sal_encoder_forward_ex(x, batch, T, w, n_layers, emb, workspace, ws_bytes, stream, nullptr);
 }
 
@@ -347,6 +468,7 @@ struct Tracer {
 
 #define SAL_TRACED(kind, expr)                              \
   do {                                                      \
+    const NvtxRange stage_(kKindNames[kind]);               \
     if (!tr.before(kind)) return SAL_ECUDA;                 \
     SAL_TRY(expr);                                          \
     if (!tr.after(kind)) return SAL_ECUDA;                  \
@@ -360,6 +482,9 @@ sal_status run_layers(float* x, int batch, int64_t T, const sal_weights* w, int 
   const int64_t M = static_cast<int64_t>(batch) * T;
   if (n_layers > 0) SAL_TRACED(SAL_KIND_ROPE_TABLE, rope_table_launch(ws.rope, chunk, s));
   for (int i = 0; i < n_layers; ++i) {
+    char name[16];
+    snprintf(name, sizeof(name), "layer %d", i);
+    const NvtxRange layer(name);
     const sal_layer& L = w->layers[i];
     SAL_TRACED(SAL_KIND_LAYERNORM, layernorm_launch(x, M, L.ln1_g, L.ln1_b, ws.h, s));
     QkvOut qo{ws.q, ws.k, ws.v, L.qn_g, L.kn_g, ws.rope, T, chunk};
@@ -379,6 +504,7 @@ sal_status run_layers(float* x, int batch, int64_t T, const sal_weights* w, int 
 
 sal_status sal_encoder_forward_ex(float* x, int batch, int64_t T, const sal_weights* w, int n_layers, void* emb,
                                   void* workspace, size_t ws_bytes, void* stream, const sal_forward_options* opts) {
+  const NvtxRange nvtx_("sal_encoder_forward_ex");
   const sal_trace* trace = opts ? opts->trace : nullptr;
   const int64_t chunk = (opts && opts->chunk > 0 && opts->chunk < T) ? opts->chunk : T;
   if (batch < 0 || T < 0 || !w || n_layers < 0 || n_layers > w->n_layers) return SAL_EINVAL;
@@ -439,6 +565,7 @@ size_t sal_encode_workspace_bytes(int batch, int64_t n_samples) {
 
 sal_status sal_encode(const float* wave, int64_t n_samples, int batch, const sal_weights* w, int n_layers,
                       void* emb, void* workspace, size_t ws_bytes, void* stream) {
+  const NvtxRange nvtx_("sal_encode");
   if (batch < 0 || n_samples < 0 || !w) return SAL_EINVAL;
   const int64_t F = sal_frame_count(n_samples), T = F / kStack;
   if (T > SAL_MAX_POSITIONS) return SAL_ESHAPE;
@@ -480,6 +607,7 @@ sal_status sal_encode(const float* wave, int64_t n_samples, int batch, const sal
 }
 
 sal_status sal_layernorm(const float* x, int64_t rows, const void* g, const void* b, void* y, void* stream) {
+  const NvtxRange nvtx_("sal_layernorm");
   if (rows < 0) return SAL_EINVAL;
   if (rows == 0) return SAL_OK;
   if (!x || !g || !b || !y || !aligned16(x) || !aligned16(g) || !aligned16(b) || !aligned16(y)) return SAL_EINVAL;
@@ -489,6 +617,7 @@ sal_status sal_layernorm(const float* x, int64_t rows, const void* g, const void
 
 sal_status sal_linear(int epilogue, const void* A, int64_t M, int K, const void* W, int N, const void* bias,
                       void* out, void* stream) {
+  const NvtxRange nvtx_("sal_linear");
   if (epilogue < SAL_EPI_STORE_F32 || epilogue > SAL_EPI_RESID_F32 || M < 0) return SAL_EINVAL;
   if (M == 0) return SAL_OK;
   if (!A || !W || !bias || !out || !aligned16(A) || !aligned16(W) || !aligned16(bias) || !aligned16(out))
@@ -499,6 +628,7 @@ sal_status sal_linear(int epilogue, const void* A, int64_t M, int K, const void*
 
 sal_status sal_qkv_rope(const void* h, int batch, int64_t T, const sal_layer* layer, void* q, void* k, void* v,
                         float* rope_cs, void* stream) {
+  const NvtxRange nvtx_("sal_qkv_rope");
   if (batch < 0 || T < 0 || !layer) return SAL_EINVAL;
   if (T > SAL_MAX_POSITIONS) return SAL_ESHAPE;
   if (batch == 0 || T == 0) return SAL_OK;
@@ -516,6 +646,7 @@ sal_status sal_qkv_rope(const void* h, int batch, int64_t T, const sal_layer* la
 
 sal_status sal_speaker_fuse(const void* H, const float* P, int64_t rows, const void* g, const void* b, void* out,
                             void* stream) {
+  const NvtxRange nvtx_("sal_speaker_fuse");
   if (rows < 0) return SAL_EINVAL;
   if (rows == 0) return SAL_OK;
   if (!H || !P || !g || !b || !out || !aligned16(H) || !aligned16(P) || !aligned16(g) || !aligned16(b) ||
@@ -526,6 +657,7 @@ sal_status sal_speaker_fuse(const void* H, const float* P, int64_t rows, const v
 }
 
 sal_status sal_connector(const void* x, int64_t rows, const void* W, const void* bias, void* out, void* stream) {
+  const NvtxRange nvtx_("sal_connector");
   if (rows < 0) return SAL_EINVAL;
   if (rows == 0) return SAL_OK;
   if (!x || !W || !bias || !out || !aligned16(x) || !aligned16(W) || !aligned16(bias) || !aligned16(out))
@@ -537,11 +669,13 @@ sal_status sal_connector(const void* x, int64_t rows, const void* W, const void*
 
 sal_status sal_attention(const void* q, const void* k, const void* v, int batch, int64_t T, void* o,
                          void* stream) {
+  const NvtxRange nvtx_("sal_attention");
   return sal_attention_chunked(q, k, v, batch, T, 0, o, stream);
 }
 
 sal_status sal_attention_chunked(const void* q, const void* k, const void* v, int batch, int64_t T,
                                  int64_t chunk, void* o, void* stream) {
+  const NvtxRange nvtx_("sal_attention_chunked");
   if (batch < 0 || T < 0) return SAL_EINVAL;
   if (T > SAL_MAX_POSITIONS) return SAL_ESHAPE;
   if (batch == 0 || T == 0) return SAL_OK;
@@ -554,6 +688,7 @@ sal_status sal_attention_chunked(const void* q, const void* k, const void* v, in
 
 sal_status sal_attention_heads(const void* q, const void* k, const void* v, int batch, int64_t T, int heads,
                                int head_dim, void* o, void* stream) {
+  const NvtxRange nvtx_("sal_attention_heads");
   if (batch < 0 || T < 0 || heads < 0) return SAL_EINVAL;
   if (head_dim != 64 && head_dim != 128) return SAL_ESHAPE;
   if (T > 2 * SAL_MAX_POSITIONS) return SAL_ESHAPE;
@@ -566,6 +701,7 @@ sal_status sal_attention_heads(const void* q, const void* k, const void* v, int 
 }
 
 sal_status sal_log_softmax(const float* z, int64_t rows, int n, int64_t ld, float* out, void* stream) {
+  const NvtxRange nvtx_("sal_log_softmax");
   if (rows < 0 || n < 0 || ld < n) return SAL_EINVAL;
   if (rows == 0 || n == 0) return SAL_OK;
   if (!z || !out) return SAL_EINVAL;
@@ -580,6 +716,7 @@ size_t sal_ctc_workspace_bytes(int batch, int64_t T) {
 
 sal_status sal_ctc_adapter(const void* h, int batch, int64_t T, const sal_ctc_weights* w, float* logp,
                            void* workspace, size_t ws_bytes, void* stream) {
+  const NvtxRange nvtx_("sal_ctc_adapter");
   if (batch < 0 || T < 0 || !w || w->n_layers < 0) return SAL_EINVAL;
   if (T > SAL_MAX_POSITIONS || batch > 4095) return SAL_ESHAPE;  // attention grid.y = 16 * batch
   if (batch == 0 || T == 0) return SAL_OK;

@@ -3,11 +3,13 @@
 
 #include <cuda.h>
 #include <cuda_runtime.h>
+#include <nvtx3/nvToolsExt.h>
 #include <stdint.h>
 
 #include <utility>
 
 #include "../../include/sal.h"
+#include "sal_check.cuh"
 
 namespace sal {
 
@@ -34,6 +36,17 @@ struct Windows {
   int64_t slot = 0;
 };
 Windows make_windows(int64_t total, int64_t core, int64_t ctx);  // sal_api.cu
+
+// An NVTX range for the lifetime of the object: every compute entry point, every encoder
+// layer and every stage of a layer is one, so a profiler that reads NVTX (Nsight Compute's
+// --nvtx filters, Nsight Systems) can attribute kernels to them. Without such a tool
+// attached a push or pop costs a few nanoseconds of host time.
+struct NvtxRange {
+  explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+  NvtxRange(const NvtxRange&) = delete;
+  NvtxRange& operator=(const NvtxRange&) = delete;
+};
 
 uint64_t wait_limit_ns();
 bool pdl_enabled();  // programmatic dependent launch (env SAL_PDL=0 turns it off)
@@ -101,14 +114,28 @@ bool make_tmap_2d_f32(CUtensorMap* map, const void* base, uint64_t inner, uint64
 bool make_tmap_3d_bf16(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1, uint64_t d2,
                        uint32_t b0, uint32_t b1, uint32_t b2);
 
+// The launch helpers have internal linkage: in the bounds-checked build each one writes
+// the range table of the translation unit that holds the kernel.
+namespace {
+
 // Launches `kernel` on `s` with programmatic dependent launch allowed: the kernel may be
 // scheduled while its predecessor on the stream is still running, runs its prologue, and
 // waits in griddepcontrol.wait (every kernel of this library does so before touching
 // global memory) until the predecessor has completed.
 // cluster_x > 1: thread-block clusters of cluster_x CTAs along x (grid.x a multiple of it).
+// Bounds-checked build: the ranges declared since the previous launch are copied into
+// this unit's table first (stream-ordered, so the previous launch has finished with it).
 template <typename... KArgs, typename... Args>
 cudaError_t launch_kernel_cluster(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
                                   unsigned cluster_x, Args&&... args) {
+#if defined(SAL_CHECKED) && defined(__CUDACC__)
+  {
+    CkTable t;
+    if (!ck_take(&t)) return cudaErrorMemoryAllocation;
+    const cudaError_t e = cudaMemcpyToSymbolAsync(sal_ck_table, &t, sizeof(t), 0, cudaMemcpyHostToDevice, s);
+    if (e != cudaSuccess) return e;
+  }
+#endif
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = grid;
   cfg.blockDim = block;
@@ -139,6 +166,8 @@ cudaError_t launch_kernel(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_
                           Args&&... args) {
   return launch_kernel_cluster(kernel, grid, block, smem, s, 1u, std::forward<Args>(args)...);
 }
+
+}  // namespace
 
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 

@@ -182,6 +182,75 @@ def weights_f32(w: dict) -> dict:
     return out
 
 
+# ----------------------------------------------------------------------------- weight file
+# The library's flat weight file (include/sal.h, "Flat weight file"): a 256-byte header,
+# then every tensor as row-major bf16 on a 256-byte boundary, globals first, then layer by
+# layer in LAYER_TENSORS order. The generator writes it; the oracle's tests and the
+# library (sal_weights_file_load) read it.
+
+WEIGHT_FILE_MAGIC = b"SALENCW1"
+WEIGHT_FILE_ORDER_GLOBAL = ("w_proj", "b_proj", "lnf_g", "lnf_b")
+
+
+def _padded_bytes(n_elems: int) -> int:
+    return (2 * n_elems + 255) // 256 * 256
+
+
+def _weight_file_tensors(w: dict):
+    """(name, layer or None, bf16 bits) in file order."""
+    for k in WEIGHT_FILE_ORDER_GLOBAL:
+        yield k, None, w[k][0]
+    for i, lw in enumerate(w["layers"]):
+        for name, _, _ in LAYER_TENSORS:
+            yield name, i, lw[name][0]
+
+
+def write_weight_file(w: dict, path: str, width: int = 1280, heads: int = 10, head_dim: int = 128,
+                      ffn: int = 5120, stack_in: int = 1024) -> int:
+    """Writes :func:`make_weights` output to `path`; returns the data size D in bytes."""
+    data = sum(_padded_bytes(b.size) for _, _, b in _weight_file_tensors(w))
+    header = bytearray(256)
+    header[0:8] = WEIGHT_FILE_MAGIC
+    fields = [1, 256, 1, width, heads, head_dim, ffn, stack_in, len(w["layers"]), 256]
+    header[8:48] = np.asarray(fields, dtype="<u4").tobytes()
+    header[48:56] = np.asarray([data], dtype="<u8").tobytes()
+    with open(path, "wb") as f:
+        f.write(bytes(header))
+        for _, _, bits in _weight_file_tensors(w):
+            raw = np.ascontiguousarray(bits, dtype="<u2").tobytes()
+            f.write(raw)
+            f.write(bytes(_padded_bytes(bits.size) - len(raw)))
+    return data
+
+
+def read_weight_file(path: str, width: int = 1280, ffn: int = 5120, head_dim: int = 128,
+                     stack_in: int = 1024) -> dict:
+    """Reads a weight file back into the :func:`make_weights` form ``(bits, f32)``."""
+    raw = np.fromfile(path, dtype=np.uint8)
+    if raw[:8].tobytes() != WEIGHT_FILE_MAGIC:
+        raise ValueError(f"{path}: not a weight file")
+    fields = raw[8:48].view("<u4")
+    n_layers = int(fields[8])
+    if tuple(int(v) for v in fields[3:8]) != (width, 10, head_dim, ffn, stack_in):
+        raise ValueError(f"{path}: sizes {tuple(fields[3:8])} differ")
+    data = int(raw[48:56].view("<u8")[0])
+    if raw.size != 256 + data:
+        raise ValueError(f"{path}: {raw.size} bytes, header says {256 + data}")
+    out: dict = {"layers": [{} for _ in range(n_layers)]}
+    shapes = {name: shp(width, stack_in) for name, shp, _ in GLOBAL_TENSORS}
+    layer_shapes = {name: shp(width, ffn, head_dim) for name, shp, _ in LAYER_TENSORS}
+    off = 256
+    order = [(k, None) for k in WEIGHT_FILE_ORDER_GLOBAL]
+    order += [(name, i) for i in range(n_layers) for name, _, _ in LAYER_TENSORS]
+    for name, i in order:
+        shape = shapes[name] if i is None else layer_shapes[name]
+        n = int(np.prod(shape))
+        bits = raw[off:off + 2 * n].view("<u2").reshape(shape).astype(np.uint16)
+        off += _padded_bytes(n)
+        (out if i is None else out["layers"][i])[name] = (bits, bf16_to_f32(bits))
+    return out
+
+
 def random_bf16(shape, seed: int, std: float = 1.0):
     """N(0, std^2) values rounded to bf16: (bits, float32 values)."""
     b = bf16_bits(np.random.default_rng(seed).normal(0.0, std, shape))

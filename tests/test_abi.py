@@ -37,6 +37,32 @@ def test_every_declared_symbol_is_exported(api):
         assert n in api.EXPORTS, f"{n} has no binding"
 
 
+def test_checked_build_exports_the_same_calls(api):
+    """libsal_checked.so (the bounds-checked build) exports every declared call too, and
+    each library says which build it is. Only host-side calls: no CUDA call is made."""
+    import ctypes
+    names = _declared()
+    for n in ("sal_checked_build", "sal_check_report", "sal_check_shrink_writable"):
+        assert n in names
+    assert api.lib().sal_checked_build() == 0
+    with api.checked_library() as lc:
+        assert api.lib() is lc
+        for n in names:
+            assert hasattr(lc, n), n
+        assert lc.sal_checked_build() == 1
+        # argument checks return before any CUDA call in the checked build as well
+        assert lc.sal_frontend(None, 16000, -1, None, None, None) == 1
+        assert lc.sal_check_report(None, None, None, None, None) == 1
+    assert api.lib().sal_checked_build() == 0
+    # the normal build has no report: SAL_EINVAL, outputs zeroed
+    c, a, s = ctypes.c_uint64(7), ctypes.c_uint64(7), ctypes.c_uint64(7)
+    f, ln = ctypes.c_int(7), ctypes.c_int(7)
+    st = api.lib().sal_check_report(ctypes.byref(c), ctypes.byref(a), ctypes.byref(f), ctypes.byref(ln),
+                                    ctypes.byref(s))
+    assert st == 1 and (c.value, a.value, f.value, ln.value, s.value) == (0, 0, 0, 0, 0)
+    api.lib().sal_check_shrink_writable(0)  # no effect in the normal build
+
+
 def test_counts_match_oracle(api):
     for n in list(range(0, 2000, 7)) + [480000, 960000, 9600000, 57600000]:
         assert api.frame_count(n) == O.frame_count(n)
@@ -44,8 +70,9 @@ def test_counts_match_oracle(api):
 
 
 def test_status_strings(api):
-    for s in range(7):
+    for s in range(8):
         assert api.status_string(s)
+        assert "unknown" not in api.status_string(s)
     assert "unknown" in api.status_string(99)
 
 
