@@ -1068,11 +1068,14 @@ sal_status attention_launch_heads(const void* q, const void* k, const void* v, i
     a.win_total = win->total;
   }
   const dim3 grid1(static_cast<unsigned>((T + kTile - 1) / kTile), static_cast<unsigned>(bh));
-  const int64_t bytes = static_cast<int64_t>(bh) * T * head_dim * 2;  // each of q, k, v and o
-  ck_declare(q, bytes, false);
-  ck_declare(k, bytes, false);
-  ck_declare(v, bytes, false);
-  ck_declare(o, bytes, true);
+  // bounds-checked build: the buffers a launch may touch, declared right before it
+  auto declare = [&] {
+    const int64_t bytes = static_cast<int64_t>(bh) * T * head_dim * 2;  // each of q, k, v and o
+    ck_declare(q, bytes, false);
+    ck_declare(k, bytes, false);
+    ck_declare(v, bytes, false);
+    ck_declare(o, bytes, true);
+  };
   if (head_dim == 64) {
     // the CTC adapter's heads: every query-tile pair to the two-tile kernel and an odd last
     // tile to a split-mode CTA of the same launch, unless it is unavailable or switched off
@@ -1085,6 +1088,7 @@ sal_status attention_launch_heads(const void* q, const void* k, const void* v, i
       const int n_qt = static_cast<int>((T + kTile - 1) / kTile);
       a.pairs = n_qt / 2;
       const dim3 grid(static_cast<unsigned>(n_qt / 2 + n_qt % 2), static_cast<unsigned>(bh));
+      declare();
       const cudaError_t e =
           n_qt % 2 ? launch_kernel(attention_pp_kernel<64, true>, grid, dim3(kThreadsPP), PPLayout<64>::kSmem, s,
                                    tq, tk, tv, a)
@@ -1092,6 +1096,7 @@ sal_status attention_launch_heads(const void* q, const void* k, const void* v, i
                                    tq, tk, tv, a);
       return e == cudaSuccess ? SAL_OK : SAL_ECUDA;
     }
+    declare();
     return launch_kernel(attention_kernel<64>, grid1, dim3(192), smem_one_tile(64), s, tq, tk, tv, a) ==
                    cudaSuccess
                ? SAL_OK
@@ -1125,6 +1130,7 @@ sal_status attention_launch_heads(const void* q, const void* k, const void* v, i
     const int rest = n_qt - 2 * P > 0 ? n_qt - 2 * P : 0;
     a.pairs = P;
     const dim3 grid(static_cast<unsigned>(P + rest), static_cast<unsigned>(bh));
+    declare();
     const cudaError_t e =
         rest > 0 ? launch_kernel(attention_pp_kernel<128, true>, grid, dim3(kThreadsPP), PPLayout<128>::kSmem, s,
                                  tq, tk, tv, a)
@@ -1132,6 +1138,7 @@ sal_status attention_launch_heads(const void* q, const void* k, const void* v, i
                                  tq, tk, tv, a);
     return e == cudaSuccess ? SAL_OK : SAL_ECUDA;
   }
+  declare();
   return launch_kernel(attention_kernel<128>, grid1, dim3(192), smem_one_tile(128), s, tq, tk, tv, a) ==
                  cudaSuccess
              ? SAL_OK

@@ -635,6 +635,20 @@ sal_status launch_bn(const GemmArgs& a, const void* A, const void* W, cudaStream
   } else {
     if (!make_tmap_2d_bf16(&tc, a.out, a.N, a.M, C::CW, 32)) return SAL_ECUDA;
   }
+  // bounds-checked build: the buffers this launch may touch (after the last early return)
+  ck_declare(A, a.M * a.K * 2, false);
+  ck_declare(W, static_cast<int64_t>(a.n_valid) * a.K * 2, false);
+  ck_declare(a.bias, static_cast<int64_t>(a.n_valid) * 2, false);
+  if constexpr (C::QKV) {
+    ck_declare(a.q, a.M * kWidth * 2, true);
+    ck_declare(a.k, a.M * kWidth * 2, true);
+    ck_declare(a.v, a.M * kWidth * 2, true);
+    ck_declare(a.qn_g, kHeadDim * 2, false);
+    ck_declare(a.kn_g, kHeadDim * 2, false);
+    ck_declare(a.rope_cs, a.rope_rows * 2 * 64 * 4, false);
+  } else {
+    ck_declare(a.out, a.M * a.N * (C::F32_OUT ? 4 : 2), true);
+  }
   if constexpr (PAIR) {
     // one cluster of two CTAs per pair of SMs, walking 256-row work units
     const int units = static_cast<int>((a.M + 2 * C::BM - 1) / (2 * C::BM)) * (a.N / BN) * a.splits;
@@ -743,20 +757,6 @@ sal_status gemm_launch(int epilogue, const void* A, int64_t M, int K, const void
       a.splits *= 2;
   }
   const bool pair = use_pair(M, N, BN, a.splits, is_qkv);
-  ck_declare(A, M * K * 2, false);
-  ck_declare(W, static_cast<int64_t>(n_valid) * K * 2, false);
-  ck_declare(bias, static_cast<int64_t>(n_valid) * 2, false);
-  if (is_qkv) {
-    ck_declare(a.q, M * kWidth * 2, true);
-    ck_declare(a.k, M * kWidth * 2, true);
-    ck_declare(a.v, M * kWidth * 2, true);
-    ck_declare(a.qn_g, kHeadDim * 2, false);
-    ck_declare(a.kn_g, kHeadDim * 2, false);
-    ck_declare(a.rope_cs, a.rope_rows * 2 * 64 * 4, false);
-  } else {
-    const bool f32 = epilogue == SAL_EPI_STORE_F32 || epilogue == SAL_EPI_RESID_F32;
-    ck_declare(out, M * N * (f32 ? 4 : 2), true);
-  }
   switch (epilogue) {
     case SAL_EPI_STORE_F32: return launch_epi<SAL_EPI_STORE_F32>(BN, pair, a, A, W, s);
     case SAL_EPI_STORE_BF16: return launch_epi<SAL_EPI_STORE_BF16>(BN, pair, a, A, W, s);

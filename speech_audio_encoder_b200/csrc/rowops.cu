@@ -281,6 +281,7 @@ sal_status layernorm_launch(const float* x, int64_t rows, const void* g, const v
   const auto gg = static_cast<const __nv_bfloat16*>(g);
   const auto bb = static_cast<const __nv_bfloat16*>(b);
   const auto yy = static_cast<__nv_bfloat16*>(y);
+  if (width != kWidth && width != 1024) return SAL_ESHAPE;
   ck_declare(x, rows * width * 4, false);
   ck_declare(g, width * 2, false);
   ck_declare(b, width * 2, false);
