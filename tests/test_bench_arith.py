@@ -51,3 +51,27 @@ def test_serving_window_work():
     assert pairs == sum(n * n for n in lens)
     assert bench.layer_work(T) == (T, T * T)
     assert bench.kernel_flops("attention", 1, T, window=(500, 50)) == 5120 * pairs
+
+
+def test_traffic_follows_the_source_hash(tmp_path, monkeypatch):
+    """The bench reports a stored DRAM figure only for the workload it was captured on and
+    only while the kernel's source hashes as it did then."""
+    import hashlib
+    import json
+    import os
+
+    src = tmp_path / "kernel.cu"
+    src.write_text("// v1\n")
+    (tmp_path / "profiles").mkdir()
+    rec = {"attention": {"workload": "rec_1h", "dram_bytes_per_launch": 123, "source": "kernel.cu",
+                         "sha256_16": hashlib.sha256(b"// v1\n").hexdigest()[:16]}}
+    (tmp_path / "profiles" / "roofline_traffic.json").write_text(json.dumps(rec))
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    assert bench._traffic("attention", "rec_1h") == 123
+    assert bench._traffic("attention", "rec_10min") is None  # another workload
+    assert bench._traffic("qkv", "rec_1h") is None  # no record
+    src.write_text("// v2\n")
+    assert bench._traffic("attention", "rec_1h") is None  # the kernel changed since the capture
+    os.remove(tmp_path / "profiles" / "roofline_traffic.json")
+    assert bench._traffic("attention", "rec_1h") is None
+
